@@ -1,0 +1,331 @@
+// api.cu -- the C ABI entry points declared in include/rattn.h: host-side
+// argument validation (nothing is launched on a bad argument), dispatch to
+// the kernels, the device error word and the TMA descriptor helper.
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "internal.h"
+
+namespace rattn {
+
+// Device-side error word written by kernels whose bounded waits gave up.
+__device__ int g_err_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultWaitNs = 4000000000ull;
+
+std::mutex g_mu;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_wait_ns[kMaxDevices] = {0};
+std::set<std::pair<const void*, int>> g_smem_done;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int elem_size(rattn_dtype dt) { return dt == RATTN_BF16 ? 2 : (dt == RATTN_F32 ? 4 : 0); }
+
+// Head-dimension support per dtype: bf16 runs on the tensor cores (D = 64 or
+// 128); fp32 runs the exact SIMT path (D a multiple of 4, at most 128).
+rattn_status check_attn_d(int D, rattn_dtype dt) {
+  if (D <= 0) return RATTN_ERR_INVALID_ARG;
+  if (dt == RATTN_BF16) return (D == 64 || D == 128) ? RATTN_OK : RATTN_ERR_UNSUPPORTED;
+  if (dt == RATTN_F32) return (D % 4 == 0 && D <= 128) ? RATTN_OK : RATTN_ERR_UNSUPPORTED;
+  return RATTN_ERR_INVALID_ARG;
+}
+
+int64_t chunks_of(int cp, rattn_layout layout) {
+  if (layout == RATTN_LAYOUT_HEAD_TAIL) return 2LL * cp;
+  if (layout == RATTN_LAYOUT_CONTIGUOUS) return cp;
+  return -1;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+rattn_status get_dev_ctx(DevCtx* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return RATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return RATTN_ERR_CUDA;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  out->err_word = g_err_ptr[dev];
+  out->wait_ns = g_wait_ns[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
+  return RATTN_OK;
+}
+
+rattn_status set_smem_attr(const void* kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto key = std::make_pair(kernel, dev);
+  if (g_smem_done.count(key)) return RATTN_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return RATTN_ERR_CUDA;
+  g_smem_done.insert(key);
+  return RATTN_OK;
+}
+
+rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,
+                            int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return RATTN_ERR_CUDA;
+  if (rows < 1) rows = 1;  // an empty segment is never read; the map still needs a non-zero extent
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(nseg), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2,
+                                 static_cast<cuuint64_t>(nseg) * rows * D * 2};
+  const cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(box_rows), 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RATTN_OK : RATTN_ERR_CUDA;
+}
+
+}  // namespace rattn
+
+using namespace rattn;
+
+extern "C" {
+
+const char* rattn_status_string(rattn_status s) {
+  switch (s) {
+    case RATTN_OK: return "RATTN_OK";
+    case RATTN_ERR_INVALID_ARG: return "RATTN_ERR_INVALID_ARG";
+    case RATTN_ERR_UNSUPPORTED: return "RATTN_ERR_UNSUPPORTED";
+    case RATTN_ERR_CUDA: return "RATTN_ERR_CUDA";
+    case RATTN_ERR_TIMEOUT: return "RATTN_ERR_TIMEOUT";
+  }
+  return "RATTN_ERR_UNKNOWN";
+}
+
+int64_t cp_layout_padded_len(int64_t L, int cp_size, rattn_layout layout) {
+  if (L < 0 || cp_size < 1) return -1;
+  const int64_t n = chunks_of(cp_size, layout);
+  if (n < 1) return -1;
+  if (L > INT64_MAX - n) return -1;
+  return (L + n - 1) / n * n;
+}
+
+rattn_status cp_layout_permute(const void* x, void* y, int32_t* pos, int B, int H, int64_t L, int64_t Lp, int D,
+                               rattn_dtype dtype, int cp_size, rattn_layout layout, void* stream) {
+  const int es = elem_size(dtype);
+  if (!es || B < 1 || H < 1 || D < 1 || L < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1)
+    return RATTN_ERR_INVALID_ARG;
+  if (Lp != cp_layout_padded_len(L, cp_size, layout)) return RATTN_ERR_INVALID_ARG;
+  if (Lp > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(D) * es) % 16) return RATTN_ERR_UNSUPPORTED;
+  if (Lp == 0) return RATTN_OK;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16) || (pos && !aligned(pos, 4))) return RATTN_ERR_INVALID_ARG;
+  return launch_permute(x, y, pos, B * H, L, Lp, D * es, cp_size, layout, static_cast<cudaStream_t>(stream));
+}
+
+rattn_status cp_layout_unpermute(const void* y, void* x, int B, int H, int64_t L, int64_t Lp, int D,
+                                 rattn_dtype dtype, int cp_size, rattn_layout layout, void* stream) {
+  const int es = elem_size(dtype);
+  if (!es || B < 1 || H < 1 || D < 1 || L < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1)
+    return RATTN_ERR_INVALID_ARG;
+  if (Lp != cp_layout_padded_len(L, cp_size, layout)) return RATTN_ERR_INVALID_ARG;
+  if (Lp > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if ((static_cast<int64_t>(D) * es) % 16) return RATTN_ERR_UNSUPPORTED;
+  if (L == 0) return RATTN_OK;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return RATTN_ERR_INVALID_ARG;
+  return launch_unpermute(y, x, B * H, L, Lp, D * es, cp_size, layout, static_cast<cudaStream_t>(stream));
+}
+
+rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v, const int32_t* q_pos,
+                               const int32_t* kv_pos, int B, int H, int64_t Lq, int64_t Lk, int D,
+                               rattn_dtype dtype, float scale, int causal, int64_t kv_valid, float* o, float* lse,
+                               void* stream) {
+  if (B < 1 || H < 1 || Lq < 0 || Lk < 0 || (causal != 0 && causal != 1) || !(scale > 0.f && scale < INFINITY))
+    return RATTN_ERR_INVALID_ARG;
+  rattn_status st = check_attn_d(D, dtype);
+  if (st != RATTN_OK) return st;
+  if (Lq > INT32_MAX - 256 || Lk > INT32_MAX - 256) return RATTN_ERR_UNSUPPORTED;
+  if (Lq == 0) return RATTN_OK;
+  if (!q || !o || !lse || !aligned(q, 16) || !aligned(o, 16) || !aligned(lse, 4)) return RATTN_ERR_INVALID_ARG;
+  if (Lk > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return RATTN_ERR_INVALID_ARG;
+  if ((q_pos && !aligned(q_pos, 4)) || (kv_pos && !aligned(kv_pos, 4))) return RATTN_ERR_INVALID_ARG;
+  FwdArgs a;
+  a.q = q;
+  a.k = Lk > 0 ? k : q;
+  a.v = Lk > 0 ? v : q;
+  a.q_pos = q_pos;
+  a.kv_pos = kv_pos;
+  a.BH = B * H;
+  a.nseg = 1;
+  a.Lq_seg = Lq;
+  a.Lk_seg = Lk;
+  a.D = D;
+  a.dtype = dtype;
+  a.scale = scale;
+  a.causal = causal;
+  a.kv_valid = kv_valid;
+  a.o = o;
+  a.o_f32 = 1;
+  a.lse = lse;
+  a.stream = static_cast<cudaStream_t>(stream);
+  if (dtype == RATTN_BF16) {
+    DevCtx ctx;
+    if ((st = get_dev_ctx(&ctx)) != RATTN_OK) return st;
+    return launch_fwd_sm100(a, ctx);
+  }
+  return launch_fwd_simt(a);
+}
+
+rattn_status rattn_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, int B, int H,
+                         int64_t Lq, int D, void* stream) {
+  if (B < 1 || H < 1 || Lq < 0 || D < 4 || D % 4) return RATTN_ERR_INVALID_ARG;
+  if (Lq == 0) return RATTN_OK;
+  if (!o_acc || !lse_acc || !o_blk || !lse_blk || !aligned(o_acc, 16) || !aligned(o_blk, 16) ||
+      !aligned(lse_acc, 4) || !aligned(lse_blk, 4))
+    return RATTN_ERR_INVALID_ARG;
+  return launch_merge(o_acc, lse_acc, o_blk, lse_blk, static_cast<int64_t>(B) * H * Lq, D,
+                      static_cast<cudaStream_t>(stream));
+}
+
+static rattn_status check_ring(const void* q, const void* k, const void* v, const int32_t* pos, int B, int H,
+                               int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout, int causal,
+                               float scale) {
+  if (B < 1 || H < 1 || Lp < 0 || cp_size < 1 || (causal != 0 && causal != 1) || !(scale > 0.f && scale < INFINITY))
+    return RATTN_ERR_INVALID_ARG;
+  const int64_t n = chunks_of(cp_size, layout);
+  if (n < 1 || Lp % n) return RATTN_ERR_INVALID_ARG;
+  rattn_status st = check_attn_d(D, dtype);
+  if (st != RATTN_OK) return st;
+  if (cp_size > 64) return RATTN_ERR_UNSUPPORTED;
+  if (Lp > INT32_MAX - 256) return RATTN_ERR_UNSUPPORTED;
+  if (Lp == 0) return RATTN_OK;
+  if (!q || !k || !v || !pos || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(pos, 4))
+    return RATTN_ERR_INVALID_ARG;
+  return RATTN_OK;
+}
+
+rattn_status rattn_ring_fwd(const void* q, const void* k, const void* v, const int32_t* pos, int B, int H,
+                            int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout, int causal,
+                            float scale, int64_t L_valid, void* o, float* lse, void* stream) {
+  rattn_status st = check_ring(q, k, v, pos, B, H, Lp, D, dtype, cp_size, layout, causal, scale);
+  if (st != RATTN_OK || Lp == 0) return st;
+  if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4)) return RATTN_ERR_INVALID_ARG;
+  FwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q_pos = pos;
+  a.kv_pos = pos;
+  a.BH = B * H;
+  a.nseg = cp_size;
+  a.Lq_seg = Lp / cp_size;
+  a.Lk_seg = Lp / cp_size;
+  a.D = D;
+  a.dtype = dtype;
+  a.scale = scale;
+  a.causal = causal;
+  a.kv_valid = L_valid;
+  a.o = o;
+  a.o_f32 = dtype == RATTN_F32;
+  a.lse = lse;
+  a.stream = static_cast<cudaStream_t>(stream);
+  if (dtype == RATTN_BF16) {
+    DevCtx ctx;
+    if ((st = get_dev_ctx(&ctx)) != RATTN_OK) return st;
+    return launch_fwd_sm100(a, ctx);
+  }
+  return launch_fwd_simt(a);
+}
+
+size_t rattn_ring_bwd_workspace_size(int B, int H, int64_t Lp, int D) {
+  if (B < 1 || H < 1 || Lp < 0 || D < 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * static_cast<size_t>(Lp);
+  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+}
+
+rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                            const float* lse, const int32_t* pos, int B, int H, int64_t Lp, int D,
+                            rattn_dtype dtype, int cp_size, rattn_layout layout, int causal, float scale,
+                            int64_t L_valid, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  rattn_status st = check_ring(q, k, v, pos, B, H, Lp, D, dtype, cp_size, layout, causal, scale);
+  if (st != RATTN_OK || Lp == 0) return st;
+  if (!o || !dout || !lse || !dq || !dk || !dv || !workspace || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(lse, 4) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(workspace, 256))
+    return RATTN_ERR_INVALID_ARG;
+  const size_t need = rattn_ring_bwd_workspace_size(B, H, Lp, D);
+  if (workspace_bytes < need) return RATTN_ERR_INVALID_ARG;
+  const size_t rows = static_cast<size_t>(B) * H * static_cast<size_t>(Lp);
+  BwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  a.pos = pos;
+  a.BH = B * H;
+  a.nseg = cp_size;
+  a.Lseg = Lp / cp_size;
+  a.D = D;
+  a.dtype = dtype;
+  a.scale = scale;
+  a.causal = causal;
+  a.kv_valid = L_valid;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dq_acc = static_cast<float*>(workspace);
+  a.delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256(rows * D * sizeof(float)));
+  a.stream = static_cast<cudaStream_t>(stream);
+  if (dtype == RATTN_BF16) {
+    DevCtx ctx;
+    if ((st = get_dev_ctx(&ctx)) != RATTN_OK) return st;
+    return launch_bwd_sm100(a, ctx);
+  }
+  return launch_bwd_simt(a);
+}
+
+rattn_status rattn_get_device_error(int* site) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(int)) != cudaSuccess) return RATTN_ERR_CUDA;
+  if (site) *site = v;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return RATTN_ERR_CUDA;
+    return RATTN_ERR_TIMEOUT;
+  }
+  return RATTN_OK;
+}
+
+rattn_status rattn_set_wait_limit_ns(unsigned long long ns) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return RATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_wait_ns[dev] = ns;  // 0 restores the default
+  return RATTN_OK;
+}
+
+}  // extern "C"

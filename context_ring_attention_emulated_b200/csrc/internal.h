@@ -1,0 +1,105 @@
+// internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/rattn.h"
+
+namespace rattn {
+
+// Per-device context every launch carries: the device-side error word and the
+// bounded-wait limit.
+struct DevCtx {
+  int* err_word;
+  unsigned long long wait_ns;
+};
+rattn_status get_dev_ctx(DevCtx* out);
+
+// Wait sites recorded in the error word.
+enum WaitSite : int {
+  SITE_FWD_LOAD = 1,
+  SITE_FWD_MMA = 2,
+  SITE_FWD_SOFTMAX = 3,
+  SITE_FWD_EPILOGUE = 4,
+  SITE_BWD_LOAD = 5,
+  SITE_BWD_MMA = 6,
+  SITE_BWD_COMPUTE = 7,
+  SITE_BWD_EPILOGUE = 8,
+  SITE_DRAIN = 9,
+};
+
+// Fixed limit for the teardown drains (copies and MMAs already in flight
+// always finish on their own; this only bounds a broken device).
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+
+// 4-D bf16 tensor map over [outer][nseg][rows][D] with a (64 x box_rows) box
+// and 128-byte swizzle; rows past `rows` read as zero.
+rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,
+                            int box_rows);
+
+// Sets the max dynamic shared memory attribute of a kernel once per device.
+rattn_status set_smem_attr(const void* kernel, int bytes);
+
+// Attention forward over segments: q viewed as [BH][nseg][Lq_seg][D], k/v as
+// [BH][nseg][Lk_seg][D]; query segment r attends key segments (r - t) mod nseg
+// for t = 0..nseg-1 (nseg = 1 for a single partial attention).
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* q_pos;   // [nseg*Lq_seg] or NULL (row index)
+  const int32_t* kv_pos;  // [nseg*Lk_seg] or NULL (row index)
+  int BH;
+  int nseg;
+  int64_t Lq_seg;
+  int64_t Lk_seg;
+  int D;
+  rattn_dtype dtype;
+  float scale;
+  int causal;
+  int64_t kv_valid;
+  void* o;        // [BH][nseg*Lq_seg][D]
+  int o_f32;      // 1: fp32 output, 0: output in `dtype`
+  float* lse;     // [BH][nseg*Lq_seg]
+  cudaStream_t stream;
+};
+rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx);
+rattn_status launch_fwd_simt(const FwdArgs& a);
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  const int32_t* pos;  // [nseg*Lseg]
+  int BH;
+  int nseg;
+  int64_t Lseg;
+  int D;
+  rattn_dtype dtype;
+  float scale;
+  int causal;
+  int64_t kv_valid;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dq_acc;  // workspace [BH][nseg*Lseg][D] fp32
+  float* delta;   // workspace [BH][nseg*Lseg] fp32
+  cudaStream_t stream;
+};
+rattn_status launch_bwd_sm100(const BwdArgs& a, const DevCtx& ctx);
+rattn_status launch_bwd_simt(const BwdArgs& a);
+
+rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int row_bytes,
+                            int cp, int layout, cudaStream_t stream);
+rattn_status launch_unpermute(const void* y, void* x, int BH, int64_t L, int64_t Lp, int row_bytes, int cp,
+                              int layout, cudaStream_t stream);
+rattn_status launch_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, int64_t rows,
+                          int D, cudaStream_t stream);
+
+}  // namespace rattn

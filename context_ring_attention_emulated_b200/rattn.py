@@ -1,0 +1,217 @@
+"""Python binding of librattn.so (the C ABI in include/rattn.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. Torch supplies device memory and the current stream. The library
+must be built (``python -m context_ring_attention_emulated_b200.build``);
+importing this module without it raises, and nothing here falls back to a CPU
+or PyTorch implementation.
+
+Functions keep the C names. Each takes tensors and infers B, H, L, D from
+their shapes; outputs are allocated with torch when not supplied.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+F32, BF16 = 0, 1
+LAYOUT_CONTIGUOUS, LAYOUT_HEAD_TAIL = 0, 1
+
+# (name, restype, argtypes) of every symbol include/rattn.h declares.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+SIGNATURES = [
+    ("rattn_status_string", ctypes.c_char_p, [_I]),
+    ("cp_layout_padded_len", _I64, [_I64, _I, _I]),
+    ("cp_layout_permute", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
+    ("cp_layout_unpermute", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
+    ("rattn_partial_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I, _I, _F, _I, _I64, _P, _P, _P]),
+    ("rattn_merge", _I, [_P, _P, _P, _P, _I, _I, _I64, _I, _P]),
+    ("rattn_ring_fwd", _I, [_P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64, _P, _P, _P]),
+    ("rattn_ring_bwd_workspace_size", ctypes.c_size_t, [_I, _I, _I64, _I]),
+    ("rattn_ring_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
+                            _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("rattn_get_device_error", _I, [ctypes.POINTER(_I)]),
+    ("rattn_set_wait_limit_ns", _I, [ctypes.c_ulonglong]),
+]
+
+
+class RattnError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {status_string(code)} ({code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m context_ring_attention_emulated_b200.build` (no fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, res, args in SIGNATURES:
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(code):
+    return lib.rattn_status_string(int(code)).decode()
+
+
+def _check(fn, code):
+    if code != OK:
+        raise RattnError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def cp_layout_padded_len(L, cp_size, layout=LAYOUT_HEAD_TAIL):
+    return int(lib.cp_layout_padded_len(int(L), int(cp_size), int(layout)))
+
+
+def cp_layout_permute(x, cp_size, layout=LAYOUT_HEAD_TAIL, y=None, pos=None, stream=None):
+    """x [B,H,L,D] -> (y [B,H,Lp,D] rank-major, pos int32 [Lp])."""
+    _need_cuda(x)
+    B, H, L, D = x.shape
+    Lp = cp_layout_padded_len(L, cp_size, layout)
+    if y is None:
+        y = torch.empty(B, H, Lp, D, dtype=x.dtype, device=x.device)
+    if pos is None:
+        pos = torch.empty(Lp, dtype=torch.int32, device=x.device)
+    _need_cuda(y, pos)
+    _check("cp_layout_permute", lib.cp_layout_permute(_ptr(x), _ptr(y), _ptr(pos), B, H, L, Lp, D,
+                                                       _dtype_code(x), cp_size, layout, _stream(stream)))
+    return y, pos
+
+
+def cp_layout_unpermute(y, L, cp_size, layout=LAYOUT_HEAD_TAIL, x=None, stream=None):
+    """y [B,H,Lp,D] rank-major -> x [B,H,L,D] global order."""
+    _need_cuda(y)
+    B, H, Lp, D = y.shape
+    if x is None:
+        x = torch.empty(B, H, L, D, dtype=y.dtype, device=y.device)
+    _need_cuda(x)
+    _check("cp_layout_unpermute", lib.cp_layout_unpermute(_ptr(y), _ptr(x), B, H, L, Lp, D, _dtype_code(y),
+                                                           cp_size, layout, _stream(stream)))
+    return x
+
+
+def rattn_partial_fwd(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True, kv_valid=2**62,
+                      o=None, lse=None, stream=None):
+    """One partial attention: returns (O fp32 [B,H,Lq,D], LSE fp32 [B,H,Lq])."""
+    _need_cuda(q, k, v, q_pos, kv_pos)
+    B, H, Lq, D = q.shape
+    Lk = k.shape[2]
+    scale = D ** -0.5 if scale is None else scale
+    if o is None:
+        o = torch.empty(B, H, Lq, D, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device)
+    _check("rattn_partial_fwd", lib.rattn_partial_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(q_pos), _ptr(kv_pos), B, H,
+                                                       Lq, Lk, D, _dtype_code(q), float(scale), int(causal),
+                                                       int(kv_valid), _ptr(o), _ptr(lse), _stream(stream)))
+    return o, lse
+
+
+def rattn_merge(o_acc, lse_acc, o_blk, lse_blk, stream=None):
+    """In-place online-softmax fold of (o_blk, lse_blk) into (o_acc, lse_acc)."""
+    _need_cuda(o_acc, lse_acc, o_blk, lse_blk)
+    B, H, Lq, D = o_acc.shape
+    _check("rattn_merge", lib.rattn_merge(_ptr(o_acc), _ptr(lse_acc), _ptr(o_blk), _ptr(lse_blk), B, H, Lq, D,
+                                           _stream(stream)))
+    return o_acc, lse_acc
+
+
+def rattn_ring_fwd(q, k, v, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None, L_valid=None,
+                   o=None, lse=None, stream=None):
+    """Emulated ring forward on rank-major q/k/v [B,H,Lp,D]: returns (O, LSE)."""
+    _need_cuda(q, k, v, pos)
+    B, H, Lp, D = q.shape
+    scale = D ** -0.5 if scale is None else scale
+    L_valid = Lp if L_valid is None else L_valid
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, H, Lp, dtype=torch.float32, device=q.device)
+    _check("rattn_ring_fwd", lib.rattn_ring_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(pos), B, H, Lp, D, _dtype_code(q),
+                                                 cp_size, layout, int(causal), float(scale), int(L_valid), _ptr(o),
+                                                 _ptr(lse), _stream(stream)))
+    return o, lse
+
+
+def rattn_ring_bwd_workspace_size(B, H, Lp, D):
+    return int(lib.rattn_ring_bwd_workspace_size(B, H, Lp, D))
+
+
+def rattn_ring_bwd(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None,
+                   L_valid=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of the ring forward (rank-major): returns (dQ, dK, dV)."""
+    _need_cuda(q, k, v, o, dout, lse, pos)
+    B, H, Lp, D = q.shape
+    scale = D ** -0.5 if scale is None else scale
+    L_valid = Lp if L_valid is None else L_valid
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = rattn_ring_bwd_workspace_size(B, H, Lp, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check("rattn_ring_bwd", lib.rattn_ring_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                                 _ptr(pos), B, H, Lp, D, _dtype_code(q), cp_size, layout,
+                                                 int(causal), float(scale), int(L_valid), _ptr(dq), _ptr(dk),
+                                                 _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def rattn_get_device_error():
+    site = ctypes.c_int(0)
+    code = lib.rattn_get_device_error(ctypes.byref(site))
+    return code, site.value
+
+
+def rattn_set_wait_limit_ns(ns):
+    _check("rattn_set_wait_limit_ns", lib.rattn_set_wait_limit_ns(int(ns)))
+
+
+# ------------------------------------------------------------- convenience
+
+def ring_attention(q, k, v, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None, stream=None):
+    """Global-order q/k/v [B,H,L,D] -> (O [B,H,L,D] global order, LSE fp32
+    [B,H,Lp] rank-major, pos int32 [Lp]): permute to the CP layout, run the
+    emulated ring, unpermute O."""
+    L = q.shape[2]
+    qp, pos = cp_layout_permute(q, cp_size, layout, stream=stream)
+    kp, _ = cp_layout_permute(k, cp_size, layout, stream=stream)
+    vp, _ = cp_layout_permute(v, cp_size, layout, stream=stream)
+    o, lse = rattn_ring_fwd(qp, kp, vp, pos, cp_size, layout, causal, scale, L_valid=L, stream=stream)
+    return cp_layout_unpermute(o, L, cp_size, layout, stream=stream), lse, pos

@@ -1,0 +1,173 @@
+/*
+ * rattn.h -- C ABI of the B200 (sm_100a) ring-attention library with
+ * context-parallel (CP) ranks emulated on one GPU.
+ *
+ * Sources, cited by page title and section:
+ *   [CP-glossary]  Ultralytics glossary "Context Parallelism", section
+ *                  "How context parallelism works" (ring attention: each device
+ *                  computes a partial attention on the KV block it holds, passes
+ *                  the block to the next device and repeats until the whole
+ *                  sequence has been seen; exact up to ordinary rounding) and
+ *                  "Practical use and trade-offs" (the 2-rank causal SDPA example
+ *                  with sequence dimension 2 and a backward pass).
+ *   [Megatron-CP]  Blog "Context Parallelism v.s. Sequence Parallelism
+ *                  (Megatron-LM)", section "Symmetric chunk assignment" (2*cp
+ *                  chunks, rank r holds chunks r and 2*cp-1-r, global position
+ *                  ids follow the pairing, pad to a multiple of 2*cp).
+ *   [Ring-page]    aiunderstanding.org "Sequence parallelism and ring attention",
+ *                  sections "Deep dive" and "Technical insight" (local Q fixed,
+ *                  K/V blocks arrive hop by hop, online softmax with a running
+ *                  max and running normaliser, transfer overlapped with math).
+ *
+ * Conventions shared by every call:
+ *   - All tensors are dense, contiguous, row-major [B, H, L, D] (sequence on
+ *     dimension 2, as in [CP-glossary]'s example), in device memory owned by
+ *     the caller. The library never allocates device memory; scratch space is
+ *     passed in by the caller (rattn_ring_bwd's workspace).
+ *   - Data pointers must be 16-byte aligned. Position arrays are int32.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). Arguments are validated on the host first;
+ *     a violation returns RATTN_ERR_INVALID_ARG or RATTN_ERR_UNSUPPORTED and
+ *     launches nothing. A failed launch returns RATTN_ERR_CUDA. No C++
+ *     exception crosses this boundary.
+ *   - dtype RATTN_BF16 runs on the tcgen05 tensor cores (bf16 operands, fp32
+ *     accumulation, D in {64, 128}); RATTN_F32 runs an exact-fp32 SIMT path
+ *     (D a multiple of 4, at most 128).
+ *   - Position arrays must be non-decreasing within every rank's slice (ring
+ *     calls) or over the whole array (rattn_partial_fwd). The layouts produced
+ *     by cp_layout_permute satisfy this; kernels use it to skip and classify
+ *     tiles. A key is visible to a query iff (!causal || kv_pos <= q_pos) and
+ *     kv_pos < kv_valid (L_valid in ring calls).
+ *   - scale (applied to q.k before the softmax) must be finite and > 0.
+ *   - LSE is the natural-log softmax normaliser log(sum_j exp(scale*q.k_j))
+ *     over visible keys, fp32; a query with no visible key gets LSE = -inf and
+ *     O = 0.
+ *   - Device-side waits are bounded. If one gives up, the kernel records an
+ *     error word and returns early; rattn_get_device_error() reports it as
+ *     RATTN_ERR_TIMEOUT.
+ */
+#ifndef RATTN_H_
+#define RATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RATTN_OK = 0,
+  RATTN_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or enum       */
+  RATTN_ERR_UNSUPPORTED = 2,   /* valid request this build does not handle   */
+  RATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
+  RATTN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up         */
+} rattn_status;
+
+typedef enum { RATTN_F32 = 0, RATTN_BF16 = 1 } rattn_dtype;
+
+/* [Megatron-CP]: CONTIGUOUS is the naive split (rank r holds the r-th of
+ * cp_size equal pieces); HEAD_TAIL is the symmetric assignment (rank r holds
+ * chunk r then chunk 2*cp_size-1-r of 2*cp_size equal chunks). */
+typedef enum { RATTN_LAYOUT_CONTIGUOUS = 0, RATTN_LAYOUT_HEAD_TAIL = 1 } rattn_layout;
+
+/* Human-readable name of a status code. Never NULL. */
+const char* rattn_status_string(rattn_status s);
+
+/* [Megatron-CP] padding rule: the smallest Lp >= L that is a multiple of
+ * 2*cp_size (HEAD_TAIL) or cp_size (CONTIGUOUS). Returns -1 on bad arguments
+ * (L < 0, cp_size < 1, unknown layout). Host only; no device work. */
+int64_t cp_layout_padded_len(int64_t L, int cp_size, rattn_layout layout);
+
+/* [Megatron-CP] layout permute: x [B,H,L,D] (global order) -> y [B,H,Lp,D]
+ * in rank-major order (rank r's slice is rows [r*Lp/cp, (r+1)*Lp/cp)), pad
+ * rows (global index >= L) zero-filled. If pos is non-NULL it receives the
+ * global position id of every slot, int32 [Lp], shared by all (b, h); pad
+ * slots carry L, L+1, ... Lp must equal cp_layout_padded_len(L, cp, layout).
+ * Bit-exact copy. x and y must not overlap. */
+rattn_status cp_layout_permute(const void* x, void* y, int32_t* pos,
+                               int B, int H, int64_t L, int64_t Lp, int D,
+                               rattn_dtype dtype, int cp_size, rattn_layout layout,
+                               void* stream);
+
+/* Inverse of cp_layout_permute: y [B,H,Lp,D] -> x [B,H,L,D]; pad rows are
+ * dropped. Bit-exact copy. x and y must not overlap. */
+rattn_status cp_layout_unpermute(const void* y, void* x,
+                                 int B, int H, int64_t L, int64_t Lp, int D,
+                                 rattn_dtype dtype, int cp_size, rattn_layout layout,
+                                 void* stream);
+
+/* [CP-glossary], [Ring-page]: one partial attention of local queries against
+ * one K/V block. q [B,H,Lq,D], k and v [B,H,Lk,D] in `dtype`; q_pos int32
+ * [Lq] and kv_pos int32 [Lk] (either may be NULL, meaning 0,1,2,...);
+ * keys with kv_pos >= kv_valid are masked (pass INT64_MAX for none).
+ * Outputs (fp32, caller-owned): o [B,H,Lq,D] = softmax-weighted average of
+ * the visible V rows, lse [B,H,Lq]. Tiles the causal relation fully masks
+ * are skipped. */
+rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v,
+                               const int32_t* q_pos, const int32_t* kv_pos,
+                               int B, int H, int64_t Lq, int64_t Lk, int D,
+                               rattn_dtype dtype, float scale, int causal, int64_t kv_valid,
+                               float* o, float* lse, void* stream);
+
+/* [Ring-page] "Technical insight": online-softmax fold of a block result into
+ * an accumulator, in place, fp32:
+ *   LSE' = m + log(exp(LSE_acc - m) + exp(LSE_blk - m)),  m = max(LSE_acc, LSE_blk)
+ *   O'   = exp(LSE_acc - LSE') O_acc + exp(LSE_blk - LSE') O_blk
+ * o_acc, o_blk [B,H,Lq,D]; lse_acc, lse_blk [B,H,Lq]. A side whose LSE is
+ * -inf contributes nothing; both -inf leaves LSE = -inf, O = 0. */
+rattn_status rattn_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk,
+                         int B, int H, int64_t Lq, int D, void* stream);
+
+/* [CP-glossary], [Ring-page]: the whole emulated ring forward. q, k, v
+ * [B,H,Lp,D] in rank-major order (as cp_layout_permute writes them) with
+ * positions pos int32 [Lp]. Every emulated rank r keeps its Q slice fixed and,
+ * for hops t = 0..cp_size-1, attends the K/V slice of rank s = (r - t) mod
+ * cp_size (blocks move to the next rank each hop), folding each block into a
+ * running max / normaliser in ring order; the next block's K/V loads overlap
+ * the current block's math. Keys with pos >= L_valid (padding) are masked.
+ * Outputs: o [B,H,Lp,D] in `dtype` (round-to-nearest-even for bf16), lse
+ * fp32 [B,H,Lp]. Lp must be a multiple of cp_size (of 2*cp_size for
+ * HEAD_TAIL); 1 <= cp_size <= 64. */
+rattn_status rattn_ring_fwd(const void* q, const void* k, const void* v, const int32_t* pos,
+                            int B, int H, int64_t Lp, int D, rattn_dtype dtype,
+                            int cp_size, rattn_layout layout, int causal, float scale,
+                            int64_t L_valid, void* o, float* lse, void* stream);
+
+/* Bytes of scratch rattn_ring_bwd needs for these sizes (fp32 dQ accumulator
+ * [B,H,Lp,D] plus the per-row dot(dO, O) vector [B,H,Lp], each 256-byte
+ * aligned). Host only. Returns 0 on bad arguments. */
+size_t rattn_ring_bwd_workspace_size(int B, int H, int64_t Lp, int D);
+
+/* [CP-glossary] "Practical use and trade-offs" (`.backward()` through the CP
+ * attention): gradients of the ring forward, recomputing P from the saved fp32
+ * LSE. Inputs as rattn_ring_fwd plus o (forward output, `dtype`), dout (dL/dO,
+ * `dtype`) and lse (fp32). Outputs dq, dk, dv [B,H,Lp,D] in `dtype`. The
+ * caller passes `workspace` (device, 256-byte aligned, at least
+ * rattn_ring_bwd_workspace_size bytes); its contents on entry are ignored and
+ * on return undefined. Calls sharing a workspace must not overlap. */
+rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const void* o,
+                            const void* dout, const float* lse, const int32_t* pos,
+                            int B, int H, int64_t Lp, int D, rattn_dtype dtype,
+                            int cp_size, rattn_layout layout, int causal, float scale,
+                            int64_t L_valid, void* dq, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device-side error word of the current device
+ * (synchronises the device). Returns RATTN_OK if no kernel recorded an
+ * error, RATTN_ERR_TIMEOUT if a bounded wait gave up (*site, if non-NULL,
+ * receives the recorded wait site), RATTN_ERR_CUDA if the read failed. */
+rattn_status rattn_get_device_error(int* site);
+
+/* Test hook: the per-wait time limit in nanoseconds used by subsequent
+ * launches on the current device (default 4e9; 0 restores the default). A
+ * tiny limit makes waits give
+ * up at once; kernels then drain their in-flight copies and MMAs (with a fixed
+ * limit) and return without touching memory they do not own. */
+rattn_status rattn_set_wait_limit_ns(unsigned long long ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RATTN_H_ */

@@ -68,9 +68,10 @@ def attention(q, k, v, scale, causal, q_pos=None, kv_pos=None, kv_valid=None, ro
     q_pos = _default_pos(Lq) if q_pos is None else np.asarray(q_pos, dtype=np.int64)
     kv_pos = _default_pos(Lk) if kv_pos is None else np.asarray(kv_pos, dtype=np.int64)
     lead = q.shape[:-2]
-    qf = q.reshape(-1, Lq, D)
-    kf = k.reshape(-1, Lk, D)
-    vf = v.reshape(-1, Lk, v.shape[-1])
+    nb = int(np.prod(lead, dtype=np.int64))
+    qf = q.reshape(nb, Lq, D)
+    kf = k.reshape(nb, Lk, D)
+    vf = v.reshape(nb, Lk, v.shape[-1])
     o = np.zeros((qf.shape[0], Lq, vf.shape[-1]))
     lse = np.zeros((qf.shape[0], Lq))
     for b in range(qf.shape[0]):
@@ -167,8 +168,8 @@ def attention_bwd(q, k, v, do, scale, causal, q_pos=None, kv_pos=None, kv_valid=
     Lk = k.shape[-2]
     q_pos = _default_pos(Lq) if q_pos is None else np.asarray(q_pos, dtype=np.int64)
     kv_pos = _default_pos(Lk) if kv_pos is None else np.asarray(kv_pos, dtype=np.int64)
-    lead = q.shape[:-2]
-    qf, kf, vf, dof = (t.reshape(-1, t.shape[-2], t.shape[-1]) for t in (q, k, v, do))
+    nb = int(np.prod(q.shape[:-2], dtype=np.int64))
+    qf, kf, vf, dof = (t.reshape(nb, t.shape[-2], t.shape[-1]) for t in (q, k, v, do))
     dq = np.zeros_like(qf)
     dk = np.zeros_like(kf)
     dv = np.zeros_like(vf)

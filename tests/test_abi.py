@@ -1,0 +1,125 @@
+"""CPU tests of the C-ABI library: it builds for sm_100a, loads, exports every
+symbol include/rattn.h declares, and rejects bad arguments on the host before
+any device work (no compute call runs here: this machine has no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.gpu_common import load_rattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rattn.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M)) - {"if", "defined"})
+
+
+@pytest.fixture(scope="module")
+def rattn():
+    return load_rattn()
+
+
+def test_every_declared_symbol_is_exported(rattn):
+    names = header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(rattn.lib, n), f"{n} declared in rattn.h but not exported"
+    assert sorted(n for n, _, _ in rattn.SIGNATURES) == names
+
+
+def test_status_strings(rattn):
+    for code, name in enumerate(["RATTN_OK", "RATTN_ERR_INVALID_ARG", "RATTN_ERR_UNSUPPORTED", "RATTN_ERR_CUDA",
+                                 "RATTN_ERR_TIMEOUT"]):
+        assert rattn.status_string(code) == name
+    assert rattn.status_string(99) == "RATTN_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("L,cp,layout,expect", [
+    (32000, 4, 1, 32000), (4096, 2, 1, 4096), (1048576, 8, 1, 1048576), (131072, 8, 0, 131072),
+    (10, 4, 1, 16), (10, 4, 0, 12), (0, 3, 1, 0), (1, 1, 1, 2), (1, 1, 0, 1),
+    (-1, 2, 1, -1), (10, 0, 1, -1), (10, 2, 7, -1)])
+def test_padded_len(rattn, L, cp, layout, expect):
+    assert rattn.lib.cp_layout_padded_len(L, cp, layout) == expect
+
+
+def test_padded_len_matches_oracle(rattn):
+    import oracle
+    for cp in range(1, 17):
+        for L in (0, 1, 5, 63, 64, 65, 1000):
+            for layout in (0, 1):
+                assert rattn.lib.cp_layout_padded_len(L, cp, layout) == oracle.padded_len(L, cp, layout)
+
+
+FAKE = 0x10000        # 16-byte aligned fake device address (never dereferenced)
+MIS = 0x10004         # misaligned
+
+
+def test_permute_rejects_bad_arguments(rattn):
+    L = rattn.lib
+    # Lp does not match the padding rule
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, 1, 1, 10, 12, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+    # bad sizes / enums
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, 0, 1, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, 1, 1, 16, 16, 64, 5, 4, 1, None) == rattn.ERR_INVALID_ARG
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, 1, 1, 16, 16, 64, 1, 0, 1, None) == rattn.ERR_INVALID_ARG
+    # null / misaligned pointers
+    assert L.cp_layout_permute(None, FAKE, FAKE, 1, 1, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+    assert L.cp_layout_permute(MIS, FAKE, FAKE, 1, 1, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+    # row not a multiple of 16 bytes
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, 1, 1, 16, 16, 3, 1, 4, 1, None) == rattn.ERR_UNSUPPORTED
+    # empty sequence is a no-op
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, 1, 1, 0, 0, 64, 1, 4, 1, None) == rattn.OK
+    assert L.cp_layout_unpermute(FAKE, FAKE, 1, 1, 10, 12, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+    assert L.cp_layout_unpermute(MIS, FAKE, 1, 1, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+
+
+def test_attention_calls_reject_bad_arguments(rattn):
+    L = rattn.lib
+    ring = lambda **kw: L.rattn_ring_fwd(kw.get("q", FAKE), FAKE, FAKE, kw.get("pos", FAKE), 1, 2,
+                                         kw.get("Lp", 256), kw.get("D", 64), kw.get("dt", 1), kw.get("cp", 2),
+                                         kw.get("layout", 1), kw.get("causal", 1), ctypes.c_float(0.125), 256,
+                                         kw.get("o", FAKE), FAKE, None)
+    assert ring(cp=0) == rattn.ERR_INVALID_ARG
+    assert ring(Lp=250) == rattn.ERR_INVALID_ARG          # not a multiple of 2*cp
+    assert ring(layout=3) == rattn.ERR_INVALID_ARG
+    assert ring(causal=2) == rattn.ERR_INVALID_ARG
+    assert ring(D=96) == rattn.ERR_UNSUPPORTED            # bf16 tensor-core path: D in {64, 128}
+    assert ring(D=132, dt=0) == rattn.ERR_UNSUPPORTED     # fp32 path: D <= 128, multiple of 4
+    assert ring(cp=65, Lp=130 * 2) == rattn.ERR_UNSUPPORTED
+    assert ring(q=MIS) == rattn.ERR_INVALID_ARG
+    assert ring(pos=None) == rattn.ERR_INVALID_ARG
+    assert ring(o=None) == rattn.ERR_INVALID_ARG
+    assert ring(Lp=0) == rattn.OK
+    part = lambda **kw: L.rattn_partial_fwd(kw.get("q", FAKE), FAKE, FAKE, None, None, 1, 1, kw.get("Lq", 8), 8,
+                                            kw.get("D", 64), 1, ctypes.c_float(kw.get("scale", 0.1)), 1, 1 << 40,
+                                            kw.get("o", FAKE), FAKE, None)
+    assert part(Lq=-1) == rattn.ERR_INVALID_ARG
+    assert part(scale=float("nan")) == rattn.ERR_INVALID_ARG
+    assert part(q=MIS) == rattn.ERR_INVALID_ARG
+    assert part(o=MIS) == rattn.ERR_INVALID_ARG
+    assert part(D=80) == rattn.ERR_UNSUPPORTED
+    assert part(Lq=0) == rattn.OK
+    assert L.rattn_merge(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 6, None) == rattn.ERR_INVALID_ARG
+    assert L.rattn_merge(MIS, FAKE, FAKE, FAKE, 1, 1, 4, 8, None) == rattn.ERR_INVALID_ARG
+    assert L.rattn_merge(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 8, None) == rattn.OK
+
+
+def test_bwd_rejects_bad_arguments_and_sizes_workspace(rattn):
+    L = rattn.lib
+    need = L.rattn_ring_bwd_workspace_size(1, 32, 32000, 128)
+    rows = 32 * 32000
+    assert need == ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    assert L.rattn_ring_bwd_workspace_size(0, 1, 1, 1) == 0
+
+    def bwd(ws=FAKE, ws_bytes=need, **kw):
+        return L.rattn_ring_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 32, 32000, 128, 1, 4, 1, 1,
+                                ctypes.c_float(0.088), 32000, FAKE, FAKE, kw.get("dv", FAKE), ws, ws_bytes, None)
+    assert bwd(ws_bytes=need - 1) == rattn.ERR_INVALID_ARG
+    assert bwd(ws=FAKE + 16) == rattn.ERR_INVALID_ARG   # workspace must be 256-byte aligned
+    assert bwd(ws=None) == rattn.ERR_INVALID_ARG
+    assert bwd(dv=None) == rattn.ERR_INVALID_ARG

@@ -1,0 +1,86 @@
+"""GPU parity of the ring backward (dQ, dK, dV from the saved LSE) against
+the oracle's textbook softmax-attention gradient, in fp64."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from context_ring_attention_emulated_b200.workloads import WORKLOADS, make_qkv, make_tensor
+from tests.gpu_common import check_grad, load_rattn, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rattn():
+    return load_rattn()
+
+
+def _run_bwd(rattn, q, k, v, do, cp, layout, causal):
+    """Permute, ring fwd, ring bwd, unpermute the gradients (global order)."""
+    L, D = q.shape[2], q.shape[3]
+    scale = D ** -0.5
+    qp, pos = rattn.cp_layout_permute(q, cp, layout)
+    kp, _ = rattn.cp_layout_permute(k, cp, layout)
+    vp, _ = rattn.cp_layout_permute(v, cp, layout)
+    dop, _ = rattn.cp_layout_permute(do, cp, layout)
+    o, lse = rattn.rattn_ring_fwd(qp, kp, vp, pos, cp, layout, causal, scale, L_valid=L)
+    dq, dk, dv = rattn.rattn_ring_bwd(qp, kp, vp, o, dop, lse, pos, cp, layout, causal, scale, L_valid=L)
+    out = [rattn.cp_layout_unpermute(t, L, cp, layout) for t in (dq, dk, dv)]
+    torch.cuda.synchronize()
+    return out
+
+
+BWD_CASES = [
+    # dtype, D, L, cp, layout, causal
+    (torch.float32, 64, 256, 2, 1, True),
+    (torch.float32, 64, 29, 3, 1, True),
+    (torch.float32, 32, 100, 4, 0, False),
+    (torch.bfloat16, 128, 1000, 4, 1, True),
+    (torch.bfloat16, 64, 4096, 2, 1, True),
+    (torch.bfloat16, 128, 29, 4, 1, True),
+    (torch.bfloat16, 128, 1000, 3, 0, False),
+    (torch.bfloat16, 64, 777, 1, 1, True),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+def test_ring_bwd_unit_grad(rattn, case):
+    dtype, D, L, cp, layout, causal = case
+    B, H = 1, 2
+    q, k, v = (make_tensor((B, H, L, D), dtype, "cuda", seed=s) for s in (31, 32, 33))
+    do = make_tensor((B, H, L, D), dtype, "cuda", seed=34)
+    dq, dk, dv = _run_bwd(rattn, q, k, v, do, cp, layout, causal)
+    ref = oracle.attention_bwd(to64(q), to64(k), to64(v), to64(do), D ** -0.5, causal)
+    for got, r in zip((dq, dk, dv), ref):
+        check_grad(got.float().cpu().numpy(), r)
+
+
+def test_ring_bwd_full_size_loss_grad(rattn):
+    """The 32k / cp=4 fwd+bwd workload with loss = mean(O.float()^2): dO is
+    derived from the oracle's O (2 O / N, rounded to bf16) and fed to both
+    sides. Two heads are checked in full against the oracle, plus an
+    unscaled dO ~ N(0, 1) run on the same heads."""
+    w = WORKLOADS["bf16_L32000_cp4_fwdbwd"]
+    q, k, v = make_qkv(w, "cuda", seed=0)
+    heads = [0, 17]
+    N = w.B * w.H * w.L * w.D
+    do = torch.zeros_like(q)
+    refs = {}
+    for h in heads:
+        qh, kh, vh = to64(q[0, h]), to64(k[0, h]), to64(v[0, h])
+        o_ref, _ = oracle.attention(qh, kh, vh, w.scale, True, row_block=1024)
+        do_h = torch.from_numpy(2.0 * o_ref / N).to(torch.bfloat16)
+        do[0, h] = do_h.cuda()
+        refs[h] = oracle.attention_bwd(qh, kh, vh, to64(do_h), w.scale, True, row_block=1024)
+    dq, dk, dv = _run_bwd(rattn, q, k, v, do, w.cp, w.layout, True)
+    for h in heads:
+        for got, r in zip((dq, dk, dv), refs[h]):
+            check_grad(got[0, h].float().cpu().numpy(), r)
+    do1 = make_tensor(q.shape, q.dtype, "cuda", seed=1)
+    dq, dk, dv = _run_bwd(rattn, q, k, v, do1, w.cp, w.layout, True)
+    for h in heads:
+        qh, kh, vh = to64(q[0, h]), to64(k[0, h]), to64(v[0, h])
+        ref = oracle.attention_bwd(qh, kh, vh, to64(do1[0, h]), w.scale, True, row_block=1024)
+        for got, r in zip((dq, dk, dv), ref):
+            check_grad(got[0, h].float().cpu().numpy(), r)

@@ -257,3 +257,12 @@ def test_pins_reject_planted_mistakes(mutant, monkeypatch):
     ob, lb = brute_attention(q, k, v, 0.7, True, pos, pos)
     ok = np.allclose(o, ob, atol=1e-12) and np.allclose(lse, lb, atol=1e-12)
     assert not ok, "a planted mistake passed the brute-force pin"
+
+
+def test_empty_key_block_sees_nothing():
+    q = np.ones((2, 3, 4, 5))
+    k = np.zeros((2, 3, 0, 5))
+    o, lse = oracle.attention(q, k, k, 0.5, False)
+    assert o.shape == (2, 3, 4, 5) and np.all(o == 0.0) and np.all(np.isneginf(lse))
+    dq, dk, dv = oracle.attention_bwd(q, k, k, q, 0.5, True)
+    assert np.all(dq == 0.0) and dk.shape == k.shape and dv.shape == k.shape
