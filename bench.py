@@ -1,0 +1,323 @@
+"""Benchmark: ring attention with emulated CP ranks on B200.
+
+One step = the whole hot path on one batch of seeded synthetic input:
+permute Q, K, V and dO to the head-tail layout, ring forward, unpermute O,
+ring backward (dQ, dK, dV from the saved LSE), unpermute the gradients.
+Default workload: the 32,000-token / cp=4 fwd+bwd configuration (B=1, H=32,
+D=128, bf16, causal). Metric: causal-adjusted TFLOP/s of fwd + bwd
+(fwd = 2*B*H*D*L^2, bwd = 2.5 x fwd).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the
+workload (the path has no cross-GPU exchange in this build); value is the
+work of all ranks over the max-over-ranks device time.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from context_ring_attention_emulated_b200.workloads import WORKLOADS, make_qkv, make_unit_grad  # noqa: E402
+
+METRIC = "ring-attn fwd/bwd TFLOP/s (causal FLOPs) on 1 B200; % of BF16 tensor peak"
+DEFAULT = "bf16_L32000_cp4_fwdbwd"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def step_flops(w):
+    fwd = w.causal_flops_fwd()
+    return fwd * (3.5 if w.bwd else 1.0), fwd
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n):
+    if n <= 1 and "RANK" not in os.environ:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", n))
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args, w, rank, world, local):
+    from context_ring_attention_emulated_b200 import rattn
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    q, k, v = make_qkv(w, dev, seed=0)
+    do = make_unit_grad(w, dev, seed=1)
+    L, cp, layout = w.L, w.cp, w.layout
+    B, H, D = w.B, w.H, w.D
+    Lp = rattn.cp_layout_padded_len(L, cp, layout)
+    pbuf = {n: torch.empty(B, H, Lp, D, dtype=q.dtype, device=dev) for n in ("q", "k", "v", "do", "o")}
+    pos = torch.empty(Lp, dtype=torch.int32, device=dev)
+    lse = torch.empty(B, H, Lp, dtype=torch.float32, device=dev)
+    grads_p = [torch.empty(B, H, Lp, D, dtype=q.dtype, device=dev) for _ in range(3)]
+    out = {n: torch.empty(B, H, L, D, dtype=q.dtype, device=dev) for n in ("o", "dq", "dk", "dv")}
+    ws = torch.empty(max(rattn.rattn_ring_bwd_workspace_size(B, H, Lp, D), 1), dtype=torch.uint8, device=dev)
+    fwd_ev, bwd_ev = [], []
+
+    def step(x, timed=False):
+        xq, xk, xv, xdo = x
+        rattn.cp_layout_permute(xq, cp, layout, y=pbuf["q"], pos=pos)
+        rattn.cp_layout_permute(xk, cp, layout, y=pbuf["k"], pos=pos)
+        rattn.cp_layout_permute(xv, cp, layout, y=pbuf["v"], pos=pos)
+        if timed:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        rattn.rattn_ring_fwd(pbuf["q"], pbuf["k"], pbuf["v"], pos, cp, layout, w.causal, w.scale, L_valid=L,
+                             o=pbuf["o"], lse=lse)
+        if timed:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(stream)
+            fwd_ev.append((e0, e1))
+        rattn.cp_layout_unpermute(pbuf["o"], L, cp, layout, x=out["o"])
+        if w.bwd:
+            rattn.cp_layout_permute(xdo, cp, layout, y=pbuf["do"], pos=pos)
+            if timed:
+                e2 = torch.cuda.Event(enable_timing=True)
+                e2.record(stream)
+            rattn.rattn_ring_bwd(pbuf["q"], pbuf["k"], pbuf["v"], pbuf["o"], pbuf["do"], lse, pos, cp, layout,
+                                 w.causal, w.scale, L_valid=L, dq=grads_p[0], dk=grads_p[1], dv=grads_p[2],
+                                 workspace=ws)
+            if timed:
+                e3 = torch.cuda.Event(enable_timing=True)
+                e3.record(stream)
+                bwd_ev.append((e2, e3))
+            for g, name in zip(grads_p, ("dq", "dk", "dv")):
+                rattn.cp_layout_unpermute(g, L, cp, layout, x=out[name])
+
+    launches_per_step = 3 + 1 + 1 + ((1 + 3 + 3) if w.bwd else 0)
+    x = (q, k, v, do)
+    for _ in range(args.warmup):
+        step(x)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(x, timed=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    err, site = rattn.rattn_get_device_error()
+    if err != rattn.OK:
+        raise RuntimeError(f"device-side wait timed out at site {site}")
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
+    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev) if bwd_ev else None
+
+    # End to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the step, D2H of its results (O, dQ, dK, dV).
+    host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in out.items()}
+    dev_in = [torch.empty_like(t) for t in (q, k, v, do)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in[:4 if w.bwd else 3])
+    d2h = sum(host_out[n].numel() * host_out[n].element_size() for n in (("o", "dq", "dk", "dv") if w.bwd else ("o",)))
+
+    def e2e_step():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        step(tuple(dev_in))
+        for n in (("o", "dq", "dk", "dv") if w.bwd else ("o",)):
+            host_out[n].copy_(out[n], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"ms": ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
+            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps}
+
+
+def cpu_sample_run(w, seconds_hint=True):
+    """The oracle as it stands on a bounded sample: one head, the first 8000
+    tokens (one emulated rank's worth), causal fwd + bwd, fp64 on the host."""
+    import numpy as np
+    import oracle
+    Ls = min(8000, w.L)
+    g = torch.Generator().manual_seed(0)
+    q, k, v, do = (torch.randn(Ls, w.D, generator=g).to(w.torch_dtype).double().numpy() for _ in range(4))
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, w.scale, w.causal, row_block=1000)
+    if w.bwd:
+        oracle.attention_bwd(q, k, v, do, w.scale, w.causal, row_block=1000)
+    dt = time.perf_counter() - t0
+    fl = 4.0 * w.D * Ls * Ls * (0.5 if w.causal else 1.0) * (3.5 if w.bwd else 1.0)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"1 head x first {Ls} tokens, {'fwd+bwd' if w.bwd else 'fwd'}, numpy fp64 "
+                      f"(BLAS threads {os.environ.get('OPENBLAS_NUM_THREADS', 'default')}), {dt:.2f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+    flops_step, fwd_flops = step_flops(w)
+    config = {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "cp": w.cp,
+              "layout": "head_tail" if w.layout == 1 else "contiguous", "causal": w.causal,
+              "step": "permute q,k,v" + (",dO" if w.bwd else "") + " -> ring fwd -> unpermute O" +
+                      (" -> ring bwd -> unpermute dQ,dK,dV" if w.bwd else ""),
+              "l2": "inputs larger than L2 (%.0f MB per tensor vs 126 MB)" % (w.B * w.H * w.L * w.D * 2 / 1e6),
+              "parallelism": "replicas"}
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        runs = [cpu_sample_run(w) for _ in range(args.warmup)]
+        runs = [cpu_sample_run(w) for _ in range(args.steps)]
+        val = statistics.median(r["value"] for r in runs)
+        cb = dict(runs[0])
+        cb["value"] = val
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": cb, "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                            "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    r = run_ours(args, w, rank, world, local)
+    pk, pk_kind = peaks()
+    value = world * flops_step * args.steps / (r["ms"] / 1e3) / 1e12
+    e2e_value = world * flops_step * args.steps / (r["e2e_ms"] / 1e3) / 1e12
+    # Dominant kernel: the backward when present (2.5x the forward's FLOPs).
+    if w.bwd:
+        kname, kflops, kms = "ring_bwd", 2.5 * fwd_flops, r["bwd_ms"]
+    else:
+        kname, kflops, kms = "ring_fwd", fwd_flops, r["fwd_ms"]
+    sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = kflops / (kms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q/K/V/dO)", "config": config,
+        "pct_of_bf16_peak": {"burst": 100.0 * value / world / burst, "sustained": 100.0 * value / world / sustained,
+                             "source": pk_kind},
+        "kernels": {"ring_fwd": {"ms": r["fwd_ms"], "tflops": fwd_flops / (r["fwd_ms"] / 1e3) / 1e12},
+                    "ring_bwd": ({"ms": r["bwd_ms"], "tflops": 2.5 * fwd_flops / (r["bwd_ms"] / 1e3) / 1e12}
+                                 if r["bwd_ms"] else None)},
+        "roofline": {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": sustained,
+                     "peak_kind": f"bf16_tflops_sustained ({pk_kind}); timed inside a long step",
+                     "unit": "TFLOP/s", "frac": achieved / sustained, "frac_of_burst": achieved / burst,
+                     "traffic": None},
+        "clocks": r["clocks"],
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"],
+    }
+    if rank == 0:
+        if world == 1:
+            line["cpu_baseline"] = cpu_sample_run(w)
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

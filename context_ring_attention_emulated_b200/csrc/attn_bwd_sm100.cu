@@ -1,6 +1,587 @@
-// attn_bwd_sm100.cu -- placeholder until the tensor-core backward lands.
+// attn_bwd_sm100.cu -- ring attention backward on the sm_100a tensor cores.
+//
+// Gradients of the ring forward ([CP-glossary] "Practical use and
+// trade-offs" runs `.backward()` through the CP attention), recomputing the
+// probabilities from the saved fp32 LSE instead of storing them:
+//   P = exp(scale Q K^T - LSE),  dV = P^T dO,  dP = dO V^T,
+//   dS = P o (dP - Delta),  Delta_i = dO_i . O_i,
+//   dQ = scale dS K,  dK = scale dS^T Q.
+// In a real ring the K/V block of rank s visits every rank r (at hop
+// (r - s) mod cp) and its dK/dV travel with it; here one CTA keeps one
+// 128-key K/V tile of rank s resident and walks every rank's query tiles in
+// that hop order, skipping tiles the causal relation fully masks. dK and dV
+// accumulate in TMEM; each query tile's dQ contribution is added into an fp32
+// workspace with vector atomics, converted to the output dtype at the end.
+//
+// Warp roles (192 threads):
+//   warp 0      producer: K, V once; per query tile Q, dO by TMA and the
+//               tile's LSE (pre-scaled by log2 e) and Delta into shared memory;
+//   warp 1      TMEM allocation and tcgen05.mma issue (one thread);
+//   warps 2..5  one thread per TMEM lane: P^T and dS^T for its key row, then
+//               the dQ read-out for its query row, finally dK/dV.
+// TMEM columns: A [0,128) S^T, then P^T (bf16, [0,64)) and dS^T ([64,128));
+// B [128,256) dP^T, then dQ; dV [256,256+D); dK [256+D,256+2D).
+#include <math.h>
+
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace rattn {
-rattn_status launch_bwd_sm100(const BwdArgs&, const DevCtx&) { return RATTN_ERR_UNSUPPORTED; }
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int BQ = 128;   // query rows per tile
+constexpr int BK = 128;   // key rows per CTA
+constexpr int kMaxHops = 64;
+
+template <int D>
+struct Cfg {
+  static constexpr int NSQ = (D == 128) ? 2 : 3;   // Q/dO stages
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOX = 128 * 128;            // one 128-row x 64-element box
+  static constexpr uint32_t T_A = 0, T_B = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr uint32_t T_COLS = 512;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;                 // NSQ stages
+  static constexpr int OFF_DO = OFF_Q + NSQ * TILE;          // NSQ stages
+  static constexpr int OFF_DS = OFF_DO + NSQ * TILE;         // 128 x 128 bf16, two boxes
+  static constexpr int OFF_LSE = OFF_DS + 2 * BOX;           // NSQ x 128 floats
+  static constexpr int OFF_DELTA = OFF_LSE + NSQ * 128 * 4;  // NSQ x 128 floats
+  static constexpr int OFF_BAR = OFF_DELTA + NSQ * 128 * 4;
+  static constexpr int NBAR = 1 + 2 * NSQ + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_HOP = OFF_MISC + 16;
+  static constexpr int SMEM = OFF_HOP + kMaxHops * 8;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+struct Params {
+  const float* lse;
+  const float* delta;
+  const int32_t* pos;
+  int BH, nseg, Lseg, nq_tiles, nk_tiles, causal;
+  long long kv_valid;
+  float scale, scale_log2;
+  float* dq_acc;
+  void* dk;
+  void* dv;
+  int* err;
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ long long posat(const Params& p, int seg, int row) {
+  return static_cast<long long>(__ldg(p.pos + static_cast<long long>(seg) * p.Lseg + row));
+}
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kDrainLimitNs) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_kv_full = bars;
+  uint64_t* bar_q_full = bars + 1;
+  uint64_t* bar_q_empty = bar_q_full + C::NSQ;
+  uint64_t* bar_s_full = bar_q_empty + C::NSQ;
+  uint64_t* bar_dp_full = bar_s_full + 1;
+  uint64_t* bar_ds_ready = bar_dp_full + 1;
+  uint64_t* bar_a_free = bar_ds_ready + 1;
+  uint64_t* bar_dq_full = bar_a_free + 1;
+  uint64_t* bar_dq_free = bar_dq_full + 1;
+  uint64_t* bar_drain = bar_dq_free + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
+  float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
+  float* s_delta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // The 128-byte swizzle needs 1024-byte aligned tiles; refuse to run otherwise.
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0 && p.err) atomicCAS(p.err, 0, SITE_BWD_LOAD);
+    return;
+  }
+
+  // Work item: key tiles with the smallest positions (seen by the most
+  // queries under causal masking) first.
+  int item = blockIdx.x;
+  const int bh = item % p.BH;
+  item /= p.BH;
+  const int s = item % p.nseg;
+  const int kt = item / p.nseg;
+  const int k0 = kt * BK;
+  const int k_rows = min(BK, p.Lseg - k0);
+  const long long k_min = posat(p, s, k0);
+  const long long k_max = posat(p, s, k0 + k_rows - 1);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv_full, 1);
+    for (int i = 0; i < C::NSQ; ++i) {
+      mbar_init(&bar_q_full[i], 1);
+      mbar_init(&bar_q_empty[i], 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_ds_ready, 128);
+    mbar_init(bar_a_free, 1);
+    mbar_init(bar_dq_full, 1);
+    mbar_init(bar_dq_free, 128);
+    mbar_init(bar_drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(s_tmem, C::T_COLS);
+
+  // Per hop t the query segment is r = (s + t) mod nseg. Visible query tiles
+  // form a suffix [first_vis, nq_tiles) and unmasked ones a suffix
+  // [first_full, nq_tiles), since positions are non-decreasing in a segment.
+  const bool live = k_min < p.kv_valid;
+  for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
+    const int r = (s + t) % p.nseg;
+    int first_vis = p.nq_tiles, first_full = p.nq_tiles;
+    if (live) {
+      if (!p.causal) {
+        first_vis = 0;
+        first_full = 0;
+      } else {
+        int lo = 0, hi = p.nq_tiles;
+        while (lo < hi) {  // first tile whose last query sees the first key
+          const int mid = (lo + hi) >> 1;
+          const long long qmax = posat(p, r, min((mid + 1) * BQ, p.Lseg) - 1);
+          if (qmax >= k_min) hi = mid; else lo = mid + 1;
+        }
+        first_vis = lo;
+        hi = p.nq_tiles;
+        while (lo < hi) {  // first tile whose first query sees every key
+          const int mid = (lo + hi) >> 1;
+          const long long qmin = posat(p, r, mid * BQ);
+          if (qmin >= k_max) hi = mid; else lo = mid + 1;
+        }
+        first_full = lo;
+      }
+    }
+    s_hop[t] = make_int2(first_vis, first_full);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  int NIT = 0;
+  for (int t = 0; t < p.nseg; ++t) NIT += p.nq_tiles - s_hop[t].x;
+
+  int issued_q = 0;
+  bool kv_issued = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (NIT > 0) {
+      if (lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_do);
+        mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
+        for (int b = 0; b < C::NBOX; ++b) {
+          tma_load_4d(smem + C::OFF_K + b * C::BOX, &tm_k, bar_kv_full, b * 64, k0, s, bh);
+          tma_load_4d(smem + C::OFF_V + b * C::BOX, &tm_v, bar_kv_full, b * 64, k0, s, bh);
+        }
+      }
+      kv_issued = true;
+      bool ok = true;
+      int it = 0;
+      for (int t = 0; t < p.nseg && ok; ++t) {
+        const int r = (s + t) % p.nseg;
+        for (int i = s_hop[t].x; i < p.nq_tiles; ++i, ++it) {
+          const int st = it % C::NSQ;
+          const uint32_t u = it / C::NSQ;
+          if (u > 0 && !warp_wait(&bar_q_empty[st], (u - 1) & 1, s_abort, p.wait_ns)) {
+            if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_LOAD);
+            ok = false;
+            break;
+          }
+          const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = lane * 4 + e;
+            const int q = i * BQ + c;
+            float l2 = INFINITY, dl = 0.f;
+            if (q < p.Lseg) {
+              const float l = __ldg(p.lse + rowbase + q);
+              l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+              dl = __ldg(p.delta + rowbase + q);
+            }
+            s_lse[st * 128 + c] = l2;
+            s_delta[st * 128 + c] = dl;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar_q_full[st], 2 * C::TILE);
+            for (int b = 0; b < C::NBOX; ++b) {
+              tma_load_4d(smem + C::OFF_Q + st * C::TILE + b * C::BOX, &tm_q, &bar_q_full[st], b * 64, i * BQ, r,
+                          bh);
+              tma_load_4d(smem + C::OFF_DO + st * C::TILE + b * C::BOX, &tm_do, &bar_q_full[st], b * 64, i * BQ,
+                          r, bh);
+            }
+          }
+          ++issued_q;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issue
+    if (lane == 0 && NIT > 0) {
+      const uint32_t idesc_t = idesc_bf16_f32(BK, BQ, 0, 0);    // S^T, dP^T: K-major A and B
+      const uint32_t idesc_g = idesc_bf16_f32(BK, D, 0, 1);     // dV, dK: A in TMEM, B MN-major
+      const uint32_t idesc_q = idesc_bf16_f32(BQ, D, 1, 1);     // dQ: A (dS) and B (K) MN-major
+      const uint32_t sK = smem_u32(smem + C::OFF_K);
+      const uint32_t sV = smem_u32(smem + C::OFF_V);
+      const uint32_t sDS = smem_u32(smem + C::OFF_DS);
+      bool ok = mbar_wait(bar_kv_full, 0, s_abort, p.wait_ns);
+      for (int it = 0; it < NIT && ok; ++it) {
+        const int st = it % C::NSQ;
+        const uint32_t sQ = smem_u32(smem + C::OFF_Q + st * C::TILE);
+        const uint32_t sDO = smem_u32(smem + C::OFF_DO + st * C::TILE);
+        ok = mbar_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns);
+        if (ok && it > 0) ok = mbar_wait(bar_a_free, (it - 1) & 1, s_abort, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T
+          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+          umma_ss(tmem + C::T_A, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idesc_t,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_s_full);
+        if (it > 0 && !(ok = mbar_wait(bar_dq_free, (it - 1) & 1, s_abort, p.wait_ns))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+          umma_ss(tmem + C::T_B, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idesc_t,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_dp_full);
+        if (!(ok = mbar_wait(bar_ds_ready, it & 1, s_abort, p.wait_ns))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {  // dV += P^T dO ; dK += dS^T Q
+          const uint64_t bdo = sdesc_sw128(sDO + kk * 2048, C::BOX, 1024);
+          const uint64_t bq = sdesc_sw128(sQ + kk * 2048, C::BOX, 1024);
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          umma_ts(tmem + C::T_DV, tmem + C::T_A + kk * 8, bdo, idesc_g, acc);
+          umma_ts(tmem + C::T_DK, tmem + C::T_A + 64 + kk * 8, bq, idesc_g, acc);
+        }
+        umma_commit(bar_a_free);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {  // dQ = dS K
+          umma_ss(tmem + C::T_B, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
+                  sdesc_sw128(sK + kk * 2048, C::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_dq_full);
+        umma_commit(&bar_q_empty[st]);
+      }
+      if (!ok) record_failure(s_abort, p.err, SITE_BWD_MMA);
+    }
+  } else {
+    // ------------------------------------------------- per-lane gradients
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key row for S^T/dP^T/dK/dV, query row for dQ
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool key_ok = row < k_rows;
+    const long long my_kpos = key_ok ? posat(p, s, k0 + row) : k_max;
+    const bool key_dead = !key_ok || my_kpos >= p.kv_valid;
+    const float sl2 = p.scale_log2;
+    uint8_t* sds = smem + C::OFF_DS;
+    bool ok = true;
+    int it = 0;
+    for (int t = 0; t < p.nseg && ok; ++t) {
+      const int r = (s + t) % p.nseg;
+      const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
+      for (int i = s_hop[t].x; i < p.nq_tiles; ++i, ++it) {
+        const int st = it % C::NSQ;
+        const float* lse2 = s_lse + st * 128;
+        const float* dlt = s_delta + st * 128;
+        // first query column of this tile that sees this key (suffix)
+        int first = 0;
+        if (key_dead) {
+          first = BQ;
+        } else if (i < s_hop[t].y) {
+          int lo = 0, hi = min(BQ, p.Lseg - i * BQ);
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (posat(p, r, i * BQ + mid) >= my_kpos) hi = mid; else lo = mid + 1;
+          }
+          first = lo;
+        }
+        if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns) ||
+            !warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
+          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + C::T_A + c * 32, sr[c]);
+        tmem_wait_ld();
+        // P^T (fp32, kept in sr) and its bf16 copy into TMEM columns [0, 64)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c0 = h * 64 + 2 * e;
+            float a = ex2_approx(fmaf(__uint_as_float(sr[c0 >> 5][c0 & 31]), sl2, -lse2[c0]));
+            float b = ex2_approx(fmaf(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), sl2, -lse2[c0 + 1]));
+            a = c0 >= first ? a : 0.f;
+            b = c0 + 1 >= first ? b : 0.f;
+            sr[c0 >> 5][c0 & 31] = __float_as_uint(a);
+            sr[(c0 + 1) >> 5][(c0 + 1) & 31] = __float_as_uint(b);
+            pk[e] = pack_bf16x2(a, b);
+          }
+          tmem_st32(tmem + lane_base + C::T_A + h * 32, pk);
+        }
+        if (!warp_wait(bar_dp_full, it & 1, s_abort, p.wait_ns)) {
+          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // dS^T = P^T o (dP^T - Delta): bf16 into TMEM [64, 128) and into the
+        // swizzled shared tile read by the dQ MMA.
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(tmem + lane_base + C::T_B + c * 32, dp);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int q0 = c * 32 + 2 * e;
+            const float a = __uint_as_float(sr[c][2 * e]) * (__uint_as_float(dp[2 * e]) - dlt[q0]);
+            const float b = __uint_as_float(sr[c][2 * e + 1]) * (__uint_as_float(dp[2 * e + 1]) - dlt[q0 + 1]);
+            pk[e] = pack_bf16x2(a, b);
+          }
+          tmem_st16(tmem + lane_base + C::T_A + 64 + c * 16, pk);
+          // 32 query columns = 4 16-byte chunks of box (c >> 1)
+          uint8_t* rowp = sds + (c >> 1) * C::BOX + row * 128;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int chunk = (c & 1) * 4 + j;
+            *reinterpret_cast<uint4*>(rowp + ((chunk ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar_ds_ready);
+        // dQ read-out: this lane's query row of the tile.
+        if (!warp_wait(bar_dq_full, it & 1, s_abort, p.wait_ns)) {
+          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int q = i * BQ + row;
+        float* dst = p.dq_acc + (rowbase + q) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t g[32];
+          tmem_ld32(tmem + lane_base + C::T_B + c * 32, g);
+          tmem_wait_ld();
+          if (q < p.Lseg) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + 4 * e),
+                        make_float4(__uint_as_float(g[4 * e]), __uint_as_float(g[4 * e + 1]),
+                                    __uint_as_float(g[4 * e + 2]), __uint_as_float(g[4 * e + 3])));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_dq_free);
+      }
+    }
+    // ------------------------------------------------------ dK, dV out
+    if (ok && NIT > 0 && !warp_wait(bar_a_free, (NIT - 1) & 1, s_abort, p.wait_ns)) {
+      if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_EPILOGUE);
+      ok = false;
+    }
+    if (ok) {
+      if (NIT > 0) tc_fence_after();
+      const long long krow = (static_cast<long long>(bh) * p.nseg + s) * p.Lseg + k0 + row;
+      __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + krow * D;
+      __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + krow * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t gk[32], gv[32];
+        if (NIT > 0) {
+          tmem_ld32(tmem + lane_base + C::T_DK + c * 32, gk);
+          tmem_ld32(tmem + lane_base + C::T_DV + c * 32, gv);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) gk[e] = gv[e] = 0u;
+        }
+        if (key_ok) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 wk, wv;
+            wk.x = pack_bf16x2(__uint_as_float(gk[8 * e + 0]) * p.scale, __uint_as_float(gk[8 * e + 1]) * p.scale);
+            wk.y = pack_bf16x2(__uint_as_float(gk[8 * e + 2]) * p.scale, __uint_as_float(gk[8 * e + 3]) * p.scale);
+            wk.z = pack_bf16x2(__uint_as_float(gk[8 * e + 4]) * p.scale, __uint_as_float(gk[8 * e + 5]) * p.scale);
+            wk.w = pack_bf16x2(__uint_as_float(gk[8 * e + 6]) * p.scale, __uint_as_float(gk[8 * e + 7]) * p.scale);
+            wv.x = pack_bf16x2(__uint_as_float(gv[8 * e + 0]), __uint_as_float(gv[8 * e + 1]));
+            wv.y = pack_bf16x2(__uint_as_float(gv[8 * e + 2]), __uint_as_float(gv[8 * e + 3]));
+            wv.z = pack_bf16x2(__uint_as_float(gv[8 * e + 4]), __uint_as_float(gv[8 * e + 5]));
+            wv.w = pack_bf16x2(__uint_as_float(gv[8 * e + 6]), __uint_as_float(gv[8 * e + 7]));
+            reinterpret_cast<uint4*>(dk + c * 32)[e] = wk;
+            reinterpret_cast<uint4*>(dv + c * 32)[e] = wv;
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  if (warp == 0 && lane == 0) {
+    if (kv_issued) drain_wait(bar_kv_full, 0);
+    for (int it = max(0, issued_q - C::NSQ); it < issued_q; ++it)
+      drain_wait(&bar_q_full[it % C::NSQ], (it / C::NSQ) & 1);
+  }
+  if (warp == 1 && lane == 0 && NIT > 0) {
+    umma_commit(bar_drain);
+    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::T_COLS);
+  }
+}
+
+// Delta_i = dO_i . O_i (fp32) and zeroing of the dQ accumulator rows: one
+// 16-lane group per row, 16-byte loads.
+template <int D>
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                float* __restrict__ delta, float* __restrict__ dq_acc, long long rows) {
+  constexpr int V = D / 8;  // 16-byte vectors per bf16 row
+  const long long gid = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+  const long long row = gid / 16;
+  const int l = static_cast<int>(gid & 15);
+  float s = 0.f;
+  if (row < rows) {
+    for (int e = l; e < V; e += 16) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + e);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + e);
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 fa = __bfloat1622float2(pa[j]);
+        const float2 fb = __bfloat1622float2(pb[j]);
+        s = fmaf(fa.x, fb.x, s);
+        s = fmaf(fa.y, fb.y, s);
+      }
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
+    for (int e = l; e < D / 4; e += 16) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (row < rows && l == 0) delta[row] = s;
+}
+
+// dq = bf16(scale * dq_acc)
+__global__ void dq_convert_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq, float scale,
+                                  long long n4) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldg(acc + i);
+    dq[i] = make_uint2(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale));
+  }
+}
+
+unsigned grid_for(long long work, int threads) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (work + threads - 1) / threads;
+  const long long cap = static_cast<long long>(sms) * 16;
+  return static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+template <int D>
+rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
+  using C = Cfg<D>;
+  if (a.Lseg > INT32_MAX - BQ || a.nseg > kMaxHops) return RATTN_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(a.BH) * a.nseg * a.Lseg;
+  const int nt = static_cast<int>((a.Lseg + 127) / 128);
+  const long long grid = static_cast<long long>(a.BH) * a.nseg * nt;
+  if (grid == 0) return RATTN_OK;
+  if (grid > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
+      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
+  if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
+  CUtensorMap tq, tk, tv, tdo;
+  rattn_status st;
+  if ((st = make_tmap_bf16(&tq, a.q, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH, BK)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH, BK)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
+  if ((st = set_smem_attr(reinterpret_cast<const void*>(&bwd_kernel<D>), C::SMEM)) != RATTN_OK) return st;
+  Params p;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.pos = a.pos;
+  p.BH = a.BH;
+  p.nseg = a.nseg;
+  p.Lseg = static_cast<int>(a.Lseg);
+  p.nq_tiles = nt;
+  p.nk_tiles = nt;
+  p.causal = a.causal;
+  p.kv_valid = a.kv_valid;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.dq_acc = a.dq_acc;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.err = ctx.err_word;
+  p.wait_ns = ctx.wait_ns;
+  bwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
+  const long long n4 = rows * D / 4;
+  dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
+                                                            static_cast<uint2*>(a.dq), a.scale, n4);
+  return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+rattn_status launch_bwd_sm100(const BwdArgs& a, const DevCtx& ctx) {
+  if (a.dtype != RATTN_BF16) return RATTN_ERR_UNSUPPORTED;
+  if (a.D == 128) return launch<128>(a, ctx);
+  if (a.D == 64) return launch<64>(a, ctx);
+  return RATTN_ERR_UNSUPPORTED;
+}
+
 }  // namespace rattn

@@ -182,6 +182,7 @@ def test_ring_fwd_full_size_sampled(rattn, name, heads):
     for h in heads:
         qh = to64(q[0, h, torch.from_numpy(rows).cuda()])
         kh, vh = to64(k[0, h]), to64(v[0, h])
-        o_ref, l_ref = oracle.attention(qh, kh, vh, w.scale, w.causal, q_pos=rows, kv_pos=np.arange(w.L))
+        o_ref, l_ref = oracle.attention(qh, kh, vh, w.scale, w.causal, q_pos=rows, kv_pos=np.arange(w.L),
+                                        row_block=64)
         check_o(o[0, h, slots].float().cpu().numpy(), o_ref, w.torch_dtype)
         check_lse(lse[0, h, slots].cpu().numpy(), l_ref, w.torch_dtype)
