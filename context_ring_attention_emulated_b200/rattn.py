@@ -37,6 +37,8 @@ SIGNATURES = [
     ("rattn_ring_bwd_workspace_size", ctypes.c_size_t, [_I, _I, _I64, _I]),
     ("rattn_ring_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
                             _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("rattn_ring_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
+                                    _P, _P, _P, _P]),
     ("rattn_get_device_error", _I, [ctypes.POINTER(_I)]),
     ("rattn_set_wait_limit_ns", _I, [ctypes.c_ulonglong]),
 ]
@@ -190,6 +192,23 @@ def rattn_ring_bwd(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL,
                                                  _ptr(pos), B, H, Lp, D, _dtype_code(q), cp_size, layout,
                                                  int(causal), float(scale), int(L_valid), _ptr(dq), _ptr(dk),
                                                  _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def rattn_ring_bwd_noalloc(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None,
+                           L_valid=None, dq=None, dk=None, dv=None, stream=None):
+    """rattn_ring_bwd without a workspace: scratch comes from the library's own
+    fixed device array (for callers that cannot allocate device memory)."""
+    _need_cuda(q, k, v, o, dout, lse, pos)
+    B, H, Lp, D = q.shape
+    scale = D ** -0.5 if scale is None else scale
+    L_valid = Lp if L_valid is None else L_valid
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check("rattn_ring_bwd_noalloc", lib.rattn_ring_bwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(pos), B, H, Lp, D, _dtype_code(q), cp_size,
+        layout, int(causal), float(scale), int(L_valid), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)))
     return dq, dk, dv
 
 

@@ -153,6 +153,32 @@ rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const v
                             int64_t L_valid, void* dq, void* dk, void* dv,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the device array rattn_ring_bwd_noalloc uses as scratch space. */
+#define RATTN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* The pages have no counterpart of this call. It is rattn_ring_bwd for
+ * callers that cannot allocate device memory: code that runs where no
+ * allocator is reachable (a plugin inside a host framework that owns all of
+ * the device's memory, a runtime that forbids allocation after start-up, or a
+ * process with a fixed memory budget), so it cannot provide a workspace.
+ * Arguments, layouts and results are those of rattn_ring_bwd, without the
+ * workspace. Scratch space is a RATTN_NOALLOC_SCRATCH_BYTES device array that
+ * is part of the library: every GPU that loads the library keeps it until the
+ * process exits, and nothing is allocated or freed by this call. A request
+ * whose rattn_ring_bwd_workspace_size exceeds that size returns
+ * RATTN_ERR_UNSUPPORTED and launches nothing. The first call on a device,
+ * with that device current, looks up the array's device address (once per
+ * device); make that first call before any stream capture on the device. All
+ * calls share the one array and it keeps the previous call's contents (the
+ * parts that must start at zero are cleared on the device by the call
+ * itself), so calls whose execution overlaps on the GPU, on any streams,
+ * race on it: order them on one stream or synchronise between them. */
+rattn_status rattn_ring_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                    const void* dout, const float* lse, const int32_t* pos,
+                                    int B, int H, int64_t Lp, int D, rattn_dtype dtype,
+                                    int cp_size, rattn_layout layout, int causal, float scale,
+                                    int64_t L_valid, void* dq, void* dk, void* dv, void* stream);
+
 /* Reads and clears the device-side error word of the current device
  * (synchronises the device). Returns RATTN_OK if no kernel recorded an
  * error, RATTN_ERR_TIMEOUT if a bounded wait gave up (*site, if non-NULL,
