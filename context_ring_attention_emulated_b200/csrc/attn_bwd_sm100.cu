@@ -120,13 +120,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Work item: key tiles with the smallest positions (seen by the most
-  // queries under causal masking) first.
+  // Work item: (batch, head) slowest, so the CTAs resident at any time share
+  // one head's Q, dO and dQ accumulator in L2; within a head the key tiles
+  // with the smallest positions (seen by the most queries) go first.
   int item = blockIdx.x;
-  const int bh = item % p.BH;
-  item /= p.BH;
   const int s = item % p.nseg;
-  const int kt = item / p.nseg;
+  item /= p.nseg;
+  const int kt = item % p.nk_tiles;
+  const int bh = item / p.nk_tiles;
   const int k0 = kt * BK;
   const int k_rows = min(BK, p.Lseg - k0);
   const long long k_min = posat(p, s, k0);

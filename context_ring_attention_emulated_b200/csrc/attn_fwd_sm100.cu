@@ -118,14 +118,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work item: heaviest query tiles (largest local index, hence largest
-  // positions under both layouts) are launched first.
+  // Work item: (batch, head) slowest, so the CTAs resident at any time share
+  // one head's K/V in L2; within a head the heaviest query tiles (largest
+  // local index, hence largest positions under both layouts) go first.
   int item = blockIdx.x;
-  const int bh = item % p.BH;
-  item /= p.BH;
   const int r = item % p.nseg;
   item /= p.nseg;
-  const int qt = p.n_qtiles - 1 - item;
+  const int qt = p.n_qtiles - 1 - (item % p.n_qtiles);
+  const int bh = item / p.n_qtiles;
   const int q0 = qt * BM;
   const int q_rows = min(BM, p.Lq_seg - q0);
   const long long q_min = qpos(p, r, q0);
