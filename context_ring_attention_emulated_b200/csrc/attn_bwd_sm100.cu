@@ -13,13 +13,16 @@
 // accumulate in TMEM; each query tile's dQ contribution is added into an fp32
 // workspace with vector atomics, converted to the output dtype at the end.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      producer: K, V once; per query tile Q, dO by TMA and the
 //               tile's LSE (pre-scaled by log2 e) and Delta into shared memory;
 //   warp 1      TMEM allocation and tcgen05.mma issue (one thread);
-//   warps 2..5  one thread per TMEM lane: P^T and dS^T for its key row, then
-//               the dQ read-out for its query row, finally dK/dV.
-// TMEM columns: A [0,128) S^T, then P^T (bf16, [0,64)) and dS^T ([64,128));
+//   warps 2..9  two warpgroups, one thread per TMEM lane each: P^T and dS^T
+//               for its key row over the warpgroup's 64 query columns, then
+//               the dQ read-out for its query row over half of D, finally
+//               half of dK/dV.
+// TMEM columns: A [0,128) S^T; warpgroup g then overwrites its own columns
+// [64g, 64g+64) with P^T (bf16, [64g, 64g+32)) and dS^T ([64g+32, 64g+64));
 // B [128,256) dP^T, then dQ; dV [256,256+D); dK [256+D,256+2D).
 #include <math.h>
 
@@ -29,7 +32,7 @@
 namespace rattn {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int BQ = 128;   // query rows per tile
 constexpr int BK = 128;   // key rows per CTA
 constexpr int kMaxHops = 64;
@@ -141,10 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_ds_ready, 128);
+    mbar_init(bar_ds_ready, 256);
     mbar_init(bar_a_free, 1);
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 128);
+    mbar_init(bar_dq_free, 256);
     mbar_init(bar_drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -282,27 +285,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(bar_dp_full);
         if (!(ok = mbar_wait(bar_ds_ready, it & 1, s_abort, p.wait_ns))) break;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {  // dV += P^T dO ; dK += dS^T Q
-          const uint64_t bdo = sdesc_sw128(sDO + kk * 2048, C::BOX, 1024);
-          const uint64_t bq = sdesc_sw128(sQ + kk * 2048, C::BOX, 1024);
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          umma_ts(tmem + C::T_DV, tmem + C::T_A + kk * 8, bdo, idesc_g, acc);
-          umma_ts(tmem + C::T_DK, tmem + C::T_A + 64 + kk * 8, bq, idesc_g, acc);
-        }
-        umma_commit(bar_a_free);
+        // dQ first, so its read-out and atomics overlap the dV / dK MMAs.
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {  // dQ = dS K
           umma_ss(tmem + C::T_B, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
                   sdesc_sw128(sK + kk * 2048, C::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_dq_full);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {  // dV += P^T dO ; dK += dS^T Q
+          const uint64_t bdo = sdesc_sw128(sDO + kk * 2048, C::BOX, 1024);
+          const uint64_t bq = sdesc_sw128(sQ + kk * 2048, C::BOX, 1024);
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t a_col = C::T_A + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s columns
+          umma_ts(tmem + C::T_DV, tmem + a_col, bdo, idesc_g, acc);
+          umma_ts(tmem + C::T_DK, tmem + a_col + 32, bq, idesc_g, acc);
+        }
+        umma_commit(bar_a_free);
         umma_commit(&bar_q_empty[st]);
       }
       if (!ok) record_failure(s_abort, p.err, SITE_BWD_MMA);
     }
   } else {
     // ------------------------------------------------- per-lane gradients
+    // Two warpgroups; warpgroup wg owns query columns [64 wg, 64 wg + 64) of
+    // every tile (and D columns [wg D/2, (wg+1) D/2) of dQ, dK, dV). Each
+    // writes its P^T / dS^T only into TMEM columns it alone has read:
+    // P^T of its columns at T_A + 64 wg, dS^T at T_A + 64 wg + 32.
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key row for S^T/dP^T/dK/dV, query row for dQ
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -310,7 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long my_kpos = key_ok ? posat(p, s, k0 + row) : k_max;
     const bool key_dead = !key_ok || my_kpos >= p.kv_valid;
     const float sl2 = p.scale_log2;
-    uint8_t* sds = smem + C::OFF_DS;
+    const int qc0 = wg * 64;              // first query column of this warpgroup
+    const uint32_t t_a = tmem + lane_base + C::T_A + wg * 64;
+    uint8_t* sds = smem + C::OFF_DS + wg * C::BOX;
     bool ok = true;
     int it = 0;
     for (int t = 0; t < p.nseg && ok; ++t) {
@@ -318,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
       for (int i = s_hop[t].x; i < p.nq_tiles; ++i, ++it) {
         const int st = it % C::NSQ;
-        const float* lse2 = s_lse + st * 128;
-        const float* dlt = s_delta + st * 128;
+        const float* lse2 = s_lse + st * 128 + qc0;
+        const float* dlt = s_delta + st * 128 + qc0;
         // first query column of this tile that sees this key (suffix)
         int first = 0;
         if (key_dead) {
@@ -332,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           first = lo;
         }
+        first -= qc0;  // relative to this warpgroup's columns
         if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns) ||
             !warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
@@ -339,17 +352,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        uint32_t sr[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_base + C::T_A + c * 32, sr[c]);
+        uint32_t sr[2][32];
+        tmem_ld32(t_a, sr[0]);
+        tmem_ld32(t_a + 32, sr[1]);
         tmem_wait_ld();
-        // P^T (fp32, kept in sr) and its bf16 copy into TMEM columns [0, 64)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        // P^T (fp32, kept in sr) and its bf16 copy into TMEM
+        {
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int c0 = h * 64 + 2 * e;
+            const int c0 = 2 * e;
             float a = ex2_approx(fmaf(__uint_as_float(sr[c0 >> 5][c0 & 31]), sl2, -lse2[c0]));
             float b = ex2_approx(fmaf(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), sl2, -lse2[c0 + 1]));
             a = c0 >= first ? a : 0.f;
@@ -358,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sr[(c0 + 1) >> 5][(c0 + 1) & 31] = __float_as_uint(b);
             pk[e] = pack_bf16x2(a, b);
           }
-          tmem_st32(tmem + lane_base + C::T_A + h * 32, pk);
+          tmem_st32(t_a, pk);
         }
         if (!warp_wait(bar_dp_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
@@ -366,27 +378,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        // dS^T = P^T o (dP^T - Delta): bf16 into TMEM [64, 128) and into the
-        // swizzled shared tile read by the dQ MMA.
+        // dS^T = P^T o (dP^T - Delta): bf16 into TMEM and into the swizzled
+        // shared tile read by the dQ MMA (box wg, row = key).
+        uint32_t dp[2][32];
+        tmem_ld32(tmem + lane_base + C::T_B + qc0, dp[0]);
+        tmem_ld32(tmem + lane_base + C::T_B + qc0 + 32, dp[1]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t dp[32];
-          tmem_ld32(tmem + lane_base + C::T_B + c * 32, dp);
-          tmem_wait_ld();
+        for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int q0 = c * 32 + 2 * e;
-            const float a = __uint_as_float(sr[c][2 * e]) * (__uint_as_float(dp[2 * e]) - dlt[q0]);
-            const float b = __uint_as_float(sr[c][2 * e + 1]) * (__uint_as_float(dp[2 * e + 1]) - dlt[q0 + 1]);
+            const float a = __uint_as_float(sr[c][2 * e]) * (__uint_as_float(dp[c][2 * e]) - dlt[q0]);
+            const float b = __uint_as_float(sr[c][2 * e + 1]) * (__uint_as_float(dp[c][2 * e + 1]) - dlt[q0 + 1]);
             pk[e] = pack_bf16x2(a, b);
           }
-          tmem_st16(tmem + lane_base + C::T_A + 64 + c * 16, pk);
-          // 32 query columns = 4 16-byte chunks of box (c >> 1)
-          uint8_t* rowp = sds + (c >> 1) * C::BOX + row * 128;
+          tmem_st16(t_a + 32 + c * 16, pk);
+          uint8_t* rowp = sds + row * 128;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int chunk = (c & 1) * 4 + j;
+            const int chunk = c * 4 + j;
             *reinterpret_cast<uint4*>(rowp + ((chunk ^ (row & 7)) << 4)) =
                 make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
@@ -395,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar_ds_ready);
-        // dQ read-out: this lane's query row of the tile.
+        // dQ read-out: this lane's query row, this warpgroup's half of D.
         if (!warp_wait(bar_dq_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
           ok = false;
@@ -403,11 +415,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const int q = i * BQ + row;
-        float* dst = p.dq_acc + (rowbase + q) * D;
+        float* dst = p.dq_acc + (rowbase + q) * D + wg * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t g[32];
-          tmem_ld32(tmem + lane_base + C::T_B + c * 32, g);
+          tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + c * 32, g);
           tmem_wait_ld();
           if (q < p.Lseg) {
 #pragma unroll
@@ -429,14 +441,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       if (NIT > 0) tc_fence_after();
       const long long krow = (static_cast<long long>(bh) * p.nseg + s) * p.Lseg + k0 + row;
-      __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + krow * D;
-      __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + krow * D;
+      __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + krow * D + wg * (D / 2);
+      __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + krow * D + wg * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t gk[32], gv[32];
         if (NIT > 0) {
-          tmem_ld32(tmem + lane_base + C::T_DK + c * 32, gk);
-          tmem_ld32(tmem + lane_base + C::T_DV + c * 32, gv);
+          tmem_ld32(tmem + lane_base + C::T_DK + wg * (D / 2) + c * 32, gk);
+          tmem_ld32(tmem + lane_base + C::T_DV + wg * (D / 2) + c * 32, gv);
           tmem_wait_ld();
         } else {
 #pragma unroll

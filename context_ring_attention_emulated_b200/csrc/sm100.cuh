@@ -66,16 +66,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the barrier phase of the given parity has completed. Gives up
-// (returns false) after limit_ns nanoseconds or as soon as *abort is set, so a
-// lost arrival can never hang the GPU.
+// (returns false) after about limit_ns nanoseconds (counted in SM cycles at an
+// assumed 2 GHz) or as soon as *abort is set, so a lost arrival can never hang
+// the GPU. The limit and the abort flag are checked on the first retry and
+// then every 64 polls, to keep the poll loop short.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
+  const long long t0 = clock64();
+  const long long limit_cycles = static_cast<long long>(limit_ns < (1ull << 61) ? limit_ns * 2 : (1ull << 62));
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (global_timer_ns() - t0 > limit_ns) return false;
+    if ((i & 63u) == 1u) {
+      if (*abort) return false;
+      if (clock64() - t0 > limit_cycles) return false;
+    }
   }
 }
 
