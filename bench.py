@@ -115,13 +115,20 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a per-rank time over all ranks (every rank gets the result)."""
     if world <= 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_tflops(flops_per_step, steps, world, ms_max):
+    """Whole-job throughput: the work of all ranks (each runs one replica of
+    the workload) over the max-over-ranks device time."""
+    return world * flops_per_step * steps / (ms_max / 1e3) / 1e12
 
 
 def run_ours(args, w, rank, world, local):
@@ -282,8 +289,8 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     r = run_ours(args, w, rank, world, local)
     pk, pk_kind = peaks()
-    value = world * flops_step * args.steps / (r["ms"] / 1e3) / 1e12
-    e2e_value = world * flops_step * args.steps / (r["e2e_ms"] / 1e3) / 1e12
+    value = aggregate_tflops(flops_step, args.steps, world, r["ms"])
+    e2e_value = aggregate_tflops(flops_step, args.steps, world, r["e2e_ms"])
     # Dominant kernel: the backward when present (2.5x the forward's FLOPs).
     if w.bwd:
         kname, kflops, kms = "ring_bwd", 2.5 * fwd_flops, r["bwd_ms"]
