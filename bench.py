@@ -31,6 +31,12 @@ from context_ring_attention_emulated_b200.workloads import WORKLOADS, make_qkv, 
 METRIC = "ring-attn fwd/bwd TFLOP/s (causal FLOPs) on 1 B200; % of BF16 tensor peak"
 DEFAULT = "bf16_L32000_cp4_fwdbwd"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of the current kernel on a half-length case, scaled to the full
+# launch by sequence length (traffic grows with the tensors). Source:
+# profiles/bwd_kernel_bf16_H32_L16000_cp4.md. Set to None when the kernel
+# changes until it is captured again.
+NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": (791.8e6 + 479.9e6) * 2}
 
 
 def peaks():
@@ -311,7 +317,7 @@ def main():
         "roofline": {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": sustained,
                      "peak_kind": f"bf16_tflops_sustained ({pk_kind}); timed inside a long step",
                      "unit": "TFLOP/s", "frac": achieved / sustained, "frac_of_burst": achieved / burst,
-                     "traffic": None},
+                     "traffic": NCU_TRAFFIC.get(w.name) if w.bwd else None},
         "clocks": r["clocks"],
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
