@@ -106,23 +106,6 @@ rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t r
   return r == CUDA_SUCCESS ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
-rattn_status make_tmap_f32(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,
-                           int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return RATTN_ERR_CUDA;
-  if (rows < 1) rows = 1;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(nseg), static_cast<cuuint64_t>(outer)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(rows) * D * 4,
-                                 static_cast<cuuint64_t>(nseg) * rows * D * 4};
-  const cuuint32_t box[4] = {32u, static_cast<cuuint32_t>(box_rows), 1u, 1u};
-  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? RATTN_OK : RATTN_ERR_CUDA;
-}
-
 }  // namespace rattn
 
 using namespace rattn;

@@ -10,9 +10,10 @@
 // (r - s) mod cp) and its dK/dV travel with it; here one CTA keeps one
 // 128-key K/V tile of rank s resident and walks every rank's query tiles in
 // that hop order, skipping tiles the causal relation fully masks. dK and dV
-// accumulate in TMEM; each query tile's dQ contribution is staged in shared
-// memory and added into an fp32 workspace by TMA reduce-adds (line-granular
-// reductions at L2), converted to the output dtype at the end.
+// accumulate in TMEM; each query tile's dQ contribution is transposed
+// through shared memory (warp-local) and added into an fp32 workspace with
+// coalesced vector reductions (whole 128-byte lines per warp instruction),
+// converted to the output dtype at the end.
 //
 // Warp roles (320 threads):
 //   warp 0      producer: K, V once; per query tile Q, dO by TMA and the
@@ -54,7 +55,7 @@ struct Cfg {
   static constexpr int OFF_LSE = OFF_DS + 2 * BOX;           // NSQ x 128 floats
   static constexpr int OFF_DELTA = OFF_LSE + NSQ * 128 * 4;  // NSQ x 128 floats
   static constexpr int OFF_BAR = OFF_DELTA + NSQ * 128 * 4;
-  static constexpr int NBAR = 1 + 2 * NSQ + 7 + 4;
+  static constexpr int NBAR = 1 + 2 * NSQ + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_HOP = OFF_MISC + 16;
   static constexpr int SMEM = OFF_HOP + kMaxHops * 8;
@@ -96,8 +97,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const __grid_constant__ CUtensorMap tm_dq, const Params p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_dq_full = bar_a_free + 1;
   uint64_t* bar_dq_free = bar_dq_full + 1;
   uint64_t* bar_drain = bar_dq_free + 1;
-  uint64_t* bar_stg_full = bar_drain + 1;   // [2]: warpgroup's staged dQ chunk written
-  uint64_t* bar_stg_free = bar_stg_full + 2;  // [2]: warpgroup's staging buffer read by the TMA
+
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
@@ -153,10 +152,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_free, 256);
     mbar_init(bar_drain, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_stg_full[i], 128);
-      mbar_init(&bar_stg_free[i], 1);
-    }
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -210,7 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
-        prefetch_tensormap(&tm_dq);
         mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
         for (int b = 0; b < C::NBOX; ++b) {
           tma_load_4d(smem + C::OFF_K + b * C::BOX, &tm_k, bar_kv_full, b * 64, k0, s, bh);
@@ -332,8 +326,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qc0 = wg * 64;              // first query column of this warpgroup
     const uint32_t t_a = tmem + lane_base + C::T_A + wg * 64;
     uint8_t* sds = smem + C::OFF_DS + wg * C::BOX;
-    const bool leader = (warp & 3) == 2 && lane == 0;  // first warp of the warpgroup, lane 0
-    uint32_t n_chunks = 0;                              // dQ chunks staged so far
     bool ok = true;
     int it = 0;
     for (int t = 0; t < p.nseg && ok; ++t) {
@@ -395,12 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_base + C::T_B + qc0, dp[0]);
         tmem_ld32(tmem + lane_base + C::T_B + qc0 + 32, dp[1]);
         tmem_wait_ld();
-        // the previous tile's last dQ chunk must have left the staging buffer
-        if (n_chunks > 0 && !warp_wait(&bar_stg_free[wg], (n_chunks - 1) & 1, s_abort, p.wait_ns)) {
-          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
-          ok = false;
-          break;
-        }
+
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t pk[16];
@@ -425,43 +412,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar_ds_ready);
         // dQ read-out: this lane's query row, this warpgroup's half of D, in
-        // 32-column chunks staged (128-byte swizzled) in this warpgroup's half
-        // of the dS tile, which the dQ MMA has finished reading; the leader
-        // adds each chunk into the fp32 accumulator with a TMA reduce.
+        // 32-column chunks. Each warp stages its own 32 rows (128-byte
+        // swizzled) in its rows of this warpgroup's half of the dS tile (the
+        // dQ MMA has finished reading it), then reads them back so that one
+        // warp instruction covers four whole 128-byte rows of the fp32
+        // accumulator and adds them with coalesced vector reductions.
         if (!warp_wait(bar_dq_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
           ok = false;
           break;
         }
         tc_fence_after();
+        {
+          const int rsub = lane >> 3;         // row within a group of four
+          const int piece = lane & 7;         // 16-byte piece of a 128-byte row
+          const int wrow0 = quarter * 32;     // this warp's first row
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t g[32];
-          tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + c * 32, g);
-          tmem_wait_ld();
-          if (n_chunks > 0 && !warp_wait(&bar_stg_free[wg], (n_chunks - 1) & 1, s_abort, p.wait_ns)) {
-            if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
-            ok = false;
-            break;
-          }
-          uint8_t* rowp = sds + row * 128;
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t g[32];
+            tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + c * 32, g);
+            tmem_wait_ld();
+            uint8_t* rowp = sds + row * 128;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
-                make_uint4(g[4 * j], g[4 * j + 1], g[4 * j + 2], g[4 * j + 3]);
-          fence_proxy_async_smem();
-          mbar_arrive(&bar_stg_full[wg]);
-          if (leader) {
-            if (!mbar_wait(&bar_stg_full[wg], n_chunks & 1, s_abort, p.wait_ns)) {
-              record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
-            } else {
-              tma_reduce_add_4d(&tm_dq, sds, wg * (D / 2) + c * 32, i * BQ, r, bh);
-              bulk_commit();
-              bulk_wait_read0();  // staging may be overwritten once the TMA has read it
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
+                  make_uint4(g[4 * j], g[4 * j + 1], g[4 * j + 2], g[4 * j + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int rr = wrow0 + k * 4 + rsub;
+              const float4 val =
+                  *reinterpret_cast<const float4*>(sds + rr * 128 + ((piece ^ (rr & 7)) << 4));
+              const int q = i * BQ + rr;
+              if (q < p.Lseg)
+                atomicAdd(reinterpret_cast<float4*>(p.dq_acc + (rowbase + q) * D + wg * (D / 2) + c * 32 +
+                                                    piece * 4),
+                          val);
             }
-            mbar_arrive(&bar_stg_free[wg]);
+            __syncwarp();
           }
-          ++n_chunks;
         }
         if (!ok) break;
         tc_fence_before();
@@ -510,7 +499,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ------------------------------------------------------------ teardown
-  if (warp >= 2 && (warp & 3) == 2 && lane == 0) bulk_wait0();  // dQ reduces complete
   if (warp == 0 && lane == 0) {
     if (kv_issued) drain_wait(bar_kv_full, 0);
     for (int it = max(0, issued_q - C::NSQ); it < issued_q; ++it)
@@ -591,13 +579,12 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo;
   rattn_status st;
   if ((st = make_tmap_bf16(&tq, a.q, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
-  if ((st = make_tmap_f32(&tdq, a.dq_acc, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
   if ((st = set_smem_attr(reinterpret_cast<const void*>(&bwd_kernel<D>), C::SMEM)) != RATTN_OK) return st;
   Params p;
   p.lse = a.lse;
@@ -617,7 +604,7 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.dv = a.dv;
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
-  bwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq, p);
+  bwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   const long long n4 = rows * D / 4;
   dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),

@@ -40,11 +40,6 @@ constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,
                             int box_rows);
 
-// 4-D fp32 tensor map over [outer][nseg][rows][D] with a (32 x box_rows)
-// box (128 bytes wide) and 128-byte swizzle, for TMA reduce-adds.
-rattn_status make_tmap_f32(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,
-                           int box_rows);
-
 // Sets the max dynamic shared memory attribute of a kernel once per device.
 rattn_status set_smem_attr(const void* kernel, int bytes);
 
