@@ -147,10 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
-    mbar_init(bar_ds_ready, 256);
+    mbar_init(bar_ds_ready, 8);
     mbar_init(bar_a_free, 1);
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 256);
+    mbar_init(bar_dq_free, 8);
     mbar_init(bar_drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -410,7 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar_ds_ready);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ds_ready);  // one arrival per warp
         // dQ read-out: this lane's query row, this warpgroup's half of D, in
         // 32-column chunks. Each warp stages its own 32 rows (128-byte
         // swizzled) in its rows of this warpgroup's half of the dS tile (the
@@ -454,7 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         tc_fence_before();
-        mbar_arrive(bar_dq_free);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dq_free);  // one arrival per warp
       }
     }
     // ------------------------------------------------------ dK, dV out

@@ -17,13 +17,17 @@
 //               NS-stage ring of shared-memory buffers (the emulated KV hop:
 //               the next block's loads run while the current block's MMAs do);
 //   warp 1      allocates TMEM and issues tcgen05.mma from one thread:
-//               S_g = Q K_g^T into one of two TMEM score buffers, then
-//               O += P_{g-1} V_{g-1} with P read from TMEM;
+//               S_g = Q K_g^T into one of three TMEM score buffers, running
+//               three tiles ahead of O += P_g V_g (P read from TMEM), so the
+//               score MMAs never wait on the previous tile's softmax;
 //   warps 2..5  softmax, one thread per query row (= TMEM lane): row max,
 //               lazy rescale of O (only when the max grows by more than
 //               2^8), exp2, row sum, P packed to bf16 into TMEM; finally the
 //               epilogue O / l and LSE.
-// TMEM columns: S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384) O [384,384+D).
+// TMEM columns: S0 [0,128) S1 [128,256) S2 [256,384) O [384,384+D); P_g is
+// written over the first 64 columns of its own score buffer. The MMA that
+// next overwrites that buffer (S_{g+3}) is issued only after the PV MMA
+// reading P_g has completed.
 #include <math.h>
 
 #include "internal.h"
@@ -43,13 +47,14 @@ struct Cfg {
   static constexpr int TILE = BM * D * 2;  // bytes of one 128 x D bf16 tile
   static constexpr int NBOX = D / 64;      // 64-element (128-byte) swizzle boxes per row
   static constexpr int BOX = BM * 128;     // bytes of one 128-row box
-  static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_P0 = 256, T_P1 = 320, T_O = 384;
+  static constexpr int NSB = 3;  // TMEM score buffers; P_g is written over its own scores
+  static constexpr uint32_t T_O = 128 * NSB;
   static constexpr uint32_t T_COLS = 512;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE;
   static constexpr int OFF_V = OFF_K + NS * TILE;
   static constexpr int OFF_BAR = OFF_V + NS * TILE;
-  static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 1 + 1;
+  static constexpr int NBAR = 1 + 4 * NS + NSB + NSB + NSB + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_HOP = OFF_MISC + 16;
   static constexpr int SMEM = OFF_HOP + kMaxHops * 8 + 1024;  // + alignment slack
@@ -107,10 +112,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_k_empty = bar_k_full + C::NS;
   uint64_t* bar_v_full = bar_k_empty + C::NS;
   uint64_t* bar_v_empty = bar_v_full + C::NS;
-  uint64_t* bar_s_full = bar_v_empty + C::NS;
-  uint64_t* bar_p_ready = bar_s_full + 2;
-  uint64_t* bar_o_done = bar_p_ready + 2;
-  uint64_t* bar_drain = bar_o_done + 1;
+  uint64_t* bar_s_full = bar_v_empty + C::NS;     // [NSB]
+  uint64_t* bar_p_ready = bar_s_full + C::NSB;    // [NSB]
+  // o_done[b]: PV_g with g % NSB == b completed. A parity wait is only sound
+  // when the waiter knows the previous phase completed; with one barrier per
+  // score buffer that previous phase is PV_{g-NSB}, which every waiter has
+  // already observed (its S_g was issued after it).
+  uint64_t* bar_o_done = bar_p_ready + C::NSB;  // [NSB]
+  uint64_t* bar_drain = bar_o_done + C::NSB;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
@@ -140,11 +149,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_v_full[i], 1);
       mbar_init(&bar_v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NSB; ++i) {
       mbar_init(&bar_s_full[i], 1);
-      mbar_init(&bar_p_ready[i], 128);
+      mbar_init(&bar_p_ready[i], 4);  // one arrival per softmax warp
     }
-    mbar_init(bar_o_done, 1);
+    for (int i = 0; i < C::NSB; ++i) mbar_init(&bar_o_done[i], 1);
     mbar_init(bar_drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -230,33 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(bar_q_full, 0, s_abort, p.wait_ns);
       if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
 
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&bar_p_ready[j & 1], (j >> 1) & 1, s_abort, p.wait_ns)) return false;
-        const int st = j % C::NS;
-        if (!mbar_wait(&bar_v_full[st], (j / C::NS) & 1, s_abort, p.wait_ns)) return false;
-        tc_fence_after();
-        const uint32_t a_t = tmem + ((j & 1) ? C::T_P1 : C::T_P0);
-        const uint32_t sVa = smem_u32(sV + st * C::TILE);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
-          const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
-          umma_ts(tmem + C::T_O, a_t + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar_o_done);
-        umma_commit(&bar_v_empty[st]);
-        return true;
-      };
-
-      for (int g = 0; g < G && ok; ++g) {
+      // S_g = Q K_g^T into score buffer g % NSB
+      auto issue_s = [&](int g) -> bool {
         const int st = g % C::NS;
-        if (!mbar_wait(&bar_k_full[st], (g / C::NS) & 1, s_abort, p.wait_ns)) {
-          record_failure(s_abort, p.err, SITE_FWD_MMA);
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&bar_k_full[st], (g / C::NS) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t d_s = tmem + ((g & 1) ? C::T_S1 : C::T_S0);
+        const uint32_t d_s = tmem + (g % C::NSB) * 128;
         const uint32_t sKa = smem_u32(sK + st * C::TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -265,14 +253,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sdesc_sw128(sKa + off, 16, 1024);
           umma_ss(d_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bar_s_full[g & 1]);
+        umma_commit(&bar_s_full[g % C::NSB]);
         umma_commit(&bar_k_empty[st]);
-        if (g >= 1 && !issue_pv(g - 1)) {
-          record_failure(s_abort, p.err, SITE_FWD_MMA);
-          ok = false;
+        return true;
+      };
+      // O += P_j V_j with P_j read from the first 64 columns of its score buffer
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(&bar_p_ready[j % C::NSB], (j / C::NSB) & 1, s_abort, p.wait_ns)) return false;
+        const int st = j % C::NS;
+        if (!mbar_wait(&bar_v_full[st], (j / C::NS) & 1, s_abort, p.wait_ns)) return false;
+        tc_fence_after();
+        const uint32_t a_t = tmem + (j % C::NSB) * 128;
+        const uint32_t sVa = smem_u32(sV + st * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
+          const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
+          umma_ts(tmem + C::T_O, a_t + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&bar_o_done[j % C::NSB]);
+        umma_commit(&bar_v_empty[st]);
+        return true;
+      };
+
+      // S runs NSB tiles ahead of PV: S_0..S_{NSB-1}, then PV_g, S_{g+NSB}, ...
+      // S_{g+NSB} overwrites P_g's buffer, so it is issued only once PV_g has
+      // completed (issue order alone does not keep a later MMA's accumulator
+      // writes behind an earlier MMA's TMEM operand reads).
+      for (int g = 0; g < min(G, C::NSB) && ok; ++g) ok = issue_s(g);
+      for (int g = 0; g < G && ok; ++g) {
+        ok = issue_pv(g);
+        if (ok && g + C::NSB < G) {
+          ok = mbar_wait(&bar_o_done[g % C::NSB], (g / C::NSB) & 1, s_abort, p.wait_ns);
+          if (ok) ok = issue_s(g + C::NSB);
         }
       }
-      if (ok && !issue_pv(G - 1)) record_failure(s_abort, p.err, SITE_FWD_MMA);
+      if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
+
     }
   } else {
     // -------------------------------------------------- softmax + epilogue
@@ -289,14 +306,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
       const int nv = s_hop[t].x, nf = s_hop[t].y;
       for (int j = 0; j < nv; ++j, ++g) {
-        if (!warp_wait(&bar_s_full[g & 1], (g >> 1) & 1, s_abort, p.wait_ns)) {
+        if (!warp_wait(&bar_s_full[g % C::NSB], (g / C::NSB) & 1, s_abort, p.wait_ns)) {
           record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t sr[4][32];
-        const uint32_t s_addr = tmem + lane_base + ((g & 1) ? C::T_S1 : C::T_S0);
+        const uint32_t s_addr = tmem + lane_base + (g % C::NSB) * 128;
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
         tmem_wait_ld();
@@ -337,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool warp_rescale = __any_sync(0xffffffffu, need && o_live) != 0;
         if (need) m_run = mx;
         if (warp_rescale) {
-          if (!warp_wait(bar_o_done, (g - 1) & 1, s_abort, p.wait_ns)) {
+          if (!warp_wait(&bar_o_done[(g - 1) % C::NSB], ((g - 1) / C::NSB) & 1, s_abort, p.wait_ns)) {
             record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
             ok = false;
             break;
@@ -358,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sum8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
-        const uint32_t p_addr = tmem + lane_base + ((g & 1) ? C::T_P1 : C::T_P0);
+        const uint32_t p_addr = s_addr;  // P over the scores, all already in registers
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
@@ -375,7 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bar_p_ready[g & 1]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p_ready[g % C::NSB]);  // one arrival per warp
       }
     }
 
@@ -383,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long out_row = (static_cast<long long>(bh) * p.nseg + r) * p.Lq_seg + q0 + row;
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
     if (ok && G > 0) {
-      if (!warp_wait(bar_o_done, (G - 1) & 1, s_abort, p.wait_ns)) {
+      if (!warp_wait(&bar_o_done[(G - 1) % C::NSB], ((G - 1) / C::NSB) & 1, s_abort, p.wait_ns)) {
         record_failure(s_abort, p.err, SITE_FWD_EPILOGUE);
         ok = false;
       }

@@ -65,18 +65,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One probe that may suspend the thread for up to hint_ns nanoseconds while the
+// phase is incomplete; the hardware resumes it as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, "
+      "p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the barrier phase of the given parity has completed. Gives up
 // (returns false) after about limit_ns nanoseconds (counted in SM cycles at an
 // assumed 2 GHz) or as soon as *abort is set, so a lost arrival can never hang
-// the GPU. The limit and the abort flag are checked on the first retry and
-// then every 64 polls, to keep the poll loop short.
+// the GPU. Waiting threads sleep in the probe (up to 1 ms, or the limit when
+// that is shorter) instead of spinning, so they do not steal issue slots from
+// the warps doing the work; the limit and the abort flag are checked on the
+// first retry and then every 64 probes.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = static_cast<uint32_t>(limit_ns < 1000000ull ? limit_ns : 1000000ull);
   const long long t0 = clock64();
   const long long limit_cycles = static_cast<long long>(limit_ns < (1ull << 61) ? limit_ns * 2 : (1ull << 62));
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_hint(bar, parity, hint)) return true;
     if ((i & 63u) == 1u) {
       if (*abort) return false;
       if (clock64() - t0 > limit_cycles) return false;
