@@ -8,6 +8,7 @@
 //
 // Both kernels are gathers: each thread moves 16-byte vectors of one output
 // row, so stores are fully coalesced and loads are coalesced within a row.
+// Rows wider than 4 KB (256 vectors) are not supported.
 #include "internal.h"
 
 namespace rattn {
@@ -29,44 +30,57 @@ __device__ __forceinline__ int global_to_slot(int g, int c, int cp, int layout) 
   return k < cp ? k * 2 * c + j : (2 * cp - 1 - k) * 2 * c + c + j;
 }
 
+// Thread layout: vpr consecutive threads move one row (vpr = row bytes / 16),
+// blockDim.x / vpr rows per block step; blockIdx.y walks (batch, head). All
+// per-vector index math is 32-bit; only the final offsets are 64-bit.
 __global__ void permute_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, int32_t* __restrict__ pos,
-                               int BH, int L, int Lp, int vec_per_row, int c, int cp, int layout) {
-  const long long total = static_cast<long long>(BH) * Lp * vec_per_row;
-  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < total;
-       v += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = v / vec_per_row;
-    const int e = static_cast<int>(v - row * vec_per_row);
-    const int bh = static_cast<int>(row / Lp);
-    const int i = static_cast<int>(row - static_cast<long long>(bh) * Lp);
-    const int g = slot_to_global(i, c, cp, layout);
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (g < L) val = __ldg(x + (static_cast<long long>(bh) * L + g) * vec_per_row + e);
-    y[v] = val;
-    if (pos && bh == 0 && e == 0) pos[i] = g;
+                               int BH, int L, int Lp, int vpr, int c, int cp, int layout) {
+  const int e = threadIdx.x % vpr;
+  const int rsub = threadIdx.x / vpr;
+  const int rpb = blockDim.x / vpr;
+  if (rsub >= rpb) return;
+  for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+    const uint4* xb = x + static_cast<long long>(bh) * L * vpr;
+    uint4* yb = y + static_cast<long long>(bh) * Lp * vpr;
+    for (int i = blockIdx.x * rpb + rsub; i < Lp; i += gridDim.x * rpb) {
+      const int g = slot_to_global(i, c, cp, layout);
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (g < L) val = __ldg(xb + static_cast<long long>(g) * vpr + e);
+      yb[static_cast<long long>(i) * vpr + e] = val;
+      if (pos && bh == 0 && e == 0) pos[i] = g;
+    }
   }
 }
 
 __global__ void unpermute_kernel(const uint4* __restrict__ y, uint4* __restrict__ x, int BH, int L, int Lp,
-                                 int vec_per_row, int c, int cp, int layout) {
-  const long long total = static_cast<long long>(BH) * L * vec_per_row;
-  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < total;
-       v += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = v / vec_per_row;
-    const int e = static_cast<int>(v - row * vec_per_row);
-    const int bh = static_cast<int>(row / L);
-    const int g = static_cast<int>(row - static_cast<long long>(bh) * L);
-    const int i = global_to_slot(g, c, cp, layout);
-    x[v] = __ldg(y + (static_cast<long long>(bh) * Lp + i) * vec_per_row + e);
+                                 int vpr, int c, int cp, int layout) {
+  const int e = threadIdx.x % vpr;
+  const int rsub = threadIdx.x / vpr;
+  const int rpb = blockDim.x / vpr;
+  if (rsub >= rpb) return;
+  for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+    const uint4* yb = y + static_cast<long long>(bh) * Lp * vpr;
+    uint4* xb = x + static_cast<long long>(bh) * L * vpr;
+    for (int g = blockIdx.x * rpb + rsub; g < L; g += gridDim.x * rpb) {
+      const int i = global_to_slot(g, c, cp, layout);
+      xb[static_cast<long long>(g) * vpr + e] = __ldg(yb + static_cast<long long>(i) * vpr + e);
+    }
   }
 }
 
-unsigned grid_for(long long work, int threads) {
+// Grid for rows x BH work items: about 16 resident 256-thread blocks per SM.
+dim3 grid_2d(long long rows, int BH, int rpb) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long want = (work + threads - 1) / threads;
-  const long long cap = static_cast<long long>(sms) * 16;  // 16 resident 256-thread CTAs per SM
-  return static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap);
+  const int gy = BH < 65535 ? BH : 65535;
+  const long long want_total = static_cast<long long>(sms) * 16;
+  long long gx = (want_total + gy - 1) / gy;
+  const long long row_blocks = (rows + rpb - 1) / rpb;
+  if (gx > row_blocks) gx = row_blocks;
+  if (gx < 1) gx = 1;
+  return dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 1);
 }
+
 
 }  // namespace
 
@@ -75,10 +89,10 @@ rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_
   const int vpr = row_bytes / 16;
   const int nchunks = layout == RATTN_LAYOUT_HEAD_TAIL ? 2 * cp : cp;
   const int c = static_cast<int>(Lp / nchunks);
-  const long long total = static_cast<long long>(BH) * Lp * vpr;
-  permute_kernel<<<grid_for(total, 256), 256, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), pos,
-                                                           BH, static_cast<int>(L), static_cast<int>(Lp), vpr, c, cp,
-                                                           layout);
+  if (vpr > 256) return RATTN_ERR_UNSUPPORTED;
+  permute_kernel<<<grid_2d(Lp, BH, 256 / vpr), 256, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
+                                                                 pos, BH, static_cast<int>(L), static_cast<int>(Lp),
+                                                                 vpr, c, cp, layout);
   return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
@@ -87,10 +101,10 @@ rattn_status launch_unpermute(const void* y, void* x, int BH, int64_t L, int64_t
   const int vpr = row_bytes / 16;
   const int nchunks = layout == RATTN_LAYOUT_HEAD_TAIL ? 2 * cp : cp;
   const int c = static_cast<int>(Lp / nchunks);
-  const long long total = static_cast<long long>(BH) * L * vpr;
-  unpermute_kernel<<<grid_for(total, 256), 256, 0, stream>>>(static_cast<const uint4*>(y), static_cast<uint4*>(x),
-                                                             BH, static_cast<int>(L), static_cast<int>(Lp), vpr, c,
-                                                             cp, layout);
+  if (vpr > 256) return RATTN_ERR_UNSUPPORTED;
+  unpermute_kernel<<<grid_2d(L, BH, 256 / vpr), 256, 0, stream>>>(static_cast<const uint4*>(y),
+                                                                  static_cast<uint4*>(x), BH, static_cast<int>(L),
+                                                                  static_cast<int>(Lp), vpr, c, cp, layout);
   return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
 }
 

@@ -84,6 +84,7 @@ int64_t cp_layout_padded_len(int64_t L, int cp_size, rattn_layout layout);
  * rows (global index >= L) zero-filled. If pos is non-NULL it receives the
  * global position id of every slot, int32 [Lp], shared by all (b, h); pad
  * slots carry L, L+1, ... Lp must equal cp_layout_padded_len(L, cp, layout).
+ * Rows must be a multiple of 16 bytes and at most 4 KB (D * sizeof(dtype)).
  * Bit-exact copy. x and y must not overlap. */
 rattn_status cp_layout_permute(const void* x, void* y, int32_t* pos,
                                int B, int H, int64_t L, int64_t Lp, int D,
