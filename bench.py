@@ -36,7 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launch by sequence length (traffic grows with the tensors). Source:
 # profiles/bwd_kernel_bf16_H32_L16000_cp4.md. Set to None when the kernel
 # changes until it is captured again.
-NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": (791.8e6 + 479.9e6) * 2}
+NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": (791.7e6 + 486.1e6) * 2}
 
 
 def peaks():
@@ -155,7 +155,8 @@ def run_ours(args, w, rank, world, local):
     ws = torch.empty(max(rattn.rattn_ring_bwd_workspace_size(B, H, Lp, D), 1), dtype=torch.uint8, device=dev)
     fwd_ev, bwd_ev = [], []
 
-    def step(x, timed=False):
+    def step(x, outs=None, timed=False):
+        outs = out if outs is None else outs
         xq, xk, xv, xdo = x
         rattn.cp_layout_permute(xq, cp, layout, y=pbuf["q"], pos=pos)
         rattn.cp_layout_permute(xk, cp, layout, y=pbuf["k"], pos=pos)
@@ -169,7 +170,7 @@ def run_ours(args, w, rank, world, local):
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
             fwd_ev.append((e0, e1))
-        rattn.cp_layout_unpermute(pbuf["o"], L, cp, layout, x=out["o"])
+        rattn.cp_layout_unpermute(pbuf["o"], L, cp, layout, x=outs["o"])
         if w.bwd:
             rattn.cp_layout_permute(xdo, cp, layout, y=pbuf["do"], pos=pos)
             if timed:
@@ -183,7 +184,7 @@ def run_ours(args, w, rank, world, local):
                 e3.record(stream)
                 bwd_ev.append((e2, e3))
             for g, name in zip(grads_p, ("dq", "dk", "dv")):
-                rattn.cp_layout_unpermute(g, L, cp, layout, x=out[name])
+                rattn.cp_layout_unpermute(g, L, cp, layout, x=outs[name])
 
     launches_per_step = 3 + 1 + 1 + ((1 + 3 + 3) if w.bwd else 0)
     x = (q, k, v, do)
@@ -209,30 +210,60 @@ def run_ours(args, w, rank, world, local):
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
     bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev) if bwd_ev else None
 
-    # End to end through the public API with host buffers: pinned H2D of the
-    # step's inputs, the step, D2H of its results (O, dQ, dK, dV).
+    # End to end through the public API with host buffers: every step copies
+    # its inputs (Q, K, V, dO) from pinned host memory and reads its results
+    # (O, dQ, dK, dV) back, all inside the timed region. Steps are pipelined
+    # over three streams with two device buffer sets: step i+1's uploads and
+    # step i-1's downloads overlap step i's kernels.
+    names = ("o", "dq", "dk", "dv") if w.bwd else ("o",)
     host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
-    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in out.items()}
-    dev_in = [torch.empty_like(t) for t in (q, k, v, do)]
-    h2d = sum(t.numel() * t.element_size() for t in host_in[:4 if w.bwd else 3])
-    d2h = sum(host_out[n].numel() * host_out[n].element_size() for n in (("o", "dq", "dk", "dv") if w.bwd else ("o",)))
+    n_in = 4 if w.bwd else 3
+    host_out = [{n: torch.empty(out[n].shape, dtype=out[n].dtype, pin_memory=True) for n in names}
+                for _ in range(2)]
+    dev_in = [[torch.empty_like(t) for t in (q, k, v, do)] for _ in range(2)]
+    dev_out = [{n: torch.empty_like(out[n]) for n in out} for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in[:n_in])
+    d2h = sum(host_out[0][n].numel() * host_out[0][n].element_size() for n in names)
+    s_h2d, s_comp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for h, d in zip(host_in, dev_in):
-            d.copy_(h, non_blocking=True)
-        step(tuple(dev_in))
-        for n in (("o", "dq", "dk", "dv") if w.bwd else ("o",)):
-            host_out[n].copy_(out[n], non_blocking=True)
+    def e2e_steps(n, start_event):
+        for st in (s_h2d, s_comp, s_d2h):
+            st.wait_event(start_event)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_h2d):
+                if i >= 2:
+                    s_h2d.wait_event(ev_comp[b])      # dev_in[b] no longer read
+                for h, d in zip(host_in[:n_in], dev_in[b][:n_in]):
+                    d.copy_(h, non_blocking=True)
+                ev_in[b].record(s_h2d)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[b])
+                if i >= 2:
+                    s_comp.wait_event(ev_out[b])     # dev_out[b] already read back
+                step(tuple(dev_in[b]), dev_out[b])
+                ev_comp[b].record(s_comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_comp[b])
+                for nm in names:
+                    host_out[b][nm].copy_(dev_out[b][nm], non_blocking=True)
+                ev_out[b].record(s_d2h)
+        return ev_out[(n - 1) % 2]
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    w0 = torch.cuda.Event()
+    w0.record(stream)
+    last = e2e_steps(max(1, args.warmup), w0)
+    stream.wait_event(last)
     torch.cuda.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    last = e2e_steps(args.steps, e0)
+    stream.wait_event(last)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
@@ -240,23 +271,39 @@ def run_ours(args, w, rank, world, local):
             "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps}
 
 
-def cpu_sample_run(w, seconds_hint=True):
-    """The oracle as it stands on a bounded sample: one head, the first 8000
-    tokens (one emulated rank's worth), causal fwd + bwd, fp64 on the host."""
+def cpu_sample_run(w, min_seconds=0.0):
+    """The oracle as it stands on a bounded sample: the first 8000 tokens (one
+    emulated rank's worth) of one head, causal fwd (+ bwd), fp64 on the host;
+    further heads are added until at least ``min_seconds`` of CPU work ran."""
     import numpy as np
     import oracle
     Ls = min(8000, w.L)
     g = torch.Generator().manual_seed(0)
-    q, k, v, do = (torch.randn(Ls, w.D, generator=g).to(w.torch_dtype).double().numpy() for _ in range(4))
-    t0 = time.perf_counter()
-    oracle.attention(q, k, v, w.scale, w.causal, row_block=1000)
-    if w.bwd:
-        oracle.attention_bwd(q, k, v, do, w.scale, w.causal, row_block=1000)
-    dt = time.perf_counter() - t0
-    fl = 4.0 * w.D * Ls * Ls * (0.5 if w.causal else 1.0) * (3.5 if w.bwd else 1.0)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"1 head x first {Ls} tokens, {'fwd+bwd' if w.bwd else 'fwd'}, numpy fp64 "
-                      f"(BLAS threads {os.environ.get('OPENBLAS_NUM_THREADS', 'default')}), {dt:.2f} s"}
+    heads, dt = 0, 0.0
+    while heads < w.B * w.H and (heads == 0 or dt < min_seconds):
+        q, k, v, do = (torch.randn(Ls, w.D, generator=g).to(w.torch_dtype).double().numpy() for _ in range(4))
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, w.scale, w.causal, row_block=1000)
+        if w.bwd:
+            oracle.attention_bwd(q, k, v, do, w.scale, w.causal, row_block=1000)
+        dt += time.perf_counter() - t0
+        heads += 1
+    fl = heads * 4.0 * w.D * Ls * Ls * (0.5 if w.causal else 1.0) * (3.5 if w.bwd else 1.0)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{heads} head(s) x first {Ls} tokens, {'fwd+bwd' if w.bwd else 'fwd'}, numpy fp64 "
+                      f"BLAS, {dt:.2f} s"}
+
+
+def blas_threads():
+    """Threads the oracle's BLAS runs with (its matmuls are where the time goes)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
 
 
 def main():
@@ -270,7 +317,7 @@ def main():
     w = WORKLOADS[args.workload]
     flops_step, fwd_flops = step_flops(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "cp": w.cp,
-              "layout": "head_tail" if w.layout == 1 else "contiguous", "causal": w.causal,
+              "layout": ("contiguous", "head_tail", "striped")[w.layout], "causal": w.causal,
               "step": "permute q,k,v" + (",dO" if w.bwd else "") + " -> ring fwd -> unpermute O" +
                       (" -> ring bwd -> unpermute dQ,dK,dV" if w.bwd else ""),
               "l2": "inputs larger than L2 (%.0f MB per tensor vs 126 MB)" % (w.B * w.H * w.L * w.D * 2 / 1e6),
@@ -325,7 +372,7 @@ def main():
     }
     if rank == 0:
         if world == 1:
-            line["cpu_baseline"] = cpu_sample_run(w)
+            line["cpu_baseline"] = cpu_sample_run(w, min_seconds=10.0)
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
