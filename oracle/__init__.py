@@ -20,17 +20,21 @@ Sources (cited by page title and section):
   * aiunderstanding.org, "Sequence parallelism and ring attention" --
     sections "Deep dive" and "Technical insight" (online softmax: running max
     and running normaliser, earlier partial sums rescaled; exact result).
+  * RoPE at carried global positions (``rotary.py``): the same Megatron blog
+    section says rotary embeddings must use the global positions of the
+    chunks a rank holds; the rotation is the published RoFormer definition.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 (brute force, closed forms, library special cases, invariants, the page's
 rank/chunk table). No function is "parity unpinned".
 """
-from .layout import CONTIGUOUS, HEAD_TAIL, padded_len, perm_index, permute, unpermute, rank_chunks
+from .layout import CONTIGUOUS, HEAD_TAIL, STRIPED, padded_len, perm_index, permute, unpermute, rank_chunks
 from .attn import (attention, merge, ring_emulate, blockwise_attention,
                         attention_bwd, visible_mask, causal_pairs_per_rank)
+from .rotary import HALF as ROPE_HALF, INTERLEAVED as ROPE_INTERLEAVED, rope, rope_grad
 
 __all__ = [
-    "CONTIGUOUS", "HEAD_TAIL", "padded_len", "perm_index", "permute", "unpermute", "rank_chunks",
+    "CONTIGUOUS", "HEAD_TAIL", "STRIPED", "padded_len", "perm_index", "permute", "unpermute", "rank_chunks",
     "attention", "merge", "ring_emulate", "blockwise_attention", "attention_bwd", "visible_mask",
-    "causal_pairs_per_rank",
+    "causal_pairs_per_rank", "ROPE_HALF", "ROPE_INTERLEAVED", "rope", "rope_grad",
 ]

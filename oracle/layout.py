@@ -10,6 +10,13 @@ section "Symmetric chunk assignment":
 The contiguous ("naive") layout is the left half of that section's figure
 caption: rank r holds the r-th of cp_size contiguous pieces.
 
+The striped layout follows the page "Sequence parallelism and ring attention"
+(aiunderstanding.org), section on the future of sequence parallelism, which
+names striped attention as a variant that rebalances the causal work; the
+reading taken is the published Striped Attention assignment (Brandon et al.,
+2023): token g goes to rank g mod cp_size, each rank keeping its tokens in
+increasing order, and the length is padded to a multiple of cp_size.
+
 Readings where the page is silent: padding goes at the tail of the global
 sequence, pad slots carry the positions L, L+1, ... they would have in the
 padded sequence, and pad values are zero. Ranks are concatenated in rank order.
@@ -18,6 +25,7 @@ import numpy as np
 
 CONTIGUOUS = 0
 HEAD_TAIL = 1
+STRIPED = 2
 
 
 def _n_chunks(cp, layout):
@@ -25,13 +33,14 @@ def _n_chunks(cp, layout):
         raise ValueError("cp_size must be >= 1")
     if layout == HEAD_TAIL:
         return 2 * cp
-    if layout == CONTIGUOUS:
+    if layout in (CONTIGUOUS, STRIPED):
         return cp
     raise ValueError("unknown layout")
 
 
 def padded_len(L, cp, layout):
-    """Smallest Lp >= L that splits into equal chunks (2*cp of them for head-tail)."""
+    """Smallest Lp >= L that splits into equal chunks (2*cp of them for
+    head-tail, cp for contiguous; striped needs the same cp equal shares)."""
     n = _n_chunks(cp, layout)
     if L < 0:
         raise ValueError("L must be >= 0")
@@ -39,7 +48,10 @@ def padded_len(L, cp, layout):
 
 
 def rank_chunks(cp, layout):
-    """List, per rank, of the global chunk indices it holds, in local order."""
+    """List, per rank, of the global chunk indices it holds, in local order
+    (chunked layouts only)."""
+    if layout == STRIPED:
+        raise ValueError("the striped layout is not made of chunks")
     if layout == HEAD_TAIL:
         return [[r, 2 * cp - 1 - r] for r in range(cp)]
     _n_chunks(cp, layout)
@@ -55,6 +67,11 @@ def perm_index(L, cp, layout):
     Lp = padded_len(L, cp, layout)
     n = _n_chunks(cp, layout)
     c = Lp // n
+    if layout == STRIPED:
+        # rank r's tokens are r, r + cp, r + 2 cp, ... (c = Lp / cp of them)
+        pos = np.array([j * cp + r for r in range(cp) for j in range(c)], dtype=np.int64)
+        src = np.where(pos < L, pos, -1)
+        return Lp, src, pos
     chunks = [np.arange(k * c, (k + 1) * c, dtype=np.int64) for k in range(n)]
     pieces = [chunks[k] for owned in rank_chunks(cp, layout) for k in owned]
     pos = np.concatenate(pieces) if pieces else np.zeros(0, np.int64)

@@ -155,7 +155,7 @@ def test_blockwise_any_chunking_equals_full(trial):
 
 
 @pytest.mark.parametrize("cp", [1, 2, 3, 4])
-@pytest.mark.parametrize("layout", [oracle.HEAD_TAIL, oracle.CONTIGUOUS])
+@pytest.mark.parametrize("layout", [oracle.HEAD_TAIL, oracle.CONTIGUOUS, oracle.STRIPED])
 @pytest.mark.parametrize("causal", [True, False])
 def test_ring_equals_full_and_is_layout_invariant(cp, layout, causal):
     L, D = 29, 4

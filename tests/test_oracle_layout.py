@@ -3,7 +3,9 @@
 Pinned to: the rank/chunk table the Megatron CP blog prints for cp_size = 4
 (tests/golden/head_tail_cp4.txt), the padding rule and the global-position
 rule of the same section, and brute-force properties (bijection, inverse,
-equal causal work per rank under head-tail).
+equal causal work per rank under head-tail). The striped layout is pinned to
+its definition (token g on rank g mod cp) and to the closed form of its
+per-rank causal work.
 """
 import os
 
@@ -46,7 +48,7 @@ def test_head_tail_slots_follow_table_cp4(c):
 @pytest.mark.parametrize("cp", list(range(1, 17)))
 @pytest.mark.parametrize("L", [0, 1, 7, 64, 97, 256])
 def test_bijection_padding_and_inverse(cp, L):
-    for layout in (oracle.HEAD_TAIL, oracle.CONTIGUOUS):
+    for layout in (oracle.HEAD_TAIL, oracle.CONTIGUOUS, oracle.STRIPED):
         Lp, src, pos = oracle.perm_index(L, cp, layout)
         m = 2 * cp if layout == oracle.HEAD_TAIL else cp
         assert Lp % m == 0 and Lp >= L and Lp - L < m
@@ -89,6 +91,34 @@ def test_head_tail_balances_causal_work(cp, c):
     naive = oracle.causal_pairs_per_rank(L, cp, oracle.CONTIGUOUS)
     assert all(a < b for a, b in zip(naive, naive[1:]))          # contiguous is imbalanced
     assert sum(naive) == sum(counts) == L * (L + 1) // 2
+
+
+@pytest.mark.parametrize("cp", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("L", [1, 10, 64, 97])
+def test_striped_token_g_on_rank_g_mod_cp(cp, L):
+    Lp, src, pos = oracle.perm_index(L, cp, oracle.STRIPED)
+    n = Lp // cp
+    assert Lp % cp == 0 and Lp - L < cp
+    for r in range(cp):
+        local = pos[r * n:(r + 1) * n]
+        assert np.all(local % cp == r)
+        assert local[0] == r and np.all(np.diff(local) == cp)   # increasing, stride cp
+
+
+@pytest.mark.parametrize("cp,n", [(2, 3), (3, 4), (4, 5), (8, 2)])
+def test_striped_causal_work_closed_form(cp, n):
+    # query j*cp + r sees j*cp + r + 1 keys; summed over j = 0..n-1
+    L = cp * n
+    counts = oracle.causal_pairs_per_rank(L, cp, oracle.STRIPED)
+    assert counts == [cp * n * (n - 1) // 2 + n * (r + 1) for r in range(cp)]
+    assert sum(counts) == L * (L + 1) // 2
+    naive = oracle.causal_pairs_per_rank(L, cp, oracle.CONTIGUOUS)
+    assert max(counts) - min(counts) == n * (cp - 1) <= max(naive) - min(naive)
+
+
+def test_striped_has_no_chunks():
+    with pytest.raises(ValueError):
+        oracle.rank_chunks(4, oracle.STRIPED)
 
 
 def test_invalid_arguments():
