@@ -30,11 +30,11 @@ rank/chunk table). No function is "parity unpinned".
 """
 from .layout import CONTIGUOUS, HEAD_TAIL, STRIPED, padded_len, perm_index, permute, unpermute, rank_chunks
 from .attn import (attention, merge, ring_emulate, blockwise_attention,
-                        attention_bwd, visible_mask, causal_pairs_per_rank)
+                        attention_bwd, visible_mask, causal_pairs_per_rank, gqa_expand, gqa_reduce)
 from .rotary import HALF as ROPE_HALF, INTERLEAVED as ROPE_INTERLEAVED, rope, rope_grad
 
 __all__ = [
     "CONTIGUOUS", "HEAD_TAIL", "STRIPED", "padded_len", "perm_index", "permute", "unpermute", "rank_chunks",
     "attention", "merge", "ring_emulate", "blockwise_attention", "attention_bwd", "visible_mask",
-    "causal_pairs_per_rank", "ROPE_HALF", "ROPE_INTERLEAVED", "rope", "rope_grad",
+    "causal_pairs_per_rank", "gqa_expand", "gqa_reduce", "ROPE_HALF", "ROPE_INTERLEAVED", "rope", "rope_grad",
 ]

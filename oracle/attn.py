@@ -212,3 +212,31 @@ def causal_pairs_per_rank(L, cp, layout):
         counts.append(tot)
     return counts
 
+
+
+def gqa_expand(x, H):
+    """Grouped key/value heads seen by the query heads: x [B, H_kv, L, D] ->
+    [B, H, L, D], query head h reading key/value head h // (H / H_kv).
+
+    The blog "Context Parallelism v.s. Sequence Parallelism (Megatron-LM)",
+    section "CP vs SP", sizes the ring's traffic by H_kv, the number of
+    key/value heads, which is below H under grouped-query attention (GQA,
+    Ainslie et al., 2023: query heads split into H_kv equal groups, each group
+    sharing one key/value head). Reading: groups are contiguous runs of query
+    heads."""
+    x = np.asarray(x)
+    H_kv = x.shape[-3]
+    if H_kv < 1 or H % H_kv:
+        raise ValueError("H must be a positive multiple of H_kv")
+    return np.repeat(x, H // H_kv, axis=-3)
+
+
+def gqa_reduce(dx, H_kv):
+    """Gradient of ``gqa_expand``: [B, H, L, D] -> [B, H_kv, L, D], summing
+    the gradients of the query heads of each group."""
+    dx = np.asarray(dx, dtype=np.float64)
+    H = dx.shape[-3]
+    if H_kv < 1 or H % H_kv:
+        raise ValueError("H must be a positive multiple of H_kv")
+    g = H // H_kv
+    return dx.reshape(dx.shape[:-3] + (H_kv, g) + dx.shape[-2:]).sum(axis=-3)

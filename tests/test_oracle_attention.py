@@ -218,6 +218,44 @@ def test_bwd_matches_torch_autograd_fp64(causal):
         np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
 
 
+# ---- grouped key/value heads (GQA) ------------------------------------------
+
+@pytest.mark.parametrize("H,H_kv", [(4, 2), (6, 3), (4, 1), (3, 3)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_gqa_matches_torch_sdpa_enable_gqa(H, H_kv, causal):
+    """torch's SDPA with enable_gqa=True (fp64, math backend) and its autograd
+    against the oracle's attention on expanded K/V heads and the gradient
+    reduced over each group."""
+    B, L, D = 2, 21, 8
+    q, do = (RNG.standard_normal((B, H, L, D)) for _ in range(2))
+    k, v = (RNG.standard_normal((B, H_kv, L, D)) for _ in range(2))
+    scale = 0.4
+    ke, ve = oracle.gqa_expand(k, H), oracle.gqa_expand(v, H)
+    o, lse = oracle.attention(q, ke, ve, scale, causal, row_block=5)
+    dq, dke, dve = oracle.attention_bwd(q, ke, ve, do, scale, causal, row_block=5)
+    dk, dv = oracle.gqa_reduce(dke, H_kv), oracle.gqa_reduce(dve, H_kv)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+        ot = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale,
+                                                              enable_gqa=True)
+    ot.backward(torch.from_numpy(do))
+    np.testing.assert_allclose(o, ot.detach().numpy(), rtol=0, atol=1e-12)
+    for got, ref in zip((dq, dk, dv), (tq.grad, tk.grad, tv.grad)):
+        assert got.shape == ref.shape
+        np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_gqa_group_membership_and_identity():
+    k = RNG.standard_normal((1, 3, 4, 2))
+    e = oracle.gqa_expand(k, 6)
+    for h in range(6):
+        assert np.array_equal(e[0, h], k[0, h // 2])      # contiguous groups of 2
+    assert np.array_equal(oracle.gqa_expand(k, 3), k)
+    assert np.array_equal(oracle.gqa_reduce(e, 3), 2 * k)  # each head counted once per group member
+    with pytest.raises(ValueError):
+        oracle.gqa_expand(k, 4)
+
+
 # ---- the pins catch planted mistakes ---------------------------------------
 
 _ORIG_2D = oatt._attention_2d
