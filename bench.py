@@ -31,6 +31,7 @@ from context_ring_attention_emulated_b200.workloads import WORKLOADS, make_qkv, 
 METRIC = "ring-attn fwd/bwd TFLOP/s (causal FLOPs) on 1 B200; % of BF16 tensor peak"
 DEFAULT = "bf16_L32000_cp4_fwdbwd"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ROPE_BASE = 10000.0  # rotary base of the RoPE workloads (RoFormer's value)
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernel on a half-length case, scaled to the full
 # launch by sequence length (traffic grows with the tensors). Source:
@@ -145,46 +146,61 @@ def run_ours(args, w, rank, world, local):
     q, k, v = make_qkv(w, dev, seed=0)
     do = make_unit_grad(w, dev, seed=1)
     L, cp, layout = w.L, w.cp, w.layout
-    B, H, D = w.B, w.H, w.D
+    B, H, D, Hkv = w.B, w.H, w.D, w.kv_heads
+    heads = {"q": H, "k": Hkv, "v": Hkv, "do": H, "o": H, "dq": H, "dk": Hkv, "dv": Hkv}
     Lp = rattn.cp_layout_padded_len(L, cp, layout)
-    pbuf = {n: torch.empty(B, H, Lp, D, dtype=q.dtype, device=dev) for n in ("q", "k", "v", "do", "o")}
+    pbuf = {n: torch.empty(B, heads[n], Lp, D, dtype=q.dtype, device=dev) for n in ("q", "k", "v", "do", "o")}
     pos = torch.empty(Lp, dtype=torch.int32, device=dev)
     lse = torch.empty(B, H, Lp, dtype=torch.float32, device=dev)
-    grads_p = [torch.empty(B, H, Lp, D, dtype=q.dtype, device=dev) for _ in range(3)]
-    out = {n: torch.empty(B, H, L, D, dtype=q.dtype, device=dev) for n in ("o", "dq", "dk", "dv")}
+    grads_p = [torch.empty(B, heads[n], Lp, D, dtype=q.dtype, device=dev) for n in ("dq", "dk", "dv")]
+    out = {n: torch.empty(B, heads[n], L, D, dtype=q.dtype, device=dev) for n in ("o", "dq", "dk", "dv")}
+    ring_fwd = rattn.rattn_ring_fwd_gqa if Hkv != H else rattn.rattn_ring_fwd
+    ring_bwd = rattn.rattn_ring_bwd_gqa if Hkv != H else rattn.rattn_ring_bwd
+
+    def permute_in(x, name):
+        if w.rope and name in ("q", "k"):
+            rattn.cp_layout_permute_rope(x, cp, layout, ROPE_BASE, rattn.ROPE_HALF, y=pbuf[name], pos=pos)
+        else:
+            rattn.cp_layout_permute(x, cp, layout, y=pbuf[name], pos=pos)
+
+    def unpermute_grad(g, name, outs):
+        if w.rope and name in ("dq", "dk"):
+            rattn.cp_layout_unpermute_rope_grad(g, L, cp, layout, ROPE_BASE, rattn.ROPE_HALF, dx=outs[name])
+        else:
+            rattn.cp_layout_unpermute(g, L, cp, layout, x=outs[name])
     ws = torch.empty(max(rattn.rattn_ring_bwd_workspace_size(B, H, Lp, D), 1), dtype=torch.uint8, device=dev)
     fwd_ev, bwd_ev = [], []
 
     def step(x, outs=None, timed=False):
         outs = out if outs is None else outs
         xq, xk, xv, xdo = x
-        rattn.cp_layout_permute(xq, cp, layout, y=pbuf["q"], pos=pos)
-        rattn.cp_layout_permute(xk, cp, layout, y=pbuf["k"], pos=pos)
-        rattn.cp_layout_permute(xv, cp, layout, y=pbuf["v"], pos=pos)
+        permute_in(xq, "q")
+        permute_in(xk, "k")
+        permute_in(xv, "v")
         if timed:
             e0 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        rattn.rattn_ring_fwd(pbuf["q"], pbuf["k"], pbuf["v"], pos, cp, layout, w.causal, w.scale, L_valid=L,
-                             o=pbuf["o"], lse=lse)
+        ring_fwd(pbuf["q"], pbuf["k"], pbuf["v"], pos, cp, layout, w.causal, w.scale, L_valid=L,
+                 o=pbuf["o"], lse=lse)
         if timed:
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
             fwd_ev.append((e0, e1))
         rattn.cp_layout_unpermute(pbuf["o"], L, cp, layout, x=outs["o"])
         if w.bwd:
-            rattn.cp_layout_permute(xdo, cp, layout, y=pbuf["do"], pos=pos)
+            permute_in(xdo, "do")
             if timed:
                 e2 = torch.cuda.Event(enable_timing=True)
                 e2.record(stream)
-            rattn.rattn_ring_bwd(pbuf["q"], pbuf["k"], pbuf["v"], pbuf["o"], pbuf["do"], lse, pos, cp, layout,
-                                 w.causal, w.scale, L_valid=L, dq=grads_p[0], dk=grads_p[1], dv=grads_p[2],
-                                 workspace=ws)
+            ring_bwd(pbuf["q"], pbuf["k"], pbuf["v"], pbuf["o"], pbuf["do"], lse, pos, cp, layout,
+                     w.causal, w.scale, L_valid=L, dq=grads_p[0], dk=grads_p[1], dv=grads_p[2],
+                     workspace=ws)
             if timed:
                 e3 = torch.cuda.Event(enable_timing=True)
                 e3.record(stream)
                 bwd_ev.append((e2, e3))
             for g, name in zip(grads_p, ("dq", "dk", "dv")):
-                rattn.cp_layout_unpermute(g, L, cp, layout, x=outs[name])
+                unpermute_grad(g, name, outs)
 
     launches_per_step = 3 + 1 + 1 + ((1 + 3 + 3) if w.bwd else 0)
     x = (q, k, v, do)
@@ -318,6 +334,8 @@ def main():
     flops_step, fwd_flops = step_flops(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "cp": w.cp,
               "layout": ("contiguous", "head_tail", "striped")[w.layout], "causal": w.causal,
+              "H_kv": w.kv_heads, "rope": ("half pairs, base %g, fused into the permute of q,k and the "
+                                              "unpermute of dQ,dK" % ROPE_BASE) if w.rope else None,
               "step": "permute q,k,v" + (",dO" if w.bwd else "") + " -> ring fwd -> unpermute O" +
                       (" -> ring bwd -> unpermute dQ,dK,dV" if w.bwd else ""),
               "l2": "inputs larger than L2 (%.0f MB per tensor vs 126 MB)" % (w.B * w.H * w.L * w.D * 2 / 1e6),

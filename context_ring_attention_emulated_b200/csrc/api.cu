@@ -54,7 +54,7 @@ rattn_status check_attn_d(int D, rattn_dtype dt) {
 
 int64_t chunks_of(int cp, rattn_layout layout) {
   if (layout == RATTN_LAYOUT_HEAD_TAIL) return 2LL * cp;
-  if (layout == RATTN_LAYOUT_CONTIGUOUS) return cp;
+  if (layout == RATTN_LAYOUT_CONTIGUOUS || layout == RATTN_LAYOUT_STRIPED) return cp;
   return -1;
 }
 
@@ -157,6 +157,43 @@ rattn_status cp_layout_unpermute(const void* y, void* x, int B, int H, int64_t L
   return launch_unpermute(y, x, B * H, L, Lp, D * es, cp_size, layout, static_cast<cudaStream_t>(stream));
 }
 
+static rattn_status check_rope(int B, int H, int64_t L, int64_t Lp, int D, rattn_dtype dtype, int cp_size,
+                               rattn_layout layout, double base, rattn_rope_style style) {
+  const int es = elem_size(dtype);
+  if (!es || B < 1 || H < 1 || D < 2 || L < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1)
+    return RATTN_ERR_INVALID_ARG;
+  if (!(base > 0.0 && base < INFINITY)) return RATTN_ERR_INVALID_ARG;
+  if (style != RATTN_ROPE_HALF && style != RATTN_ROPE_INTERLEAVED) return RATTN_ERR_INVALID_ARG;
+  if (Lp != cp_layout_padded_len(L, cp_size, layout)) return RATTN_ERR_INVALID_ARG;
+  if (Lp > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  const int64_t row = static_cast<int64_t>(D) * es;
+  if (D % 2 || row % 16 || row > 4096) return RATTN_ERR_UNSUPPORTED;
+  if (style == RATTN_ROPE_HALF && (row / 2) % 16) return RATTN_ERR_UNSUPPORTED;
+  return RATTN_OK;
+}
+
+rattn_status cp_layout_permute_rope(const void* x, void* y, int32_t* pos, int B, int H, int64_t L, int64_t Lp,
+                                    int D, rattn_dtype dtype, int cp_size, rattn_layout layout, double rope_base,
+                                    rattn_rope_style style, void* stream) {
+  rattn_status st = check_rope(B, H, L, Lp, D, dtype, cp_size, layout, rope_base, style);
+  if (st != RATTN_OK) return st;
+  if (Lp == 0) return RATTN_OK;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16) || (pos && !aligned(pos, 4))) return RATTN_ERR_INVALID_ARG;
+  return launch_permute_rope(x, y, pos, B * H, L, Lp, D, dtype, cp_size, layout, rope_base, style,
+                             static_cast<cudaStream_t>(stream));
+}
+
+rattn_status cp_layout_unpermute_rope_grad(const void* dy, void* dx, int B, int H, int64_t L, int64_t Lp, int D,
+                                           rattn_dtype dtype, int cp_size, rattn_layout layout, double rope_base,
+                                           rattn_rope_style style, void* stream) {
+  rattn_status st = check_rope(B, H, L, Lp, D, dtype, cp_size, layout, rope_base, style);
+  if (st != RATTN_OK) return st;
+  if (L == 0) return RATTN_OK;
+  if (!dx || !dy || !aligned(dx, 16) || !aligned(dy, 16)) return RATTN_ERR_INVALID_ARG;
+  return launch_unpermute_rope_grad(dy, dx, B * H, L, Lp, D, dtype, cp_size, layout, rope_base, style,
+                                    static_cast<cudaStream_t>(stream));
+}
+
 rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v, const int32_t* q_pos,
                                const int32_t* kv_pos, int B, int H, int64_t Lq, int64_t Lk, int D,
                                rattn_dtype dtype, float scale, int causal, int64_t kv_valid, float* o, float* lse,
@@ -228,6 +265,14 @@ static rattn_status check_ring(const void* q, const void* k, const void* v, cons
 rattn_status rattn_ring_fwd(const void* q, const void* k, const void* v, const int32_t* pos, int B, int H,
                             int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout, int causal,
                             float scale, int64_t L_valid, void* o, float* lse, void* stream) {
+  return rattn_ring_fwd_gqa(q, k, v, pos, B, H, H, Lp, D, dtype, cp_size, layout, causal, scale, L_valid, o, lse,
+                            stream);
+}
+
+rattn_status rattn_ring_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* pos, int B, int H,
+                                int H_kv, int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout,
+                                int causal, float scale, int64_t L_valid, void* o, float* lse, void* stream) {
+  if (H_kv < 1 || H < 1 || H % H_kv) return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_ring(q, k, v, pos, B, H, Lp, D, dtype, cp_size, layout, causal, scale);
   if (st != RATTN_OK || Lp == 0) return st;
   if (!o || !lse || !aligned(o, 16) || !aligned(lse, 4)) return RATTN_ERR_INVALID_ARG;
@@ -238,6 +283,7 @@ rattn_status rattn_ring_fwd(const void* q, const void* k, const void* v, const i
   a.q_pos = pos;
   a.kv_pos = pos;
   a.BH = B * H;
+  a.group = H / H_kv;
   a.nseg = cp_size;
   a.Lq_seg = Lp / cp_size;
   a.Lk_seg = Lp / cp_size;
@@ -269,6 +315,16 @@ rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const v
                             rattn_dtype dtype, int cp_size, rattn_layout layout, int causal, float scale,
                             int64_t L_valid, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                             void* stream) {
+  return rattn_ring_bwd_gqa(q, k, v, o, dout, lse, pos, B, H, H, Lp, D, dtype, cp_size, layout, causal, scale,
+                            L_valid, dq, dk, dv, workspace, workspace_bytes, stream);
+}
+
+rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                const float* lse, const int32_t* pos, int B, int H, int H_kv, int64_t Lp, int D,
+                                rattn_dtype dtype, int cp_size, rattn_layout layout, int causal, float scale,
+                                int64_t L_valid, void* dq, void* dk, void* dv, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (H_kv < 1 || H < 1 || H % H_kv) return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_ring(q, k, v, pos, B, H, Lp, D, dtype, cp_size, layout, causal, scale);
   if (st != RATTN_OK || Lp == 0) return st;
   if (!o || !dout || !lse || !dq || !dk || !dv || !workspace || !aligned(o, 16) || !aligned(dout, 16) ||
@@ -286,6 +342,7 @@ rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const v
   a.lse = lse;
   a.pos = pos;
   a.BH = B * H;
+  a.group = H / H_kv;
   a.nseg = cp_size;
   a.Lseg = Lp / cp_size;
   a.D = D;

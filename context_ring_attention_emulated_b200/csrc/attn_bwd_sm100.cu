@@ -66,7 +66,7 @@ struct Params {
   const float* lse;
   const float* delta;
   const int32_t* pos;
-  int BH, nseg, Lseg, nq_tiles, nk_tiles, causal;
+  int BH, group, nseg, Lseg, nq_tiles, nk_tiles, causal;
   long long kv_valid;
   float scale, scale_log2;
   float* dq_acc;
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int s = item % p.nseg;
   item /= p.nseg;
   const int kt = item % p.nk_tiles;
-  const int bh = item / p.nk_tiles;
+  const int kvh = item / p.nk_tiles;  // (batch, key/value head); its query heads are kvh * group + j
   const int k0 = kt * BK;
   const int k_rows = min(BK, p.Lseg - k0);
   const long long k_min = posat(p, s, k0);
@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *s_tmem;
   int NIT = 0;
   for (int t = 0; t < p.nseg; ++t) NIT += p.nq_tiles - s_hop[t].x;
+  NIT *= p.group;  // the same tiles for every query head of the group
 
   int issued_q = 0;
   bool kv_issued = false;
@@ -207,13 +208,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tm_do);
         mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE);
         for (int b = 0; b < C::NBOX; ++b) {
-          tma_load_4d(smem + C::OFF_K + b * C::BOX, &tm_k, bar_kv_full, b * 64, k0, s, bh);
-          tma_load_4d(smem + C::OFF_V + b * C::BOX, &tm_v, bar_kv_full, b * 64, k0, s, bh);
+          tma_load_4d(smem + C::OFF_K + b * C::BOX, &tm_k, bar_kv_full, b * 64, k0, s, kvh);
+          tma_load_4d(smem + C::OFF_V + b * C::BOX, &tm_v, bar_kv_full, b * 64, k0, s, kvh);
         }
       }
       kv_issued = true;
       bool ok = true;
       int it = 0;
+      for (int hq = 0; hq < p.group && ok; ++hq) {
+      const int bh = kvh * p.group + hq;  // (batch, query head)
       for (int t = 0; t < p.nseg && ok; ++t) {
         const int r = (s + t) % p.nseg;
         for (int i = s_hop[t].x; i < p.nq_tiles; ++i, ++it) {
@@ -250,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++issued_q;
         }
+      }
       }
     }
   } else if (warp == 1) {
@@ -328,6 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sds = smem + C::OFF_DS + wg * C::BOX;
     bool ok = true;
     int it = 0;
+    for (int hq = 0; hq < p.group && ok; ++hq) {
+    const int bh = kvh * p.group + hq;  // (batch, query head)
     for (int t = 0; t < p.nseg && ok; ++t) {
       const int r = (s + t) % p.nseg;
       const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
@@ -459,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar_dq_free);  // one arrival per warp
       }
     }
+    }
     // ------------------------------------------------------ dK, dV out
     if (ok && NIT > 0 && !warp_wait(bar_a_free, (NIT - 1) & 1, s_abort, p.wait_ns)) {
       if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_EPILOGUE);
@@ -466,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       if (NIT > 0) tc_fence_after();
-      const long long krow = (static_cast<long long>(bh) * p.nseg + s) * p.Lseg + k0 + row;
+      const long long krow = (static_cast<long long>(kvh) * p.nseg + s) * p.Lseg + k0 + row;
       __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + krow * D + wg * (D / 2);
       __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + krow * D + wg * (D / 2);
 #pragma unroll
@@ -575,7 +582,8 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   if (a.Lseg > INT32_MAX - BQ || a.nseg > kMaxHops) return RATTN_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(a.BH) * a.nseg * a.Lseg;
   const int nt = static_cast<int>((a.Lseg + 127) / 128);
-  const long long grid = static_cast<long long>(a.BH) * a.nseg * nt;
+  if (a.group < 1 || a.BH % a.group) return RATTN_ERR_INVALID_ARG;
+  const long long grid = static_cast<long long>(a.BH / a.group) * a.nseg * nt;  // one CTA per key/value tile
   if (grid == 0) return RATTN_OK;
   if (grid > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
   bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
@@ -584,8 +592,8 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   CUtensorMap tq, tk, tv, tdo;
   rattn_status st;
   if ((st = make_tmap_bf16(&tq, a.q, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
-  if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH, BK)) != RATTN_OK) return st;
-  if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH, BK)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
   if ((st = set_smem_attr(reinterpret_cast<const void*>(&bwd_kernel<D>), C::SMEM)) != RATTN_OK) return st;
   Params p;
@@ -593,6 +601,7 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.delta = a.delta;
   p.pos = a.pos;
   p.BH = a.BH;
+  p.group = a.group;
   p.nseg = a.nseg;
   p.Lseg = static_cast<int>(a.Lseg);
   p.nq_tiles = nt;

@@ -64,7 +64,7 @@ struct Cfg {
 struct Params {
   const int32_t* q_pos;
   const int32_t* kv_pos;
-  int BH, nseg, Lq_seg, Lk_seg, n_qtiles, causal;
+  int BH, group, nseg, Lq_seg, Lk_seg, n_qtiles, causal;
   long long kv_valid;
   float scale_log2;
   void* o;
@@ -129,12 +129,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Work item: (batch, head) slowest, so the CTAs resident at any time share
   // one head's K/V in L2; within a head the heaviest query tiles (largest
-  // local index, hence largest positions under both layouts) go first.
+  // local index, hence largest positions under every layout) go first.
   int item = blockIdx.x;
   const int r = item % p.nseg;
   item /= p.nseg;
   const int qt = p.n_qtiles - 1 - (item % p.n_qtiles);
   const int bh = item / p.n_qtiles;
+  const int kvh = bh / p.group;  // (batch, key/value head): query heads of a group are contiguous
   const int q0 = qt * BM;
   const int q_rows = min(BM, p.Lq_seg - q0);
   const long long q_min = qpos(p, r, q0);
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&bar_k_full[st], C::TILE);
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_4d(sK + st * C::TILE + b * C::BOX, &tm_k, &bar_k_full[st], b * 64, j * BN, s, bh);
+            tma_load_4d(sK + st * C::TILE + b * C::BOX, &tm_k, &bar_k_full[st], b * 64, j * BN, s, kvh);
           ++issued_k;
           if (u > 0 && !mbar_wait(&bar_v_empty[st], (u - 1) & 1, s_abort, p.wait_ns)) {
             record_failure(s_abort, p.err, SITE_FWD_LOAD);
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mbar_arrive_expect_tx(&bar_v_full[st], C::TILE);
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_4d(sV + st * C::TILE + b * C::BOX, &tm_v, &bar_v_full[st], b * 64, j * BN, s, bh);
+            tma_load_4d(sV + st * C::TILE + b * C::BOX, &tm_v, &bar_v_full[st], b * 64, j * BN, s, kvh);
           ++issued_v;
         }
       }
@@ -479,13 +480,15 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
   CUtensorMap tq, tk, tv;
   rattn_status st;
   if ((st = make_tmap_bf16(&tq, a.q, D, a.Lq_seg, a.nseg, a.BH, BM)) != RATTN_OK) return st;
-  if ((st = make_tmap_bf16(&tk, a.k, D, a.Lk_seg, a.nseg, a.BH, BN)) != RATTN_OK) return st;
-  if ((st = make_tmap_bf16(&tv, a.v, D, a.Lk_seg, a.nseg, a.BH, BN)) != RATTN_OK) return st;
+  if (a.group < 1 || a.BH % a.group) return RATTN_ERR_INVALID_ARG;
+  if ((st = make_tmap_bf16(&tk, a.k, D, a.Lk_seg, a.nseg, a.BH / a.group, BN)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tv, a.v, D, a.Lk_seg, a.nseg, a.BH / a.group, BN)) != RATTN_OK) return st;
   if ((st = set_smem_attr(reinterpret_cast<const void*>(&fwd_kernel<D>), C::SMEM)) != RATTN_OK) return st;
   Params p;
   p.q_pos = a.q_pos;
   p.kv_pos = a.kv_pos;
   p.BH = a.BH;
+  p.group = a.group;
   p.nseg = a.nseg;
   p.Lq_seg = static_cast<int>(a.Lq_seg);
   p.Lk_seg = static_cast<int>(a.Lk_seg);

@@ -28,7 +28,7 @@ struct SimtFwd {
   const float* v;
   const int32_t* q_pos;
   const int32_t* kv_pos;
-  int BH, nseg, Lq_seg, Lk_seg, D, causal;
+  int BH, group, nseg, Lq_seg, Lk_seg, D, causal;
   long long kv_valid;
   float scale;
   float* o;
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(kRows) fwd_simt_kernel(const SimtFwd p) {
 
   for (int t = 0; t < p.nseg; ++t) {
     const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-    const long long kbase = (static_cast<long long>(bh) * p.nseg + s) * p.Lk_seg;
+    const long long kbase = (static_cast<long long>(bh / p.group) * p.nseg + s) * p.Lk_seg;
     for (int k0 = 0; k0 < p.Lk_seg; k0 += kTile) {
       const long long first = pos_at(p.kv_pos, static_cast<long long>(s) * p.Lk_seg, k0);
       if (first >= p.kv_valid || (p.causal && first > blk_max)) break;  // positions are non-decreasing
@@ -120,7 +120,7 @@ struct SimtBwd {
   const float* dout;
   const float* lse;
   const int32_t* pos;
-  int BH, nseg, Lseg, D, causal;
+  int BH, group, nseg, Lseg, D, causal;
   long long kv_valid;
   float scale;
   float* dq;
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(kRows) dq_simt_kernel(const SimtBwd p) {
   const float dl = valid ? p.delta[qbase + row] : 0.f;
   for (int t = 0; t < p.nseg; ++t) {
     const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-    const long long kbase = (static_cast<long long>(bh) * p.nseg + s) * p.Lseg;
+    const long long kbase = (static_cast<long long>(bh / p.group) * p.nseg + s) * p.Lseg;
     for (int k0 = 0; k0 < p.Lseg; k0 += kTile) {
       const long long first = p.pos[static_cast<long long>(s) * p.Lseg + k0];
       if (first >= p.kv_valid || (p.causal && first > blk_max)) break;
@@ -203,7 +203,8 @@ __global__ void __launch_bounds__(kRows) dq_simt_kernel(const SimtBwd p) {
 }
 
 // One thread per key row: dV_j = sum_i P_ij dO_i, dK_j = scale sum_i dS_ij q_i,
-// over the queries of every rank (the K/V block visits every rank's Q).
+// over the queries of every rank (the K/V block visits every rank's Q) and of
+// every query head of the key/value head's group.
 template <int DMAX>
 __global__ void __launch_bounds__(kRows) dkdv_simt_kernel(const SimtBwd p) {
   __shared__ float sq[kTile][DMAX];
@@ -215,10 +216,10 @@ __global__ void __launch_bounds__(kRows) dkdv_simt_kernel(const SimtBwd p) {
   const int kt = item % nkt;
   item /= nkt;
   const int s = item % p.nseg;
-  const int bh = item / p.nseg;
+  const int kvh = item / p.nseg;  // (batch, key/value head)
   const int row = kt * kRows + threadIdx.x;
   const bool valid = row < p.Lseg;
-  const long long kbase = (static_cast<long long>(bh) * p.nseg + s) * p.Lseg;
+  const long long kbase = (static_cast<long long>(kvh) * p.nseg + s) * p.Lseg;
   const int first_row = kt * kRows;
   const long long my_pos = p.pos[static_cast<long long>(s) * p.Lseg + (valid ? row : first_row)];
   const long long blk_min = p.pos[static_cast<long long>(s) * p.Lseg + first_row];
@@ -231,8 +232,9 @@ __global__ void __launch_bounds__(kRows) dkdv_simt_kernel(const SimtBwd p) {
     gk[d] = 0.f;
     gv[d] = 0.f;
   }
-  for (int r = 0; r < p.nseg; ++r) {
-    const long long qbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
+  for (int hr = 0; hr < p.group * p.nseg; ++hr) {
+    const int r = hr % p.nseg;
+    const long long qbase = (static_cast<long long>(kvh * p.group + hr / p.nseg) * p.nseg + r) * p.Lseg;
     for (int q0 = 0; q0 < p.Lseg; q0 += kTile) {
       const int n = min(kTile, p.Lseg - q0);
       const long long last = p.pos[static_cast<long long>(r) * p.Lseg + q0 + n - 1];
@@ -296,7 +298,7 @@ rattn_status bwd_launch(const SimtBwd& p, cudaStream_t stream) {
   if (grid > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
   delta_simt_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(p, rows);
   dq_simt_kernel<DMAX><<<static_cast<unsigned>(grid), kRows, 0, stream>>>(p);
-  dkdv_simt_kernel<DMAX><<<static_cast<unsigned>(grid), kRows, 0, stream>>>(p);
+  dkdv_simt_kernel<DMAX><<<static_cast<unsigned>(grid / p.group), kRows, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
@@ -304,6 +306,7 @@ rattn_status bwd_launch(const SimtBwd& p, cudaStream_t stream) {
 
 rattn_status launch_fwd_simt(const FwdArgs& a) {
   if (a.dtype != RATTN_F32 || a.D > 128 || a.D % 4) return RATTN_ERR_UNSUPPORTED;
+  if (a.group < 1 || a.BH % a.group) return RATTN_ERR_INVALID_ARG;
   if (a.Lq_seg > INT32_MAX - kRows || a.Lk_seg > INT32_MAX - kTile) return RATTN_ERR_UNSUPPORTED;
   SimtFwd p;
   p.q = static_cast<const float*>(a.q);
@@ -312,6 +315,7 @@ rattn_status launch_fwd_simt(const FwdArgs& a) {
   p.q_pos = a.q_pos;
   p.kv_pos = a.kv_pos;
   p.BH = a.BH;
+  p.group = a.group;
   p.nseg = a.nseg;
   p.Lq_seg = static_cast<int>(a.Lq_seg);
   p.Lk_seg = static_cast<int>(a.Lk_seg);
@@ -328,6 +332,7 @@ rattn_status launch_fwd_simt(const FwdArgs& a) {
 
 rattn_status launch_bwd_simt(const BwdArgs& a) {
   if (a.dtype != RATTN_F32 || a.D > 128 || a.D % 4) return RATTN_ERR_UNSUPPORTED;
+  if (a.group < 1 || a.BH % a.group) return RATTN_ERR_INVALID_ARG;
   if (a.Lseg > INT32_MAX - kRows) return RATTN_ERR_UNSUPPORTED;
   SimtBwd p;
   p.q = static_cast<const float*>(a.q);
@@ -338,6 +343,7 @@ rattn_status launch_bwd_simt(const BwdArgs& a) {
   p.lse = a.lse;
   p.pos = a.pos;
   p.BH = a.BH;
+  p.group = a.group;
   p.nseg = a.nseg;
   p.Lseg = static_cast<int>(a.Lseg);
   p.D = a.D;

@@ -52,7 +52,8 @@ struct FwdArgs {
   const void* v;
   const int32_t* q_pos;   // [nseg*Lq_seg] or NULL (row index)
   const int32_t* kv_pos;  // [nseg*Lk_seg] or NULL (row index)
-  int BH;
+  int BH;         // batch x query heads
+  int group = 1;  // query heads per key/value head (GQA); K/V hold BH / group heads
   int nseg;
   int64_t Lq_seg;
   int64_t Lk_seg;
@@ -77,7 +78,8 @@ struct BwdArgs {
   const void* dout;
   const float* lse;
   const int32_t* pos;  // [nseg*Lseg]
-  int BH;
+  int BH;              // batch x query heads
+  int group = 1;       // query heads per key/value head (GQA); K/V, dK, dV hold BH / group heads
   int nseg;
   int64_t Lseg;
   int D;
@@ -99,6 +101,11 @@ rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_
                             int cp, int layout, cudaStream_t stream);
 rattn_status launch_unpermute(const void* y, void* x, int BH, int64_t L, int64_t Lp, int row_bytes, int cp,
                               int layout, cudaStream_t stream);
+rattn_status launch_permute_rope(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int D,
+                                 rattn_dtype dtype, int cp, int layout, double base, int style, cudaStream_t stream);
+rattn_status launch_unpermute_rope_grad(const void* dy, void* dx, int BH, int64_t L, int64_t Lp, int D,
+                                        rattn_dtype dtype, int cp, int layout, double base, int style,
+                                        cudaStream_t stream);
 rattn_status launch_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, int64_t rows,
                           int D, cudaStream_t stream);
 

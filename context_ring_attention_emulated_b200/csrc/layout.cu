@@ -4,31 +4,17 @@
 // tokens is cut into 2*cp chunks of c = Lp/(2*cp); rank r holds chunk r
 // followed by chunk 2*cp-1-r, ranks concatenated in rank order, and every slot
 // keeps its global position id. CONTIGUOUS (the naive split) is the identity.
+// STRIPED ([Ring-page], striped attention) gives token g to rank g mod cp.
 // Padding goes at the tail of the global sequence and is zero-filled.
 //
 // Both kernels are gathers: each thread moves 16-byte vectors of one output
 // row, so stores are fully coalesced and loads are coalesced within a row.
 // Rows wider than 4 KB (256 vectors) are not supported.
+#include "cp_map.cuh"
 #include "internal.h"
 
 namespace rattn {
 namespace {
-
-// Global position held by slot i of the permuted sequence.
-__device__ __forceinline__ int slot_to_global(int i, int c, int cp, int layout) {
-  if (layout == RATTN_LAYOUT_CONTIGUOUS) return i;
-  const int r = i / (2 * c);
-  const int j = i - r * 2 * c;
-  return j < c ? r * c + j : (2 * cp - 1 - r) * c + (j - c);
-}
-
-// Slot of the permuted sequence that holds global position g.
-__device__ __forceinline__ int global_to_slot(int g, int c, int cp, int layout) {
-  if (layout == RATTN_LAYOUT_CONTIGUOUS) return g;
-  const int k = g / c;
-  const int j = g - k * c;
-  return k < cp ? k * 2 * c + j : (2 * cp - 1 - k) * 2 * c + c + j;
-}
 
 // Thread layout: vpr consecutive threads move one row (vpr = row bytes / 16),
 // blockDim.x / vpr rows per block step; blockIdx.y walks (batch, head). All
@@ -87,8 +73,7 @@ dim3 grid_2d(long long rows, int BH, int rpb) {
 rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int row_bytes,
                             int cp, int layout, cudaStream_t stream) {
   const int vpr = row_bytes / 16;
-  const int nchunks = layout == RATTN_LAYOUT_HEAD_TAIL ? 2 * cp : cp;
-  const int c = static_cast<int>(Lp / nchunks);
+  const int c = cp_map_c(Lp, cp, layout);
   if (vpr > 256) return RATTN_ERR_UNSUPPORTED;
   permute_kernel<<<grid_2d(Lp, BH, 256 / vpr), 256, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
                                                                  pos, BH, static_cast<int>(L), static_cast<int>(Lp),
@@ -99,8 +84,7 @@ rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_
 rattn_status launch_unpermute(const void* y, void* x, int BH, int64_t L, int64_t Lp, int row_bytes, int cp,
                               int layout, cudaStream_t stream) {
   const int vpr = row_bytes / 16;
-  const int nchunks = layout == RATTN_LAYOUT_HEAD_TAIL ? 2 * cp : cp;
-  const int c = static_cast<int>(Lp / nchunks);
+  const int c = cp_map_c(Lp, cp, layout);
   if (vpr > 256) return RATTN_ERR_UNSUPPORTED;
   unpermute_kernel<<<grid_2d(L, BH, 256 / vpr), 256, 0, stream>>>(static_cast<const uint4*>(y),
                                                                   static_cast<uint4*>(x), BH, static_cast<int>(L),

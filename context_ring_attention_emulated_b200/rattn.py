@@ -19,24 +19,31 @@ LIB_PATH = os.path.join(_PKG, "librattn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
-LAYOUT_CONTIGUOUS, LAYOUT_HEAD_TAIL = 0, 1
+LAYOUT_CONTIGUOUS, LAYOUT_HEAD_TAIL, LAYOUT_STRIPED = 0, 1, 2
+ROPE_HALF, ROPE_INTERLEAVED = 0, 1
 
 # (name, restype, argtypes) of every symbol include/rattn.h declares.
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _I64 = ctypes.c_int64
 _F = ctypes.c_float
+_D = ctypes.c_double
 SIGNATURES = [
     ("rattn_status_string", ctypes.c_char_p, [_I]),
     ("cp_layout_padded_len", _I64, [_I64, _I, _I]),
     ("cp_layout_permute", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
     ("cp_layout_unpermute", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
+    ("cp_layout_permute_rope", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _D, _I, _P]),
+    ("cp_layout_unpermute_rope_grad", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _D, _I, _P]),
     ("rattn_partial_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I, _I, _F, _I, _I64, _P, _P, _P]),
     ("rattn_merge", _I, [_P, _P, _P, _P, _I, _I, _I64, _I, _P]),
     ("rattn_ring_fwd", _I, [_P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64, _P, _P, _P]),
     ("rattn_ring_bwd_workspace_size", ctypes.c_size_t, [_I, _I, _I64, _I]),
     ("rattn_ring_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
                             _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    ("rattn_ring_fwd_gqa", _I, [_P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64, _P, _P, _P]),
+    ("rattn_ring_bwd_gqa", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
+                                _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("rattn_ring_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
                                     _P, _P, _P, _P]),
     ("rattn_get_device_error", _I, [ctypes.POINTER(_I)]),
@@ -128,6 +135,39 @@ def cp_layout_unpermute(y, L, cp_size, layout=LAYOUT_HEAD_TAIL, x=None, stream=N
     return x
 
 
+def cp_layout_permute_rope(x, cp_size, layout=LAYOUT_HEAD_TAIL, rope_base=10000.0, style=ROPE_HALF, y=None,
+                           pos=None, stream=None):
+    """x [B,H,L,D] -> (y [B,H,Lp,D] rank-major with RoPE at the global
+    positions, pos int32 [Lp])."""
+    _need_cuda(x)
+    B, H, L, D = x.shape
+    Lp = cp_layout_padded_len(L, cp_size, layout)
+    if y is None:
+        y = torch.empty(B, H, Lp, D, dtype=x.dtype, device=x.device)
+    if pos is None:
+        pos = torch.empty(Lp, dtype=torch.int32, device=x.device)
+    _need_cuda(y, pos)
+    _check("cp_layout_permute_rope", lib.cp_layout_permute_rope(
+        _ptr(x), _ptr(y), _ptr(pos), B, H, L, Lp, D, _dtype_code(x), cp_size, layout, float(rope_base),
+        int(style), _stream(stream)))
+    return y, pos
+
+
+def cp_layout_unpermute_rope_grad(dy, L, cp_size, layout=LAYOUT_HEAD_TAIL, rope_base=10000.0, style=ROPE_HALF,
+                                  dx=None, stream=None):
+    """dy [B,H,Lp,D] rank-major (gradient w.r.t. the rotated tensor) ->
+    dx [B,H,L,D] global order (gradient w.r.t. the un-rotated input)."""
+    _need_cuda(dy)
+    B, H, Lp, D = dy.shape
+    if dx is None:
+        dx = torch.empty(B, H, L, D, dtype=dy.dtype, device=dy.device)
+    _need_cuda(dx)
+    _check("cp_layout_unpermute_rope_grad", lib.cp_layout_unpermute_rope_grad(
+        _ptr(dy), _ptr(dx), B, H, L, Lp, D, _dtype_code(dy), cp_size, layout, float(rope_base), int(style),
+        _stream(stream)))
+    return dx
+
+
 def rattn_partial_fwd(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True, kv_valid=2**62,
                       o=None, lse=None, stream=None):
     """One partial attention: returns (O fp32 [B,H,Lq,D], LSE fp32 [B,H,Lq])."""
@@ -192,6 +232,51 @@ def rattn_ring_bwd(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL,
                                                  _ptr(pos), B, H, Lp, D, _dtype_code(q), cp_size, layout,
                                                  int(causal), float(scale), int(L_valid), _ptr(dq), _ptr(dk),
                                                  _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def rattn_ring_fwd_gqa(q, k, v, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None, L_valid=None,
+                       o=None, lse=None, stream=None):
+    """Ring forward with grouped key/value heads: q [B,H,Lp,D], k/v
+    [B,H_kv,Lp,D] (H_kv from k's shape); returns (O [B,H,Lp,D], LSE)."""
+    _need_cuda(q, k, v, pos)
+    B, H, Lp, D = q.shape
+    H_kv = k.shape[1]
+    if k.shape != (B, H_kv, Lp, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H_kv, Lp, D] matching q")
+    scale = D ** -0.5 if scale is None else scale
+    L_valid = Lp if L_valid is None else L_valid
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, H, Lp, dtype=torch.float32, device=q.device)
+    _check("rattn_ring_fwd_gqa", lib.rattn_ring_fwd_gqa(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(pos), B, H, H_kv, Lp, D, _dtype_code(q), cp_size, layout, int(causal),
+        float(scale), int(L_valid), _ptr(o), _ptr(lse), _stream(stream)))
+    return o, lse
+
+
+def rattn_ring_bwd_gqa(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None,
+                       L_valid=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of rattn_ring_fwd_gqa: returns (dQ [B,H,Lp,D], dK, dV
+    [B,H_kv,Lp,D], each summed over its group of query heads)."""
+    _need_cuda(q, k, v, o, dout, lse, pos)
+    B, H, Lp, D = q.shape
+    H_kv = k.shape[1]
+    if k.shape != (B, H_kv, Lp, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H_kv, Lp, D] matching q")
+    scale = D ** -0.5 if scale is None else scale
+    L_valid = Lp if L_valid is None else L_valid
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = rattn_ring_bwd_workspace_size(B, H, Lp, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check("rattn_ring_bwd_gqa", lib.rattn_ring_bwd_gqa(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(pos), B, H, H_kv, Lp, D, _dtype_code(q),
+        cp_size, layout, int(causal), float(scale), int(L_valid), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
     return dq, dk, dv
 
 

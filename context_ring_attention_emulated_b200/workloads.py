@@ -16,6 +16,7 @@ import torch
 
 LAYOUT_CONTIGUOUS = 0
 LAYOUT_HEAD_TAIL = 1
+LAYOUT_STRIPED = 2
 
 
 @dataclass(frozen=True)
@@ -31,6 +32,12 @@ class Workload:
     layout: int
     mult: float = 1.0
     bwd: bool = False
+    H_kv: int = 0       # key/value heads (grouped-query attention); 0 means H
+    rope: bool = False  # rotate Q and K at their global positions while permuting
+
+    @property
+    def kv_heads(self):
+        return self.H_kv or self.H
 
     @property
     def torch_dtype(self):
@@ -55,16 +62,29 @@ WORKLOADS = {
                                            LAYOUT_CONTIGUOUS, 0.5),
     "bf16_L32000_cp4_fwdbwd": Workload("bf16_L32000_cp4_fwdbwd", "bf16", 1, 32, 32000, 128, True, 4,
                                        LAYOUT_HEAD_TAIL, 1.0, True),
+    # The 32k / cp=4 shapes under the striped assignment (token g on rank g mod cp).
+    "bf16_L32000_cp4_striped": Workload("bf16_L32000_cp4_striped", "bf16", 1, 32, 32000, 128, True, 4,
+                                        LAYOUT_STRIPED),
+    "bf16_L32000_cp4_striped_fwdbwd": Workload("bf16_L32000_cp4_striped_fwdbwd", "bf16", 1, 32, 32000, 128, True,
+                                               4, LAYOUT_STRIPED, 1.0, True),
+    # The 32k / cp=4 step with 8 key/value heads shared by 32 query heads (GQA).
+    "bf16_L32000_cp4_gqa8_fwdbwd": Workload("bf16_L32000_cp4_gqa8_fwdbwd", "bf16", 1, 32, 32000, 128, True, 4,
+                                            LAYOUT_HEAD_TAIL, 1.0, True, H_kv=8),
+    # The 32k / cp=4 step with RoPE fused into the permute of Q, K and the
+    # unpermute of dQ, dK.
+    "bf16_L32000_cp4_rope_fwdbwd": Workload("bf16_L32000_cp4_rope_fwdbwd", "bf16", 1, 32, 32000, 128, True, 4,
+                                            LAYOUT_HEAD_TAIL, 1.0, True, rope=True),
 }
 
 
 def make_qkv(w: Workload, device="cpu", seed=0):
-    """Q, K, V [B, H, L, D] in the workload's dtype, from one seeded generator."""
+    """Q [B, H, L, D] and K, V [B, H_kv, L, D] in the workload's dtype, from
+    one seeded generator."""
     g = torch.Generator(device=device)
     g.manual_seed(seed)
     out = []
-    for _ in range(3):
-        x = torch.randn(w.B, w.H, w.L, w.D, generator=g, device=device, dtype=torch.float32)
+    for heads in (w.H, w.kv_heads, w.kv_heads):
+        x = torch.randn(w.B, heads, w.L, w.D, generator=g, device=device, dtype=torch.float32)
         if w.mult != 1.0:
             x.mul_(w.mult)
         out.append(x.to(w.torch_dtype))

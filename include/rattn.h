@@ -68,14 +68,22 @@ typedef enum { RATTN_F32 = 0, RATTN_BF16 = 1 } rattn_dtype;
 
 /* [Megatron-CP]: CONTIGUOUS is the naive split (rank r holds the r-th of
  * cp_size equal pieces); HEAD_TAIL is the symmetric assignment (rank r holds
- * chunk r then chunk 2*cp_size-1-r of 2*cp_size equal chunks). */
-typedef enum { RATTN_LAYOUT_CONTIGUOUS = 0, RATTN_LAYOUT_HEAD_TAIL = 1 } rattn_layout;
+ * chunk r then chunk 2*cp_size-1-r of 2*cp_size equal chunks).
+ * [Ring-page] (future of sequence parallelism: striped attention rebalances
+ * the causal work): STRIPED gives token g to rank g mod cp_size, each rank
+ * keeping its tokens in increasing order (the Striped Attention assignment of
+ * Brandon et al., 2023). */
+typedef enum {
+  RATTN_LAYOUT_CONTIGUOUS = 0,
+  RATTN_LAYOUT_HEAD_TAIL = 1,
+  RATTN_LAYOUT_STRIPED = 2
+} rattn_layout;
 
 /* Human-readable name of a status code. Never NULL. */
 const char* rattn_status_string(rattn_status s);
 
 /* [Megatron-CP] padding rule: the smallest Lp >= L that is a multiple of
- * 2*cp_size (HEAD_TAIL) or cp_size (CONTIGUOUS). Returns -1 on bad arguments
+ * 2*cp_size (HEAD_TAIL) or cp_size (CONTIGUOUS, STRIPED). Returns -1 on bad arguments
  * (L < 0, cp_size < 1, unknown layout). Host only; no device work. */
 int64_t cp_layout_padded_len(int64_t L, int cp_size, rattn_layout layout);
 
@@ -97,6 +105,39 @@ rattn_status cp_layout_unpermute(const void* y, void* x,
                                  int B, int H, int64_t L, int64_t Lp, int D,
                                  rattn_dtype dtype, int cp_size, rattn_layout layout,
                                  void* stream);
+
+/* Rotary position embedding pairings. [Megatron-CP] "Symmetric chunk
+ * assignment" requires RoPE to use every token's global position; the
+ * rotation is RoFormer's (Su et al., 2021): pair i of a head vector turns by
+ * the angle p * base^(-2i/D) at position p, (a, b) -> (a cos - b sin,
+ * a sin + b cos). HALF pairs (x[i], x[i + D/2]) (the "rotate half" form);
+ * INTERLEAVED pairs (x[2i], x[2i+1]). */
+typedef enum { RATTN_ROPE_HALF = 0, RATTN_ROPE_INTERLEAVED = 1 } rattn_rope_style;
+
+/* cp_layout_permute with RoPE fused in: y[slot] = rotate(x[g], g) where g is
+ * the slot's global position (pos[slot], which is written as in
+ * cp_layout_permute when pos is non-NULL); pad rows are zero. The angle is
+ * formed in fp64 and reduced modulo 2*pi there; cos/sin of the remainder and
+ * the rotation run in fp32, which rounds once (RNE) to dtype. Same layout, alignment and size rules as
+ * cp_layout_permute, plus: rope_base finite and > 0; D even; for HALF the
+ * half row D/2 * sizeof(dtype) must be a multiple of 16 bytes (bf16: D % 16
+ * == 0; fp32: D % 8 == 0), else RATTN_ERR_UNSUPPORTED. x and y must not
+ * overlap. */
+rattn_status cp_layout_permute_rope(const void* x, void* y, int32_t* pos,
+                                    int B, int H, int64_t L, int64_t Lp, int D,
+                                    rattn_dtype dtype, int cp_size, rattn_layout layout,
+                                    double rope_base, rattn_rope_style style, void* stream);
+
+/* Gradient of cp_layout_permute_rope: dx [B,H,L,D] (global order) receives
+ * rotate(dy[slot(g)], -angle(g)) -- the inverse rotation, which is the
+ * rotation's transpose -- for dy [B,H,Lp,D] in rank-major order (the
+ * gradient with respect to the permuted, rotated tensor, e.g. the dQ or dK
+ * that rattn_ring_bwd returns); pad rows are dropped. Arguments and rules as
+ * cp_layout_permute_rope. */
+rattn_status cp_layout_unpermute_rope_grad(const void* dy, void* dx,
+                                           int B, int H, int64_t L, int64_t Lp, int D,
+                                           rattn_dtype dtype, int cp_size, rattn_layout layout,
+                                           double rope_base, rattn_rope_style style, void* stream);
 
 /* [CP-glossary], [Ring-page]: one partial attention of local queries against
  * one K/V block. q [B,H,Lq,D], k and v [B,H,Lk,D] in `dtype`; q_pos int32
@@ -153,6 +194,30 @@ rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const v
                             int cp_size, rattn_layout layout, int causal, float scale,
                             int64_t L_valid, void* dq, void* dk, void* dv,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* [Megatron-CP] "CP vs SP": the ring moves the K/V of H_kv heads, fewer than
+ * the H query heads under grouped-query attention (GQA, Ainslie et al., 2023:
+ * the query heads form H_kv equal groups, each group sharing one key/value
+ * head). rattn_ring_fwd with grouped key/value heads: q, o [B,H,Lp,D], lse
+ * [B,H,Lp]; k, v [B,H_kv,Lp,D]; H a positive multiple of H_kv; query head h
+ * attends key/value head h / (H / H_kv) (contiguous groups). H_kv == H is
+ * rattn_ring_fwd. H not a multiple of H_kv returns RATTN_ERR_INVALID_ARG. */
+rattn_status rattn_ring_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* pos,
+                                int B, int H, int H_kv, int64_t Lp, int D, rattn_dtype dtype,
+                                int cp_size, rattn_layout layout, int causal, float scale,
+                                int64_t L_valid, void* o, float* lse, void* stream);
+
+/* Gradients of rattn_ring_fwd_gqa: dq [B,H,Lp,D]; dk, dv [B,H_kv,Lp,D], each
+ * the sum over the group's query heads (the chain rule through the shared
+ * heads). q, o, dout, lse have H heads; k, v have H_kv. The workspace is sized
+ * by the query heads: rattn_ring_bwd_workspace_size(B, H, Lp, D). H_kv == H
+ * is rattn_ring_bwd. */
+rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, const int32_t* pos,
+                                int B, int H, int H_kv, int64_t Lp, int D, rattn_dtype dtype,
+                                int cp_size, rattn_layout layout, int causal, float scale,
+                                int64_t L_valid, void* dq, void* dk, void* dv,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /* Size of the device array rattn_ring_bwd_noalloc uses as scratch space. */
 #define RATTN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -42,7 +42,7 @@ def test_status_strings(rattn):
 @pytest.mark.parametrize("L,cp,layout,expect", [
     (32000, 4, 1, 32000), (4096, 2, 1, 4096), (1048576, 8, 1, 1048576), (131072, 8, 0, 131072),
     (10, 4, 1, 16), (10, 4, 0, 12), (0, 3, 1, 0), (1, 1, 1, 2), (1, 1, 0, 1),
-    (-1, 2, 1, -1), (10, 0, 1, -1), (10, 2, 7, -1)])
+    (-1, 2, 1, -1), (10, 0, 1, -1), (10, 2, 7, -1), (10, 4, 2, 12), (32000, 4, 2, 32000), (0, 3, 2, 0)])
 def test_padded_len(rattn, L, cp, layout, expect):
     assert rattn.lib.cp_layout_padded_len(L, cp, layout) == expect
 
@@ -51,7 +51,7 @@ def test_padded_len_matches_oracle(rattn):
     import oracle
     for cp in range(1, 17):
         for L in (0, 1, 5, 63, 64, 65, 1000):
-            for layout in (0, 1):
+            for layout in (0, 1, 2):
                 assert rattn.lib.cp_layout_padded_len(L, cp, layout) == oracle.padded_len(L, cp, layout)
 
 
@@ -76,6 +76,47 @@ def test_permute_rejects_bad_arguments(rattn):
     assert L.cp_layout_permute(FAKE, FAKE, FAKE, 1, 1, 0, 0, 64, 1, 4, 1, None) == rattn.OK
     assert L.cp_layout_unpermute(FAKE, FAKE, 1, 1, 10, 12, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
     assert L.cp_layout_unpermute(MIS, FAKE, 1, 1, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_INVALID_ARG
+
+
+def test_rope_permute_rejects_bad_arguments(rattn):
+    L = rattn.lib
+    pr = lambda **kw: L.cp_layout_permute_rope(kw.get("x", FAKE), FAKE, FAKE, 1, 1, kw.get("L", 16),
+                                               kw.get("Lp", 16), kw.get("D", 64), kw.get("dt", 1), 4,
+                                               kw.get("layout", 1), ctypes.c_double(kw.get("base", 1e4)),
+                                               kw.get("style", 0), None)
+    assert pr(base=0.0) == rattn.ERR_INVALID_ARG
+    assert pr(base=float("inf")) == rattn.ERR_INVALID_ARG
+    assert pr(base=float("nan")) == rattn.ERR_INVALID_ARG
+    assert pr(style=2) == rattn.ERR_INVALID_ARG
+    assert pr(Lp=24) == rattn.ERR_INVALID_ARG
+    assert pr(layout=5) == rattn.ERR_INVALID_ARG
+    assert pr(x=MIS) == rattn.ERR_INVALID_ARG
+    assert pr(x=None) == rattn.ERR_INVALID_ARG
+    assert pr(D=8, style=0) == rattn.ERR_UNSUPPORTED      # bf16 HALF: half row of 8 bytes
+    assert pr(D=4, dt=0, style=0) == rattn.ERR_UNSUPPORTED
+    assert pr(D=3, dt=0, style=1) == rattn.ERR_UNSUPPORTED
+    assert pr(D=4096) == rattn.ERR_UNSUPPORTED            # row above 4 KB
+    assert pr(L=0, Lp=0) == rattn.OK
+    ug = lambda **kw: L.cp_layout_unpermute_rope_grad(kw.get("dy", FAKE), FAKE, 1, 1, kw.get("L", 16),
+                                                      kw.get("Lp", 16), 64, 1, 4, 1,
+                                                      ctypes.c_double(kw.get("base", 1e4)), kw.get("style", 1), None)
+    assert ug(base=-1.0) == rattn.ERR_INVALID_ARG
+    assert ug(dy=MIS) == rattn.ERR_INVALID_ARG
+    assert ug(Lp=32) == rattn.ERR_INVALID_ARG
+    assert ug(L=0, Lp=0) == rattn.OK
+
+
+def test_gqa_calls_reject_bad_arguments(rattn):
+    L = rattn.lib
+    fwd = lambda H, Hkv: L.rattn_ring_fwd_gqa(FAKE, FAKE, FAKE, FAKE, 1, H, Hkv, 256, 64, 1, 2, 1, 1,
+                                              ctypes.c_float(0.125), 256, FAKE, FAKE, None)
+    assert fwd(4, 3) == rattn.ERR_INVALID_ARG      # H not a multiple of H_kv
+    assert fwd(4, 0) == rattn.ERR_INVALID_ARG
+    assert fwd(2, 4) == rattn.ERR_INVALID_ARG
+    bwd = lambda H, Hkv: L.rattn_ring_bwd_gqa(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, H, Hkv, 256, 64, 1, 2, 1,
+                                              1, ctypes.c_float(0.125), 256, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert bwd(6, 4) == rattn.ERR_INVALID_ARG
+    assert bwd(4, -2) == rattn.ERR_INVALID_ARG
 
 
 def test_attention_calls_reject_bad_arguments(rattn):

@@ -41,6 +41,9 @@ BWD_CASES = [
     (torch.bfloat16, 128, 29, 4, 1, True),
     (torch.bfloat16, 128, 1000, 3, 0, False),
     (torch.bfloat16, 64, 777, 1, 1, True),
+    (torch.bfloat16, 128, 1000, 4, 2, True),
+    (torch.bfloat16, 64, 29, 3, 2, True),
+    (torch.float32, 64, 29, 3, 2, True),
 ]
 
 

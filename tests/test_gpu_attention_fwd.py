@@ -138,6 +138,11 @@ RAGGED = [
     (torch.bfloat16, 128, 2048, 8, 1, False, 1, 1),    # head-tail non-causal
     (torch.float32, 64, 29, 3, 1, True, 1, 2),
     (torch.float32, 128, 300, 2, 0, False, 1, 1),
+    (torch.bfloat16, 128, 1000, 4, 2, True, 1, 2),     # striped: a masked diagonal tile every hop
+    (torch.bfloat16, 64, 29, 4, 2, True, 2, 1),        # striped, padded to 32
+    (torch.bfloat16, 128, 2048, 8, 2, False, 1, 1),    # striped non-causal
+    (torch.bfloat16, 64, 4100, 3, 2, True, 1, 1),      # striped, padded, several tiles per hop
+    (torch.float32, 64, 29, 3, 2, True, 1, 2),
 ]
 
 
@@ -159,7 +164,7 @@ def _sampled_rows(L, c, n_random, seed):
 
 
 @pytest.mark.parametrize("name,heads", [("bf16_L32000_cp4", None), ("bf16_L131072_cp8_noncausal", [0, 7]),
-                                        ("bf16_L1M_cp8", [0, 5])])
+                                        ("bf16_L1M_cp8", [0, 5]), ("bf16_L32000_cp4_striped", [0, 31])])
 def test_ring_fwd_full_size_sampled(rattn, name, heads):
     """Full-size workloads in the launch configuration the bench times;
     the oracle evaluates sampled query rows (first/last 4 of every chunk plus

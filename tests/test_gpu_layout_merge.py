@@ -23,7 +23,8 @@ def _bits(t):
 @pytest.mark.parametrize("dtype,D", [(torch.float32, 64), (torch.bfloat16, 128), (torch.bfloat16, 8),
                                      (torch.float32, 4)])
 @pytest.mark.parametrize("L,cp,layout", [(256, 2, 1), (4096, 2, 1), (29, 3, 1), (29, 3, 0), (1000, 4, 1),
-                                         (7, 8, 1), (1, 1, 1), (130, 16, 1), (97, 5, 0)])
+                                         (7, 8, 1), (1, 1, 1), (130, 16, 1), (97, 5, 0), (29, 3, 2),
+                                         (1000, 4, 2), (7, 8, 2), (130, 16, 2), (4096, 2, 2)])
 def test_permute_unpermute_bit_exact(rattn, dtype, D, L, cp, layout):
     x = make_tensor((2, 3, L, D), dtype, "cuda", seed=L + cp)
     y, pos = rattn.cp_layout_permute(x, cp, layout)
@@ -36,7 +37,8 @@ def test_permute_unpermute_bit_exact(rattn, dtype, D, L, cp, layout):
     assert np.array_equal(_bits(back), _bits(x))
 
 
-@pytest.mark.parametrize("name", ["bf16_L32000_cp4", "bf16_L1M_cp8", "bf16_L131072_cp8_noncausal"])
+@pytest.mark.parametrize("name", ["bf16_L32000_cp4", "bf16_L1M_cp8", "bf16_L131072_cp8_noncausal",
+                                  "bf16_L32000_cp4_striped"])
 def test_permute_full_size(rattn, name):
     w = WORKLOADS[name]
     x = make_tensor((w.B, w.H, w.L, w.D), w.torch_dtype, "cuda", seed=3)
