@@ -11,7 +11,7 @@
 // 128-key K/V tile of rank s resident and walks every rank's query tiles in
 // that hop order, skipping tiles the causal relation fully masks. dK and dV
 // accumulate in TMEM; each query tile's dQ contribution is transposed
-// through shared memory (warp-local) and added into an fp32 workspace with
+// within 8-lane groups by shuffles and added into an fp32 workspace with
 // coalesced vector reductions (whole 128-byte lines per warp instruction),
 // converted to the output dtype at the end.
 //
@@ -92,6 +92,37 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
+}
+
+// In: v = 32 consecutive fp32 values (8 float4 slots) of this lane's row.
+// Lanes 8g..8g+7 transpose their 8 x 8 float4 slots by xor shuffles (three
+// butterfly stages), after which lane (g, j) holds, in slot k, float4 j of
+// row 8g + k; then one reduction per slot adds four whole 128-byte rows per
+// warp instruction. dst = element (row 8g, column 4j) of this warp's rows;
+// only rows k < rows_left exist.
+template <int D>
+__device__ __forceinline__ void transpose_reduce(uint32_t (&v)[32], float* dst, int rows_left) {
+  const int j = threadIdx.x & 7;
+#pragma unroll
+  for (int sh = 4; sh >= 1; sh >>= 1) {
+    const bool hi = (j & sh) != 0;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      if (x & sh) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t send = hi ? v[4 * x + e] : v[4 * (x | sh) + e];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, sh);
+        if (hi) v[4 * x + e] = recv;
+        else v[4 * (x | sh) + e] = recv;
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (k < rows_left)
+      red_add_v4(dst + static_cast<long long>(k) * D, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
+                 __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
 }
 
 template <int D>
@@ -419,11 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_ds_ready);  // one arrival per warp
         // dQ read-out: this lane's query row, this warpgroup's half of D, in
-        // 32-column chunks. Each warp stages its own 32 rows (128-byte
-        // swizzled) in its rows of this warpgroup's half of the dS tile (the
-        // dQ MMA has finished reading it), then reads them back so that one
-        // warp instruction covers four whole 128-byte rows of the fp32
-        // accumulator and adds them with coalesced vector reductions.
+        // 32-column chunks, transposed within 8-lane groups by shuffles so
+        // that one warp instruction covers four whole 128-byte rows of the
+        // fp32 accumulator (coalesced vector reductions; no shared-memory
+        // round trip, whose bandwidth the MMAs need).
         if (!warp_wait(bar_dq_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
           ok = false;
@@ -431,33 +461,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         {
-          const int rsub = lane >> 3;         // row within a group of four
-          const int piece = lane & 7;         // 16-byte piece of a 128-byte row
-          const int wrow0 = quarter * 32;     // this warp's first row
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            uint32_t g[32];
-            tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + c * 32, g);
-            tmem_wait_ld();
-            uint8_t* rowp = sds + row * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) =
-                  make_uint4(g[4 * j], g[4 * j + 1], g[4 * j + 2], g[4 * j + 3]);
-            __syncwarp();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const int rr = wrow0 + k * 4 + rsub;
-              const float4 val =
-                  *reinterpret_cast<const float4*>(sds + rr * 128 + ((piece ^ (rr & 7)) << 4));
-              const int q = i * BQ + rr;
-              if (q < p.Lseg)
-                atomicAdd(reinterpret_cast<float4*>(p.dq_acc + (rowbase + q) * D + wg * (D / 2) + c * 32 +
-                                                    piece * 4),
-                          val);
-            }
-            __syncwarp();
-          }
+          const int gi = lane >> 3, gj = lane & 7;
+          float* dst0 = p.dq_acc + (rowbase + static_cast<long long>(i) * BQ + quarter * 32 + gi * 8) * D +
+                        wg * (D / 2) + gj * 4;
+          const int rows_left = p.Lseg - (i * BQ + quarter * 32 + gi * 8);
+          uint32_t g0[32], g1[32];
+          tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2), g0);
+          if constexpr (D == 128) tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + 32, g1);
+          tmem_wait_ld();
+          transpose_reduce<D>(g0, dst0, rows_left);
+          if constexpr (D == 128) transpose_reduce<D>(g1, dst0 + 32, rows_left);
         }
         if (!ok) break;
         tc_fence_before();
