@@ -22,8 +22,10 @@ Conventions (readings where the pages are silent):
 import numpy as np
 
 
-def visible_mask(q_pos, kv_pos, causal, kv_valid=None):
-    """Boolean [Lq, Lk] matrix of visible (query, key) pairs."""
+def visible_mask(q_pos, kv_pos, causal, kv_valid=None, q_seg=None, kv_seg=None):
+    """Boolean [Lq, Lk] matrix of visible (query, key) pairs. With segment ids
+    (packed sequences) a key is visible only to queries of its own segment,
+    and a key whose segment id is negative (padding) to none."""
     q_pos = np.asarray(q_pos, dtype=np.int64)
     kv_pos = np.asarray(kv_pos, dtype=np.int64)
     m = np.ones((q_pos.shape[0], kv_pos.shape[0]), dtype=bool)
@@ -31,6 +33,10 @@ def visible_mask(q_pos, kv_pos, causal, kv_valid=None):
         m &= kv_pos[None, :] <= q_pos[:, None]
     if kv_valid is not None:
         m &= kv_pos[None, :] < kv_valid
+    if kv_seg is not None:
+        q_seg = np.asarray(q_seg, dtype=np.int64)
+        kv_seg = np.asarray(kv_seg, dtype=np.int64)
+        m &= (kv_seg[None, :] == q_seg[:, None]) & (kv_seg[None, :] >= 0)
     return m
 
 
@@ -53,12 +59,15 @@ def _attention_2d(q, k, v, scale, mask):
     return o, lse
 
 
-def attention(q, k, v, scale, causal, q_pos=None, kv_pos=None, kv_valid=None, row_block=256):
+def attention(q, k, v, scale, causal, q_pos=None, kv_pos=None, kv_valid=None, row_block=256, q_seg=None,
+              kv_seg=None):
     """Full softmax attention in float64.
 
     q [..., Lq, D], k/v [..., Lk, D] (any float dtype; computed in float64 from
     the exact values given). Returns O [..., Lq, D] and LSE [..., Lq].
     Query rows are evaluated in independent blocks of ``row_block`` rows.
+    Optional segment ids restrict every query to the keys of its own segment
+    (packed sequences).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -77,7 +86,8 @@ def attention(q, k, v, scale, causal, q_pos=None, kv_pos=None, kv_valid=None, ro
     for b in range(qf.shape[0]):
         for r0 in range(0, Lq, row_block):
             r1 = min(Lq, r0 + row_block)
-            mask = visible_mask(q_pos[r0:r1], kv_pos, causal, kv_valid)
+            mask = visible_mask(q_pos[r0:r1], kv_pos, causal, kv_valid,
+                                None if q_seg is None else np.asarray(q_seg)[r0:r1], kv_seg)
             o[b, r0:r1], lse[b, r0:r1] = _attention_2d(qf[b, r0:r1], kf[b], vf[b], scale, mask)
     return o.reshape(lead + (Lq, vf.shape[-1])), lse.reshape(lead + (Lq,))
 
@@ -123,7 +133,7 @@ def blockwise_attention(q, k, v, scale, causal, key_blocks, q_pos=None, kv_pos=N
     return o, lse
 
 
-def ring_emulate(q, k, v, pos, cp, scale, causal, kv_valid=None):
+def ring_emulate(q, k, v, pos, cp, scale, causal, kv_valid=None, seg=None):
     """The ring of the pages, emulated: q/k/v [..., Lp, D] in permuted
     (rank-major) order with positions ``pos``. Rank r keeps its local Q fixed;
     at hop t it holds the K/V block of rank s = (r - t) mod cp (blocks move to
@@ -144,14 +154,16 @@ def ring_emulate(q, k, v, pos, cp, scale, causal, kv_valid=None):
             s = (r - t) % cp
             keys = slice(s * n, (s + 1) * n)
             ob, lb = attention(q[..., rows, :], k[..., keys, :], v[..., keys, :], scale, causal,
-                               q_pos=pos[rows], kv_pos=pos[keys], kv_valid=kv_valid)
+                               q_pos=pos[rows], kv_pos=pos[keys], kv_valid=kv_valid,
+                               q_seg=None if seg is None else seg[rows], kv_seg=None if seg is None else seg[keys])
             o_acc, lse_acc = merge(o_acc, lse_acc, ob, lb)
         o[..., rows, :] = o_acc
         lse[..., rows] = lse_acc
     return o, lse
 
 
-def attention_bwd(q, k, v, do, scale, causal, q_pos=None, kv_pos=None, kv_valid=None, row_block=256):
+def attention_bwd(q, k, v, do, scale, causal, q_pos=None, kv_pos=None, kv_valid=None, row_block=256, q_seg=None,
+                  kv_seg=None):
     """Gradient of O = softmax(scale Q K^T) V (masked) for upstream dO, float64.
 
     Textbook softmax-attention gradient (the pages only call ``.backward()``):
@@ -176,7 +188,8 @@ def attention_bwd(q, k, v, do, scale, causal, q_pos=None, kv_pos=None, kv_valid=
     for b in range(qf.shape[0]):
         for r0 in range(0, Lq, row_block):
             r1 = min(Lq, r0 + row_block)
-            mask = visible_mask(q_pos[r0:r1], kv_pos, causal, kv_valid)
+            mask = visible_mask(q_pos[r0:r1], kv_pos, causal, kv_valid,
+                                None if q_seg is None else np.asarray(q_seg)[r0:r1], kv_seg)
             s = np.where(mask, scale * (qf[b, r0:r1] @ kf[b].T), -np.inf)
             m = s.max(axis=1, initial=-np.inf)
             m_safe = np.where(np.isfinite(m), m, 0.0)

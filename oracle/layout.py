@@ -100,3 +100,59 @@ def unpermute(y, L, cp, layout):
         if src[i] >= 0:
             x[..., src[i], :] = y[..., i, :]
     return x
+
+
+def varlen_index(cu_seqlens, cp, layout):
+    """Layout of a pack of sequences with boundaries cu_seqlens [nseq + 1].
+
+    Returns (Tp, src, pos, seg, gkey), each per slot of the permuted pack:
+    src = index into the unpadded pack or -1 for padding, pos = position inside
+    the sequence (padding continues L_i, L_i + 1, ...), seg = sequence id or -1
+    for padding, gkey = offset of the sequence in the padded pack + pos.
+    Rank r's slice (rows [r Tp / cp, (r + 1) Tp / cp)) holds, for every
+    sequence in order, the rows rank r holds under ``perm_index`` of that
+    sequence alone.
+    """
+    cu = [int(x) for x in cu_seqlens]
+    if any(b < a for a, b in zip(cu, cu[1:])) or (cu and cu[0] != 0):
+        raise ValueError("cu_seqlens must start at 0 and be non-decreasing")
+    per_rank = [[] for _ in range(cp)]
+    offset = 0
+    for i in range(len(cu) - 1):
+        L = cu[i + 1] - cu[i]
+        Lp, src_i, pos_i = perm_index(L, cp, layout)
+        n = Lp // cp
+        for r in range(cp):
+            for j in range(r * n, (r + 1) * n):
+                real = src_i[j] >= 0
+                per_rank[r].append((cu[i] + src_i[j] if real else -1, pos_i[j], i if real else -1,
+                                    offset + pos_i[j]))
+        offset += Lp
+    rows = [t for r in range(cp) for t in per_rank[r]]
+    Tp = len(rows)
+    src = np.array([t[0] for t in rows], dtype=np.int64)
+    pos = np.array([t[1] for t in rows], dtype=np.int64)
+    seg = np.array([t[2] for t in rows], dtype=np.int64)
+    gkey = np.array([t[3] for t in rows], dtype=np.int64)
+    return Tp, src, pos, seg, gkey
+
+
+def varlen_permute(x, cu_seqlens, cp, layout):
+    """x [..., T, D] (a pack) -> y [..., Tp, D] in rank-major order; pad rows zero."""
+    Tp, src, _, _, _ = varlen_index(cu_seqlens, cp, layout)
+    y = np.zeros(x.shape[:-2] + (Tp, x.shape[-1]), dtype=x.dtype)
+    for i in range(Tp):
+        if src[i] >= 0:
+            y[..., i, :] = x[..., src[i], :]
+    return y
+
+
+def varlen_unpermute(y, cu_seqlens, cp, layout):
+    """Inverse of varlen_permute: y [..., Tp, D] -> x [..., T, D], pad rows dropped."""
+    Tp, src, _, _, _ = varlen_index(cu_seqlens, cp, layout)
+    T = int(cu_seqlens[-1])
+    x = np.zeros(y.shape[:-2] + (T, y.shape[-1]), dtype=y.dtype)
+    for i in range(Tp):
+        if src[i] >= 0:
+            x[..., src[i], :] = y[..., i, :]
+    return x
