@@ -148,7 +148,12 @@ def run_ours(args, w, rank, world, local):
     L, cp, layout = w.L, w.cp, w.layout
     B, H, D, Hkv = w.B, w.H, w.D, w.kv_heads
     heads = {"q": H, "k": Hkv, "v": Hkv, "do": H, "o": H, "dq": H, "dk": Hkv, "dv": Hkv}
-    Lp = rattn.cp_layout_padded_len(L, cp, layout)
+    if w.docs:  # packed sequences: host-side layout plan, index arrays resident on the device
+        plan = rattn.cp_layout_varlen_plan(w.cu_seqlens, cp, layout)
+        Lp = plan["Tp"]
+        src, gkey, segid = (plan[n].to(dev) for n in ("src", "gkey", "segid"))
+    else:
+        Lp = rattn.cp_layout_padded_len(L, cp, layout)
     pbuf = {n: torch.empty(B, heads[n], Lp, D, dtype=q.dtype, device=dev) for n in ("q", "k", "v", "do", "o")}
     pos = torch.empty(Lp, dtype=torch.int32, device=dev)
     lse = torch.empty(B, H, Lp, dtype=torch.float32, device=dev)
@@ -156,15 +161,27 @@ def run_ours(args, w, rank, world, local):
     out = {n: torch.empty(B, heads[n], L, D, dtype=q.dtype, device=dev) for n in ("o", "dq", "dk", "dv")}
     ring_fwd = rattn.rattn_ring_fwd_gqa if Hkv != H else rattn.rattn_ring_fwd
     ring_bwd = rattn.rattn_ring_bwd_gqa if Hkv != H else rattn.rattn_ring_bwd
+    if w.docs:
+        def ring_fwd(q_, k_, v_, pos_, cp_, layout_, causal_, scale_, L_valid=None, o=None, lse=None):
+            return rattn.rattn_ring_fwd_varlen(q_, k_, v_, gkey, segid, cp_, causal_, scale_, o=o, lse=lse)
+
+        def ring_bwd(q_, k_, v_, o_, do_, lse_, pos_, cp_, layout_, causal_, scale_, L_valid=None, dq=None, dk=None,
+                     dv=None, workspace=None):
+            return rattn.rattn_ring_bwd_varlen(q_, k_, v_, o_, do_, lse_, gkey, segid, cp_, causal_, scale_, dq=dq,
+                                               dk=dk, dv=dv, workspace=workspace)
 
     def permute_in(x, name):
-        if w.rope and name in ("q", "k"):
+        if w.docs:
+            rattn.cp_layout_gather(x, src, y=pbuf[name])
+        elif w.rope and name in ("q", "k"):
             rattn.cp_layout_permute_rope(x, cp, layout, ROPE_BASE, rattn.ROPE_HALF, y=pbuf[name], pos=pos)
         else:
             rattn.cp_layout_permute(x, cp, layout, y=pbuf[name], pos=pos)
 
-    def unpermute_grad(g, name, outs):
-        if w.rope and name in ("dq", "dk"):
+    def unpermute_grad(g, name, outs):  # unpermute of O and of the gradients
+        if w.docs:
+            rattn.cp_layout_scatter(g, src, L, x=outs[name])
+        elif w.rope and name in ("dq", "dk"):
             rattn.cp_layout_unpermute_rope_grad(g, L, cp, layout, ROPE_BASE, rattn.ROPE_HALF, dx=outs[name])
         else:
             rattn.cp_layout_unpermute(g, L, cp, layout, x=outs[name])
@@ -186,7 +203,7 @@ def run_ours(args, w, rank, world, local):
             e1 = torch.cuda.Event(enable_timing=True)
             e1.record(stream)
             fwd_ev.append((e0, e1))
-        rattn.cp_layout_unpermute(pbuf["o"], L, cp, layout, x=outs["o"])
+        unpermute_grad(pbuf["o"], "o", outs)
         if w.bwd:
             permute_in(xdo, "do")
             if timed:
@@ -334,7 +351,7 @@ def main():
     flops_step, fwd_flops = step_flops(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "cp": w.cp,
               "layout": ("contiguous", "head_tail", "striped")[w.layout], "causal": w.causal,
-              "H_kv": w.kv_heads, "rope": ("half pairs, base %g, fused into the permute of q,k and the "
+              "docs": len(w.docs) or None, "H_kv": w.kv_heads, "rope": ("half pairs, base %g, fused into the permute of q,k and the "
                                               "unpermute of dQ,dK" % ROPE_BASE) if w.rope else None,
               "step": "permute q,k,v" + (",dO" if w.bwd else "") + " -> ring fwd -> unpermute O" +
                       (" -> ring bwd -> unpermute dQ,dK,dV" if w.bwd else ""),

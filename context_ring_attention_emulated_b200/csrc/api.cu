@@ -5,6 +5,7 @@
 #include <set>
 #include <utility>
 
+#include "cp_map.cuh"
 #include "internal.h"
 
 namespace rattn {
@@ -157,6 +158,72 @@ rattn_status cp_layout_unpermute(const void* y, void* x, int B, int H, int64_t L
   return launch_unpermute(y, x, B * H, L, Lp, D * es, cp_size, layout, static_cast<cudaStream_t>(stream));
 }
 
+rattn_status cp_layout_varlen_plan(const int32_t* cu_seqlens, int nseq, int cp_size, rattn_layout layout,
+                                   int64_t* Tp, int32_t* src, int32_t* pos, int32_t* segid, int32_t* gkey) {
+  if (!cu_seqlens || nseq < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1 || !Tp) return RATTN_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return RATTN_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int i = 0; i < nseq; ++i) {
+    const int64_t L = static_cast<int64_t>(cu_seqlens[i + 1]) - cu_seqlens[i];
+    if (L < 0) return RATTN_ERR_INVALID_ARG;
+    total += cp_layout_padded_len(L, cp_size, layout);
+    if (total > INT32_MAX) return RATTN_ERR_INVALID_ARG;
+  }
+  *Tp = total;
+  if (!src && !pos && !segid && !gkey) return RATTN_OK;
+  // Rank r's slice holds, for every sequence in order, the rows rank r holds
+  // when that sequence alone is permuted.
+  const int64_t per_rank = total / cp_size;
+  int64_t seq_off = 0, rank_off = 0;  // sequence offset in the padded pack / in a rank slice
+  for (int i = 0; i < nseq; ++i) {
+    const int L = cu_seqlens[i + 1] - cu_seqlens[i];
+    const int Lp = static_cast<int>(cp_layout_padded_len(L, cp_size, layout));
+    const int n = Lp / cp_size;
+    const int c = cp_map_c(Lp, cp_size, layout);
+    for (int r = 0; r < cp_size; ++r) {
+      for (int t = 0; t < n; ++t) {
+        const int g = slot_to_global(r * n + t, c, cp_size, layout);
+        const int64_t slot = r * per_rank + rank_off + t;
+        if (src) src[slot] = g < L ? cu_seqlens[i] + g : -1;
+        if (pos) pos[slot] = g;
+        if (segid) segid[slot] = 2 * i + (g < L ? 0 : 1);
+        if (gkey) gkey[slot] = static_cast<int32_t>(seq_off + g);
+      }
+    }
+    seq_off += Lp;
+    rank_off += n;
+  }
+  return RATTN_OK;
+}
+
+static rattn_status check_gather(const void* a, const void* b, const int32_t* src, int B, int H, int64_t Ta,
+                                 int64_t Tb, int D, rattn_dtype dtype) {
+  const int es = elem_size(dtype);
+  if (!es || B < 1 || H < 1 || D < 1 || Ta < 0 || Tb < 0) return RATTN_ERR_INVALID_ARG;
+  if (Ta > INT32_MAX || Tb > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  const int64_t row = static_cast<int64_t>(D) * es;
+  if (row % 16 || row > 4096) return RATTN_ERR_UNSUPPORTED;
+  return RATTN_OK;
+}
+
+rattn_status cp_layout_gather(const void* x, void* y, const int32_t* src, int B, int H, int64_t T_in,
+                              int64_t T_out, int D, rattn_dtype dtype, void* stream) {
+  rattn_status st = check_gather(x, y, src, B, H, T_in, T_out, D, dtype);
+  if (st != RATTN_OK || T_out == 0) return st;
+  if (!y || !src || !aligned(y, 16) || !aligned(src, 4) || (T_in > 0 && (!x || !aligned(x, 16))))
+    return RATTN_ERR_INVALID_ARG;
+  return launch_gather(T_in > 0 ? x : y, y, src, B * H, T_in, T_out, D * elem_size(dtype),
+                       static_cast<cudaStream_t>(stream));
+}
+
+rattn_status cp_layout_scatter(const void* y, void* x, const int32_t* src, int B, int H, int64_t T_y,
+                               int64_t T_x, int D, rattn_dtype dtype, void* stream) {
+  rattn_status st = check_gather(y, x, src, B, H, T_y, T_x, D, dtype);
+  if (st != RATTN_OK || T_y == 0 || T_x == 0) return st;
+  if (!x || !y || !src || !aligned(x, 16) || !aligned(y, 16) || !aligned(src, 4)) return RATTN_ERR_INVALID_ARG;
+  return launch_scatter(y, x, src, B * H, T_y, T_x, D * elem_size(dtype), static_cast<cudaStream_t>(stream));
+}
+
 static rattn_status check_rope(int B, int H, int64_t L, int64_t Lp, int D, rattn_dtype dtype, int cp_size,
                                rattn_layout layout, double base, rattn_rope_style style) {
   const int es = elem_size(dtype);
@@ -269,9 +336,10 @@ rattn_status rattn_ring_fwd(const void* q, const void* k, const void* v, const i
                             stream);
 }
 
-rattn_status rattn_ring_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* pos, int B, int H,
-                                int H_kv, int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout,
-                                int causal, float scale, int64_t L_valid, void* o, float* lse, void* stream) {
+static rattn_status ring_fwd_impl(const void* q, const void* k, const void* v, const int32_t* pos,
+                                  const int32_t* seg, int B, int H, int H_kv, int64_t Lp, int D, rattn_dtype dtype,
+                                  int cp_size, rattn_layout layout, int causal, float scale, int64_t L_valid, void* o,
+                                  float* lse, void* stream) {
   if (H_kv < 1 || H < 1 || H % H_kv) return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_ring(q, k, v, pos, B, H, Lp, D, dtype, cp_size, layout, causal, scale);
   if (st != RATTN_OK || Lp == 0) return st;
@@ -282,6 +350,7 @@ rattn_status rattn_ring_fwd_gqa(const void* q, const void* k, const void* v, con
   a.v = v;
   a.q_pos = pos;
   a.kv_pos = pos;
+  a.seg = seg;
   a.BH = B * H;
   a.group = H / H_kv;
   a.nseg = cp_size;
@@ -304,6 +373,22 @@ rattn_status rattn_ring_fwd_gqa(const void* q, const void* k, const void* v, con
   return launch_fwd_simt(a);
 }
 
+rattn_status rattn_ring_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* pos, int B, int H,
+                                int H_kv, int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout,
+                                int causal, float scale, int64_t L_valid, void* o, float* lse, void* stream) {
+  return ring_fwd_impl(q, k, v, pos, nullptr, B, H, H_kv, Lp, D, dtype, cp_size, layout, causal, scale, L_valid, o,
+                       lse, stream);
+}
+
+rattn_status rattn_ring_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* gkey,
+                                   const int32_t* segid, int B, int H, int H_kv, int64_t Tp, int D,
+                                   rattn_dtype dtype, int cp_size, int causal, float scale, void* o, float* lse,
+                                   void* stream) {
+  if (Tp > 0 && (!segid || !aligned(segid, 4))) return RATTN_ERR_INVALID_ARG;
+  return ring_fwd_impl(q, k, v, gkey, segid, B, H, H_kv, Tp, D, dtype, cp_size, RATTN_LAYOUT_CONTIGUOUS, causal,
+                       scale, INT64_MAX, o, lse, stream);
+}
+
 size_t rattn_ring_bwd_workspace_size(int B, int H, int64_t Lp, int D) {
   if (B < 1 || H < 1 || Lp < 0 || D < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * static_cast<size_t>(Lp);
@@ -319,11 +404,11 @@ rattn_status rattn_ring_bwd(const void* q, const void* k, const void* v, const v
                             L_valid, dq, dk, dv, workspace, workspace_bytes, stream);
 }
 
-rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                                const float* lse, const int32_t* pos, int B, int H, int H_kv, int64_t Lp, int D,
-                                rattn_dtype dtype, int cp_size, rattn_layout layout, int causal, float scale,
-                                int64_t L_valid, void* dq, void* dk, void* dv, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+static rattn_status ring_bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                  const float* lse, const int32_t* pos, const int32_t* seg, int B, int H, int H_kv,
+                                  int64_t Lp, int D, rattn_dtype dtype, int cp_size, rattn_layout layout, int causal,
+                                  float scale, int64_t L_valid, void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
   if (H_kv < 1 || H < 1 || H % H_kv) return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_ring(q, k, v, pos, B, H, Lp, D, dtype, cp_size, layout, causal, scale);
   if (st != RATTN_OK || Lp == 0) return st;
@@ -341,6 +426,7 @@ rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, con
   a.dout = dout;
   a.lse = lse;
   a.pos = pos;
+  a.seg = seg;
   a.BH = B * H;
   a.group = H / H_kv;
   a.nseg = cp_size;
@@ -362,6 +448,26 @@ rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, con
     return launch_bwd_sm100(a, ctx);
   }
   return launch_bwd_simt(a);
+}
+
+rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                const float* lse, const int32_t* pos, int B, int H, int H_kv, int64_t Lp, int D,
+                                rattn_dtype dtype, int cp_size, rattn_layout layout, int causal, float scale,
+                                int64_t L_valid, void* dq, void* dk, void* dv, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return ring_bwd_impl(q, k, v, o, dout, lse, pos, nullptr, B, H, H_kv, Lp, D, dtype, cp_size, layout, causal, scale,
+                       L_valid, dq, dk, dv, workspace, workspace_bytes, stream);
+}
+
+rattn_status rattn_ring_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                   const float* lse, const int32_t* gkey, const int32_t* segid, int B, int H,
+                                   int H_kv, int64_t Tp, int D, rattn_dtype dtype, int cp_size, int causal,
+                                   float scale, void* dq, void* dk, void* dv, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (Tp > 0 && (!segid || !aligned(segid, 4))) return RATTN_ERR_INVALID_ARG;
+  return ring_bwd_impl(q, k, v, o, dout, lse, gkey, segid, B, H, H_kv, Tp, D, dtype, cp_size,
+                       RATTN_LAYOUT_CONTIGUOUS, causal, scale, INT64_MAX, dq, dk, dv, workspace, workspace_bytes,
+                       stream);
 }
 
 rattn_status rattn_get_device_error(int* site) {

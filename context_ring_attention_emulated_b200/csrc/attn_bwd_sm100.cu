@@ -57,7 +57,9 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_DELTA + NSQ * 128 * 4;
   static constexpr int NBAR = 1 + 2 * NSQ + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_HOP = OFF_MISC + 16;
+  static constexpr int OFF_FULL = OFF_MISC + 16;            // NSQ ints: tile needs no masking
+  static constexpr int OFF_HOP = OFF_FULL + 16;             // int2 table
+  static_assert(OFF_HOP % 8 == 0 && OFF_BAR % 8 == 0, "shared-memory alignment");
   static constexpr int SMEM = OFF_HOP + kMaxHops * 8;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -66,6 +68,7 @@ struct Params {
   const float* lse;
   const float* delta;
   const int32_t* pos;
+  const int32_t* seg;  // packed sequences: segid per slot, or NULL
   int BH, group, nseg, Lseg, nq_tiles, nk_tiles, causal;
   long long kv_valid;
   float scale, scale_log2;
@@ -75,6 +78,10 @@ struct Params {
   int* err;
   unsigned long long wait_ns;
 };
+
+__device__ __forceinline__ int segat(const Params& p, int rank, int row) {
+  return __ldg(p.seg + static_cast<long long>(rank) * p.Lseg + row);
+}
 
 __device__ __forceinline__ long long posat(const Params& p, int seg, int row) {
   return static_cast<long long>(__ldg(p.pos + static_cast<long long>(seg) * p.Lseg + row));
@@ -145,7 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
+  int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);       // per hop: visible query tiles [x, y)
+  volatile int* s_full = reinterpret_cast<volatile int*>(smem + C::OFF_FULL);  // per Q/dO stage
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* s_delta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
 
@@ -191,39 +199,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Per hop t the query segment is r = (s + t) mod nseg. Visible query tiles
   // form a suffix [first_vis, nq_tiles) and unmasked ones a suffix
   // [first_full, nq_tiles), since positions are non-decreasing in a segment.
+  // Per hop t the query segment is r = (s + t) mod nseg. Visible query tiles
+  // form a range [first_vis, end_vis): positions (and segids for packed
+  // sequences) are non-decreasing in a segment, so both ends are found by
+  // binary search; without packed sequences end_vis = nq_tiles.
   const bool live = k_min < p.kv_valid;
+  const int sk_lo = p.seg ? segat(p, s, k0) : 0;
+  const int sk_hi = p.seg ? segat(p, s, k0 + k_rows - 1) : 0;
   for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
     const int r = (s + t) % p.nseg;
-    int first_vis = p.nq_tiles, first_full = p.nq_tiles;
+    int first_vis = p.nq_tiles, end_vis = p.nq_tiles;
     if (live) {
-      if (!p.causal) {
-        first_vis = 0;
-        first_full = 0;
-      } else {
-        int lo = 0, hi = p.nq_tiles;
-        while (lo < hi) {  // first tile whose last query sees the first key
-          const int mid = (lo + hi) >> 1;
-          const long long qmax = posat(p, r, min((mid + 1) * BQ, p.Lseg) - 1);
-          if (qmax >= k_min) hi = mid; else lo = mid + 1;
-        }
-        first_vis = lo;
+      int lo = 0, hi = p.nq_tiles;
+      while (lo < hi) {  // first tile whose last query may see a key of this tile
+        const int mid = (lo + hi) >> 1;
+        const int last = min((mid + 1) * BQ, p.Lseg) - 1;
+        const bool reach = (!p.causal || posat(p, r, last) >= k_min) && (!p.seg || segat(p, r, last) >= sk_lo);
+        if (reach) hi = mid; else lo = mid + 1;
+      }
+      first_vis = lo;
+      if (p.seg) {
         hi = p.nq_tiles;
-        while (lo < hi) {  // first tile whose first query sees every key
+        while (lo < hi) {  // first tile wholly past the key tile's last segment
           const int mid = (lo + hi) >> 1;
-          const long long qmin = posat(p, r, mid * BQ);
-          if (qmin >= k_max) hi = mid; else lo = mid + 1;
+          if (segat(p, r, mid * BQ) > sk_hi) hi = mid; else lo = mid + 1;
         }
-        first_full = lo;
+        end_vis = lo;
       }
     }
-    s_hop[t] = make_int2(first_vis, first_full);
+    s_hop[t] = make_int2(first_vis, end_vis);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   int NIT = 0;
-  for (int t = 0; t < p.nseg; ++t) NIT += p.nq_tiles - s_hop[t].x;
+  for (int t = 0; t < p.nseg; ++t) NIT += s_hop[t].y - s_hop[t].x;
   NIT *= p.group;  // the same tiles for every query head of the group
 
   int issued_q = 0;
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bh = kvh * p.group + hq;  // (batch, query head)
       for (int t = 0; t < p.nseg && ok; ++t) {
         const int r = (s + t) % p.nseg;
-        for (int i = s_hop[t].x; i < p.nq_tiles; ++i, ++it) {
+        for (int i = s_hop[t].x; i < s_hop[t].y; ++i, ++it) {
           const int st = it % C::NSQ;
           const uint32_t u = it / C::NSQ;
           if (u > 0 && !warp_wait(&bar_q_empty[st], (u - 1) & 1, s_abort, p.wait_ns)) {
@@ -271,6 +282,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             s_lse[st * 128 + c] = l2;
             s_delta[st * 128 + c] = dl;
+          }
+          if (lane == 0) {
+            // No element of this tile pair is masked when every query sees
+            // every key: all in one real sequence (packed) and, when causal,
+            // the first query at or after the last key.
+            const int qa = i * BQ, qb = min(qa + BQ, p.Lseg) - 1;
+            bool full = !p.causal || posat(p, r, qa) >= k_max;
+            if (p.seg)
+              full = full && sk_lo == sk_hi && (sk_lo & 1) == 0 && segat(p, r, qa) == sk_lo && segat(p, r, qb) == sk_lo;
+            s_full[st] = full ? 1 : 0;
           }
           __syncwarp();
           if (lane == 0) {
@@ -356,7 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = row < k_rows;
     const long long my_kpos = key_ok ? posat(p, s, k0 + row) : k_max;
-    const bool key_dead = !key_ok || my_kpos >= p.kv_valid;
+    const int my_seg = (p.seg && key_ok) ? segat(p, s, k0 + row) : 0;
+    const bool key_dead = !key_ok || my_kpos >= p.kv_valid || (my_seg & 1);  // odd segid: padding
     const float sl2 = p.scale_log2;
     const int qc0 = wg * 64;              // first query column of this warpgroup
     const uint32_t t_a = tmem + lane_base + C::T_A + wg * 64;
@@ -368,23 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < p.nseg && ok; ++t) {
       const int r = (s + t) % p.nseg;
       const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
-      for (int i = s_hop[t].x; i < p.nq_tiles; ++i, ++it) {
+      for (int i = s_hop[t].x; i < s_hop[t].y; ++i, ++it) {
         const int st = it % C::NSQ;
         const float* lse2 = s_lse + st * 128 + qc0;
         const float* dlt = s_delta + st * 128 + qc0;
-        // first query column of this tile that sees this key (suffix)
-        int first = 0;
-        if (key_dead) {
-          first = BQ;
-        } else if (i < s_hop[t].y) {
-          int lo = 0, hi = min(BQ, p.Lseg - i * BQ);
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (posat(p, r, i * BQ + mid) >= my_kpos) hi = mid; else lo = mid + 1;
-          }
-          first = lo;
-        }
-        first -= qc0;  // relative to this warpgroup's columns
         if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns) ||
             !warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
@@ -392,6 +401,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        // query columns of this tile that see this key: [first, last)
+        int first = 0, last = BQ;
+        if (key_dead) {
+          first = BQ;
+        } else if (!s_full[st]) {
+          const int n = min(BQ, p.Lseg - i * BQ);
+          int lo = 0, hi = n;
+          while (lo < hi) {  // first query at or after this key (same sequence when packed)
+            const int mid = (lo + hi) >> 1;
+            const bool past = p.causal ? posat(p, r, i * BQ + mid) >= my_kpos
+                                       : (!p.seg || segat(p, r, i * BQ + mid) >= my_seg);
+            if (past) hi = mid; else lo = mid + 1;
+          }
+          first = lo;
+          if (p.seg) {
+            hi = n;
+            while (lo < hi) {  // first query of a later sequence
+              const int mid = (lo + hi) >> 1;
+              if (segat(p, r, i * BQ + mid) > my_seg) hi = mid; else lo = mid + 1;
+            }
+            last = lo;
+          }
+        }
+        first -= qc0;  // relative to this warpgroup's columns
+        last -= qc0;
         uint32_t sr[2][32];
         tmem_ld32(t_a, sr[0]);
         tmem_ld32(t_a + 32, sr[1]);
@@ -404,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c0 = 2 * e;
             float a = ex2_approx(fmaf(__uint_as_float(sr[c0 >> 5][c0 & 31]), sl2, -lse2[c0]));
             float b = ex2_approx(fmaf(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), sl2, -lse2[c0 + 1]));
-            a = c0 >= first ? a : 0.f;
-            b = c0 + 1 >= first ? b : 0.f;
+            a = (c0 >= first && c0 < last) ? a : 0.f;
+            b = (c0 + 1 >= first && c0 + 1 < last) ? b : 0.f;
             sr[c0 >> 5][c0 & 31] = __float_as_uint(a);
             sr[(c0 + 1) >> 5][(c0 + 1) & 31] = __float_as_uint(b);
             pk[e] = pack_bf16x2(a, b);
@@ -613,6 +647,7 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.lse = a.lse;
   p.delta = a.delta;
   p.pos = a.pos;
+  p.seg = a.seg;
   p.BH = a.BH;
   p.group = a.group;
   p.nseg = a.nseg;

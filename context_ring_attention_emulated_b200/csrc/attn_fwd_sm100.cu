@@ -56,14 +56,16 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_V + NS * TILE;
   static constexpr int NBAR = 1 + 4 * NS + NSB + NSB + NSB + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_HOP = OFF_MISC + 16;
-  static constexpr int SMEM = OFF_HOP + kMaxHops * 8 + 1024;  // + alignment slack
+  static constexpr int OFF_HOP = (OFF_MISC + 16 + 15) / 16 * 16;  // int4 table: 16-byte aligned
+  static constexpr int SMEM = OFF_HOP + kMaxHops * 16 + 1024;        // + alignment slack
+  static_assert(OFF_HOP % 16 == 0 && OFF_BAR % 8 == 0, "shared-memory alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 struct Params {
   const int32_t* q_pos;
   const int32_t* kv_pos;
+  const int32_t* seg;  // packed sequences: segid per slot (q and kv), or NULL
   int BH, group, nseg, Lq_seg, Lk_seg, n_qtiles, causal;
   long long kv_valid;
   float scale_log2;
@@ -79,6 +81,11 @@ __device__ __forceinline__ long long qpos(const Params& p, int seg, int row) {
 }
 __device__ __forceinline__ long long kpos(const Params& p, int seg, int row) {
   return p.kv_pos ? static_cast<long long>(__ldg(p.kv_pos + static_cast<long long>(seg) * p.Lk_seg + row)) : row;
+}
+// segid of a slot (packed sequences; only called when p.seg is set). Query and
+// key slots share one array (rank-major, Lq_seg == Lk_seg in ring calls).
+__device__ __forceinline__ int segat(const Params& p, int rank, int row) {
+  return __ldg(p.seg + static_cast<long long>(rank) * p.Lk_seg + row);
 }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -122,7 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_drain = bar_o_done + C::NSB;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
+  // per hop: x = first visible K/V tile, y = end of the visible tiles,
+  // [z, w) = tiles with no masked element
+  int4* s_hop = reinterpret_cast<int4*>(smem + C::OFF_HOP);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -161,36 +170,72 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) tmem_alloc(s_tmem, C::T_COLS);
 
-  // Per hop: n_vis = leading K/V tiles not fully masked, n_full = leading
-  // tiles with no masked element. Positions are non-decreasing within a
-  // segment, so both sets are prefixes found by binary search.
+  // Per hop: the K/V tiles not fully masked form a range [first, n_vis) and
+  // the tiles with no masked element a range [f_lo, f_hi) inside it; keys are
+  // sorted by position (and by segid for packed sequences) within a segment,
+  // so every bound is found by binary search. Without packed sequences the
+  // visible tiles are a prefix.
   for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
     const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-    int lo = 0, hi = nk_tiles;
+    const int sq_lo = p.seg ? segat(p, r, q0) : 0;
+    const int sq_hi = p.seg ? segat(p, r, q0 + q_rows - 1) : 0;
+    int first = 0;
+    if (p.seg) {  // first tile whose last key is in the query tile's first segment or later
+      int lo = 0, hi = nk_tiles;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (segat(p, s, min((mid + 1) * BN, p.Lk_seg) - 1) >= sq_lo) hi = mid; else lo = mid + 1;
+      }
+      first = lo;
+    }
+    int lo = first, hi = nk_tiles;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
       const long long kmin = kpos(p, s, mid * BN);
-      const bool vis = kmin < p.kv_valid && (!p.causal || kmin <= q_max);
+      const bool vis = kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!p.seg || segat(p, s, mid * BN) <= sq_hi);
       if (vis) lo = mid + 1; else hi = mid;
     }
     const int n_vis = lo;
-    lo = 0;
-    hi = n_vis;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      const bool complete = (mid + 1) * BN <= p.Lk_seg;
-      const long long kmax = kpos(p, s, min((mid + 1) * BN, p.Lk_seg) - 1);
-      const bool full = complete && kmax < p.kv_valid && (!p.causal || kmax <= q_min);
-      if (full) lo = mid + 1; else hi = mid;
+    int f_lo = first, f_hi = first;
+    const bool one_seg = !p.seg || (sq_lo == sq_hi && (sq_lo & 1) == 0);
+    if (one_seg && first < n_vis) {
+      int a = first, b = n_vis;
+      if (p.seg) {  // tiles lying wholly in the query tile's segment: [a, b)
+        lo = first;
+        hi = n_vis;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (segat(p, s, mid * BN) >= sq_lo) hi = mid; else lo = mid + 1;
+        }
+        a = lo;
+        lo = a;
+        hi = n_vis;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (segat(p, s, min((mid + 1) * BN, p.Lk_seg) - 1) > sq_lo) hi = mid; else lo = mid + 1;
+        }
+        b = lo;
+      }
+      lo = a;
+      hi = b;
+      while (lo < hi) {  // leading tiles of [a, b) visible to every query row
+        const int mid = (lo + hi) >> 1;
+        const bool complete = (mid + 1) * BN <= p.Lk_seg;
+        const long long kmax = kpos(p, s, min((mid + 1) * BN, p.Lk_seg) - 1);
+        const bool full = complete && kmax < p.kv_valid && (!p.causal || kmax <= q_min);
+        if (full) lo = mid + 1; else hi = mid;
+      }
+      f_lo = a;
+      f_hi = lo;
     }
-    s_hop[t] = make_int2(n_vis, lo);
+    s_hop[t] = make_int4(first, n_vis, f_lo, f_hi);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   int G = 0;
-  for (int t = 0; t < p.nseg; ++t) G += s_hop[t].x;
+  for (int t = 0; t < p.nseg; ++t) G += s_hop[t].y - s_hop[t].x;
 
   int issued_k = 0, issued_v = 0;  // producer bookkeeping for the drain
 
@@ -206,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0;
       for (int t = 0; t < p.nseg && ok; ++t) {
         const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-        const int nv = s_hop[t].x;
-        for (int j = 0; j < nv; ++j, ++g) {
+        const int nv = s_hop[t].y;
+        for (int j = s_hop[t].x; j < nv; ++j, ++g) {
           const int st = g % C::NS;
           const uint32_t u = g / C::NS;
           if (u > 0 && !mbar_wait(&bar_k_empty[st], (u - 1) & 1, s_abort, p.wait_ns)) {
@@ -299,14 +344,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool row_valid = row < q_rows;
     const long long my_pos = row_valid ? qpos(p, r, q0 + row) : q_max;
+    const int my_seg = (p.seg && row_valid) ? segat(p, r, q0 + row) : 1;  // odd: sees nothing
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int g = 0;
     for (int t = 0; t < p.nseg && ok; ++t) {
       const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-      const int nv = s_hop[t].x, nf = s_hop[t].y;
-      for (int j = 0; j < nv; ++j, ++g) {
+      const int nv = s_hop[t].y, f_lo = s_hop[t].z, f_hi = s_hop[t].w;
+      for (int j = s_hop[t].x; j < nv; ++j, ++g) {
         if (!warp_wait(&bar_s_full[g % C::NSB], (g / C::NSB) & 1, s_abort, p.wait_ns)) {
           record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
           ok = false;
@@ -318,20 +364,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sr[c]);
         tmem_wait_ld();
-        if (j >= nf) {
-          // Masked tile: the visible keys of this row form a prefix of the tile.
-          int lo = 0, hi = min(BN, p.Lk_seg - j * BN);
+        if (j < f_lo || j >= f_hi) {
+          // Masked tile: the visible keys of this row form a contiguous run
+          // [klo, khi) of the tile (a prefix without packed sequences).
+          const int n = min(BN, p.Lk_seg - j * BN);
+          int klo = 0;
+          if (p.seg) {
+            int lo = 0, hi = n;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (segat(p, s, j * BN + mid) >= my_seg) hi = mid; else lo = mid + 1;
+            }
+            klo = (my_seg & 1) ? n : lo;
+          }
+          int lo = klo, hi = n;
           while (lo < hi) {
             const int mid = (lo + hi) >> 1;
             const long long kp = kpos(p, s, j * BN + mid);
-            const bool vis = kp < p.kv_valid && (!p.causal || kp <= my_pos);
+            const bool vis = kp < p.kv_valid && (!p.causal || kp <= my_pos) &&
+                             (!p.seg || segat(p, s, j * BN + mid) == my_seg);
             if (vis) lo = mid + 1; else hi = mid;
           }
+          const int khi = lo;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (c * 32 + i >= lo) sr[c][i] = __float_as_uint(-INFINITY);
+              if (c * 32 + i < klo || c * 32 + i >= khi) sr[c][i] = __float_as_uint(-INFINITY);
         }
         float mx8[8];
 #pragma unroll
@@ -489,6 +548,7 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
   Params p;
   p.q_pos = a.q_pos;
   p.kv_pos = a.kv_pos;
+  p.seg = a.seg;
   p.BH = a.BH;
   p.group = a.group;
   p.nseg = a.nseg;

@@ -28,6 +28,7 @@ struct SimtFwd {
   const float* v;
   const int32_t* q_pos;
   const int32_t* kv_pos;
+  const int32_t* seg;  // packed sequences: segid per slot (q and kv share it), or NULL
   int BH, group, nseg, Lq_seg, Lk_seg, D, causal;
   long long kv_valid;
   float scale;
@@ -39,11 +40,19 @@ __device__ __forceinline__ long long pos_at(const int32_t* pos, long long base, 
   return pos ? static_cast<long long>(pos[base + row]) : row;
 }
 
+// Packed sequences: a key is visible only to queries with the same even segid.
+__device__ __forceinline__ bool seg_ok(const int32_t* seg, long long qi, long long ki) {
+  if (!seg) return true;
+  const int sk = seg[ki];
+  return sk == seg[qi] && (sk & 1) == 0;
+}
+
 template <int DMAX>
 __global__ void __launch_bounds__(kRows) fwd_simt_kernel(const SimtFwd p) {
   __shared__ float sk[kTile][DMAX];
   __shared__ float sv[kTile][DMAX];
   __shared__ long long skp[kTile];
+  __shared__ int sks[kTile];
   const int nqt = (p.Lq_seg + kRows - 1) / kRows;
   int item = blockIdx.x;
   const int qt = item % nqt;
@@ -53,6 +62,7 @@ __global__ void __launch_bounds__(kRows) fwd_simt_kernel(const SimtFwd p) {
   const int row = qt * kRows + threadIdx.x;
   const bool valid = row < p.Lq_seg;
   const long long qbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lq_seg;
+  const int my_seg = p.seg ? p.seg[static_cast<long long>(r) * p.Lq_seg + (valid ? row : 0)] : 0;
   const int last_row = min(qt * kRows + kRows, p.Lq_seg) - 1;
   const long long my_pos = pos_at(p.q_pos, static_cast<long long>(r) * p.Lq_seg, valid ? row : last_row);
   const long long blk_max = pos_at(p.q_pos, static_cast<long long>(r) * p.Lq_seg, last_row);
@@ -79,12 +89,15 @@ __global__ void __launch_bounds__(kRows) fwd_simt_kernel(const SimtFwd p) {
         sk[kr][d] = in ? p.k[(kbase + k0 + kr) * p.D + d] : 0.f;
         sv[kr][d] = in ? p.v[(kbase + k0 + kr) * p.D + d] : 0.f;
       }
-      for (int kr = threadIdx.x; kr < kTile; kr += kRows)
+      for (int kr = threadIdx.x; kr < kTile; kr += kRows) {
         skp[kr] = kr < n ? pos_at(p.kv_pos, static_cast<long long>(s) * p.Lk_seg, k0 + kr) : LLONG_MAX;
+        sks[kr] = (kr < n && p.seg) ? p.seg[static_cast<long long>(s) * p.Lk_seg + k0 + kr] : 0;
+      }
       __syncthreads();
       for (int kr = 0; kr < n; ++kr) {
         const long long kp = skp[kr];
         if (kp >= p.kv_valid || (p.causal && kp > my_pos)) continue;
+        if (p.seg && (sks[kr] != my_seg || (my_seg & 1))) continue;
         float x = 0.f;
 #pragma unroll
         for (int d = 0; d < DMAX; ++d) x = fmaf(qr[d], sk[kr][d], x);
@@ -120,6 +133,7 @@ struct SimtBwd {
   const float* dout;
   const float* lse;
   const int32_t* pos;
+  const int32_t* seg;  // packed sequences: segid per slot, or NULL
   int BH, group, nseg, Lseg, D, causal;
   long long kv_valid;
   float scale;
@@ -155,6 +169,7 @@ __global__ void __launch_bounds__(kRows) dq_simt_kernel(const SimtBwd p) {
   const int last_row = min(qt * kRows + kRows, p.Lseg) - 1;
   const long long my_pos = p.pos[static_cast<long long>(r) * p.Lseg + (valid ? row : last_row)];
   const long long blk_max = p.pos[static_cast<long long>(r) * p.Lseg + last_row];
+  const long long my_slot = static_cast<long long>(r) * p.Lseg + (valid ? row : last_row);
   float qr[DMAX], dor[DMAX], g[DMAX];
 #pragma unroll
   for (int d = 0; d < DMAX; ++d) {
@@ -185,6 +200,7 @@ __global__ void __launch_bounds__(kRows) dq_simt_kernel(const SimtBwd p) {
       for (int kr = 0; kr < n; ++kr) {
         const long long kp = skp[kr];
         if (kp >= p.kv_valid || (p.causal && kp > my_pos)) continue;
+        if (!seg_ok(p.seg, my_slot, static_cast<long long>(s) * p.Lseg + k0 + kr)) continue;
         float x = 0.f, dp = 0.f;
 #pragma unroll
         for (int d = 0; d < DMAX; ++d) {
@@ -224,6 +240,7 @@ __global__ void __launch_bounds__(kRows) dkdv_simt_kernel(const SimtBwd p) {
   const long long my_pos = p.pos[static_cast<long long>(s) * p.Lseg + (valid ? row : first_row)];
   const long long blk_min = p.pos[static_cast<long long>(s) * p.Lseg + first_row];
   const bool key_live = valid && my_pos < p.kv_valid;
+  const long long my_slot = static_cast<long long>(s) * p.Lseg + (valid ? row : first_row);
   float kr_[DMAX], vr[DMAX], gk[DMAX], gv[DMAX];
 #pragma unroll
   for (int d = 0; d < DMAX; ++d) {
@@ -255,6 +272,7 @@ __global__ void __launch_bounds__(kRows) dkdv_simt_kernel(const SimtBwd p) {
       if (!key_live) continue;
       for (int qr = 0; qr < n; ++qr) {
         if (p.causal && my_pos > sqp[qr]) continue;
+        if (!seg_ok(p.seg, static_cast<long long>(r) * p.Lseg + q0 + qr, my_slot)) continue;
         float x = 0.f, dp = 0.f;
 #pragma unroll
         for (int d = 0; d < DMAX; ++d) {
@@ -314,6 +332,7 @@ rattn_status launch_fwd_simt(const FwdArgs& a) {
   p.v = static_cast<const float*>(a.v);
   p.q_pos = a.q_pos;
   p.kv_pos = a.kv_pos;
+  p.seg = a.seg;
   p.BH = a.BH;
   p.group = a.group;
   p.nseg = a.nseg;
@@ -342,6 +361,7 @@ rattn_status launch_bwd_simt(const BwdArgs& a) {
   p.dout = static_cast<const float*>(a.dout);
   p.lse = a.lse;
   p.pos = a.pos;
+  p.seg = a.seg;
   p.BH = a.BH;
   p.group = a.group;
   p.nseg = a.nseg;

@@ -12,7 +12,7 @@
 namespace rattn {
 
 // Global position held by slot i of the permuted sequence.
-__device__ __forceinline__ int slot_to_global(int i, int c, int cp, int layout) {
+__host__ __device__ __forceinline__ int slot_to_global(int i, int c, int cp, int layout) {
   if (layout == RATTN_LAYOUT_CONTIGUOUS) return i;
   if (layout == RATTN_LAYOUT_STRIPED) {
     const int r = i / c;
@@ -24,7 +24,7 @@ __device__ __forceinline__ int slot_to_global(int i, int c, int cp, int layout) 
 }
 
 // Slot of the permuted sequence that holds global position g.
-__device__ __forceinline__ int global_to_slot(int g, int c, int cp, int layout) {
+__host__ __device__ __forceinline__ int global_to_slot(int g, int c, int cp, int layout) {
   if (layout == RATTN_LAYOUT_CONTIGUOUS) return g;
   if (layout == RATTN_LAYOUT_STRIPED) {
     const int j = g / cp;

@@ -52,6 +52,7 @@ struct FwdArgs {
   const void* v;
   const int32_t* q_pos;   // [nseg*Lq_seg] or NULL (row index)
   const int32_t* kv_pos;  // [nseg*Lk_seg] or NULL (row index)
+  const int32_t* seg = nullptr;  // packed sequences: segid per slot (shared by q and kv), or NULL
   int BH;         // batch x query heads
   int group = 1;  // query heads per key/value head (GQA); K/V hold BH / group heads
   int nseg;
@@ -78,6 +79,7 @@ struct BwdArgs {
   const void* dout;
   const float* lse;
   const int32_t* pos;  // [nseg*Lseg]
+  const int32_t* seg = nullptr;  // packed sequences: segid per slot, or NULL
   int BH;              // batch x query heads
   int group = 1;       // query heads per key/value head (GQA); K/V, dK, dV hold BH / group heads
   int nseg;
@@ -99,6 +101,10 @@ rattn_status launch_bwd_simt(const BwdArgs& a);
 
 rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int row_bytes,
                             int cp, int layout, cudaStream_t stream);
+rattn_status launch_gather(const void* x, void* y, const int32_t* src, int BH, int64_t T_in, int64_t T_out,
+                           int row_bytes, cudaStream_t stream);
+rattn_status launch_scatter(const void* y, void* x, const int32_t* src, int BH, int64_t T_y, int64_t T_x,
+                            int row_bytes, cudaStream_t stream);
 rattn_status launch_unpermute(const void* y, void* x, int BH, int64_t L, int64_t Lp, int row_bytes, int cp,
                               int layout, cudaStream_t stream);
 rattn_status launch_permute_rope(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int D,

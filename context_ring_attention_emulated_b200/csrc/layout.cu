@@ -54,6 +54,42 @@ __global__ void unpermute_kernel(const uint4* __restrict__ y, uint4* __restrict_
   }
 }
 
+// Varlen gather: y[bh][i] = src[i] in [0, T_in) ? x[bh][src[i]] : 0.
+__global__ void gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, const int32_t* __restrict__ src,
+                              int BH, int T_in, int T_out, int vpr) {
+  const int e = threadIdx.x % vpr;
+  const int rsub = threadIdx.x / vpr;
+  const int rpb = blockDim.x / vpr;
+  if (rsub >= rpb) return;
+  for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+    const uint4* xb = x + static_cast<long long>(bh) * T_in * vpr;
+    uint4* yb = y + static_cast<long long>(bh) * T_out * vpr;
+    for (int i = blockIdx.x * rpb + rsub; i < T_out; i += gridDim.x * rpb) {
+      const int g = __ldg(src + i);
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      if (g >= 0 && g < T_in) val = __ldg(xb + static_cast<long long>(g) * vpr + e);
+      yb[static_cast<long long>(i) * vpr + e] = val;
+    }
+  }
+}
+
+// Varlen scatter: x[bh][src[i]] = y[bh][i] for src[i] in [0, T_x).
+__global__ void scatter_kernel(const uint4* __restrict__ y, uint4* __restrict__ x, const int32_t* __restrict__ src,
+                               int BH, int T_y, int T_x, int vpr) {
+  const int e = threadIdx.x % vpr;
+  const int rsub = threadIdx.x / vpr;
+  const int rpb = blockDim.x / vpr;
+  if (rsub >= rpb) return;
+  for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+    const uint4* yb = y + static_cast<long long>(bh) * T_y * vpr;
+    uint4* xb = x + static_cast<long long>(bh) * T_x * vpr;
+    for (int i = blockIdx.x * rpb + rsub; i < T_y; i += gridDim.x * rpb) {
+      const int g = __ldg(src + i);
+      if (g >= 0 && g < T_x) xb[static_cast<long long>(g) * vpr + e] = __ldg(yb + static_cast<long long>(i) * vpr + e);
+    }
+  }
+}
+
 // Grid for rows x BH work items: about 16 resident 256-thread blocks per SM.
 dim3 grid_2d(long long rows, int BH, int rpb) {
   int dev = 0, sms = 148;
@@ -69,6 +105,26 @@ dim3 grid_2d(long long rows, int BH, int rpb) {
 
 
 }  // namespace
+
+rattn_status launch_gather(const void* x, void* y, const int32_t* src, int BH, int64_t T_in, int64_t T_out,
+                           int row_bytes, cudaStream_t stream) {
+  const int vpr = row_bytes / 16;
+  if (vpr > 256) return RATTN_ERR_UNSUPPORTED;
+  gather_kernel<<<grid_2d(T_out, BH, 256 / vpr), 256, 0, stream>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), src, BH, static_cast<int>(T_in), static_cast<int>(T_out),
+      vpr);
+  return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
+}
+
+rattn_status launch_scatter(const void* y, void* x, const int32_t* src, int BH, int64_t T_y, int64_t T_x,
+                            int row_bytes, cudaStream_t stream) {
+  const int vpr = row_bytes / 16;
+  if (vpr > 256) return RATTN_ERR_UNSUPPORTED;
+  scatter_kernel<<<grid_2d(T_y, BH, 256 / vpr), 256, 0, stream>>>(
+      static_cast<const uint4*>(y), static_cast<uint4*>(x), src, BH, static_cast<int>(T_y), static_cast<int>(T_x),
+      vpr);
+  return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
+}
 
 rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int row_bytes,
                             int cp, int layout, cudaStream_t stream) {

@@ -33,6 +33,12 @@ SIGNATURES = [
     ("cp_layout_padded_len", _I64, [_I64, _I, _I]),
     ("cp_layout_permute", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
     ("cp_layout_unpermute", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
+    ("cp_layout_varlen_plan", _I, [_P, _I, _I, _I, ctypes.POINTER(_I64), _P, _P, _P, _P]),
+    ("cp_layout_gather", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _P]),
+    ("cp_layout_scatter", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _P]),
+    ("rattn_ring_fwd_varlen", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _P, _P]),
+    ("rattn_ring_bwd_varlen", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _I, _F,
+                                   _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("cp_layout_permute_rope", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _D, _I, _P]),
     ("cp_layout_unpermute_rope_grad", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _D, _I, _P]),
     ("rattn_partial_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I, _I, _F, _I, _I64, _P, _P, _P]),
@@ -166,6 +172,83 @@ def cp_layout_unpermute_rope_grad(dy, L, cp_size, layout=LAYOUT_HEAD_TAIL, rope_
         _ptr(dy), _ptr(dx), B, H, L, Lp, D, _dtype_code(dy), cp_size, layout, float(rope_base), int(style),
         _stream(stream)))
     return dx
+
+
+def cp_layout_varlen_plan(cu_seqlens, cp_size, layout=LAYOUT_HEAD_TAIL):
+    """Host-side layout of a pack of sequences (boundaries cu_seqlens, a list or
+    1-D int tensor starting at 0). Returns a dict of CPU int32 tensors
+    src, pos, segid, gkey [Tp] and Tp."""
+    cu = torch.as_tensor(cu_seqlens, dtype=torch.int32).contiguous().cpu()
+    nseq = cu.numel() - 1
+    tp = ctypes.c_int64(0)
+    _check("cp_layout_varlen_plan", lib.cp_layout_varlen_plan(_ptr(cu), nseq, cp_size, layout, ctypes.byref(tp),
+                                                                None, None, None, None))
+    out = {n: torch.empty(tp.value, dtype=torch.int32) for n in ("src", "pos", "segid", "gkey")}
+    _check("cp_layout_varlen_plan", lib.cp_layout_varlen_plan(
+        _ptr(cu), nseq, cp_size, layout, ctypes.byref(tp), _ptr(out["src"]), _ptr(out["pos"]), _ptr(out["segid"]),
+        _ptr(out["gkey"])))
+    out["Tp"] = tp.value
+    return out
+
+
+def cp_layout_gather(x, src, y=None, stream=None):
+    """y[:, :, i] = x[:, :, src[i]] (zero rows where src[i] < 0); src device int32."""
+    _need_cuda(x, src)
+    B, H, T, D = x.shape
+    T_out = src.numel()
+    if y is None:
+        y = torch.empty(B, H, T_out, D, dtype=x.dtype, device=x.device)
+    _need_cuda(y)
+    _check("cp_layout_gather", lib.cp_layout_gather(_ptr(x), _ptr(y), _ptr(src), B, H, T, T_out, D, _dtype_code(x),
+                                                     _stream(stream)))
+    return y
+
+
+def cp_layout_scatter(y, src, T_x, x=None, stream=None):
+    """x[:, :, src[i]] = y[:, :, i] for src[i] >= 0; x [B, H, T_x, D]."""
+    _need_cuda(y, src)
+    B, H, T_y, D = y.shape
+    if x is None:
+        x = torch.zeros(B, H, T_x, D, dtype=y.dtype, device=y.device)
+    _need_cuda(x)
+    _check("cp_layout_scatter", lib.cp_layout_scatter(_ptr(y), _ptr(x), _ptr(src), B, H, T_y, T_x, D,
+                                                       _dtype_code(y), _stream(stream)))
+    return x
+
+
+def rattn_ring_fwd_varlen(q, k, v, gkey, segid, cp_size, causal=True, scale=None, o=None, lse=None, stream=None):
+    """Ring forward over a packed layout (cp_layout_varlen_plan order); gkey and
+    segid device int32 [Tp]. Returns (O, LSE)."""
+    _need_cuda(q, k, v, gkey, segid)
+    B, H, Tp, D = q.shape
+    H_kv = k.shape[1]
+    scale = D ** -0.5 if scale is None else scale
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(B, H, Tp, dtype=torch.float32, device=q.device) if lse is None else lse
+    _check("rattn_ring_fwd_varlen", lib.rattn_ring_fwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gkey), _ptr(segid), B, H, H_kv, Tp, D, _dtype_code(q), cp_size, int(causal),
+        float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+    return o, lse
+
+
+def rattn_ring_bwd_varlen(q, k, v, o, dout, lse, gkey, segid, cp_size, causal=True, scale=None, dq=None, dk=None,
+                          dv=None, workspace=None, stream=None):
+    """Gradients of rattn_ring_fwd_varlen: returns (dQ, dK, dV)."""
+    _need_cuda(q, k, v, o, dout, lse, gkey, segid)
+    B, H, Tp, D = q.shape
+    H_kv = k.shape[1]
+    scale = D ** -0.5 if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = rattn_ring_bwd_workspace_size(B, H, Tp, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check("rattn_ring_bwd_varlen", lib.rattn_ring_bwd_varlen(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(gkey), _ptr(segid), B, H, H_kv, Tp, D,
+        _dtype_code(q), cp_size, int(causal), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def rattn_partial_fwd(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True, kv_valid=2**62,

@@ -34,6 +34,7 @@ class Workload:
     bwd: bool = False
     H_kv: int = 0       # key/value heads (grouped-query attention); 0 means H
     rope: bool = False  # rotate Q and K at their global positions while permuting
+    docs: tuple = ()    # packed sequences: document lengths summing to L (empty: one sequence)
 
     @property
     def kv_heads(self):
@@ -48,9 +49,33 @@ class Workload:
         return self.D ** -0.5
 
     def causal_flops_fwd(self):
-        """Algorithmic forward FLOPs: 4*B*H*D*L^2, halved when causal."""
-        f = 4.0 * self.B * self.H * self.D * self.L * self.L
+        """Algorithmic forward FLOPs: 4*B*H*D*L^2, halved when causal; for a
+        pack of documents the sum of L_i^2 over the documents replaces L^2."""
+        sq = sum(d * d for d in self.docs) if self.docs else self.L * self.L
+        f = 4.0 * self.B * self.H * self.D * sq
         return f / 2 if self.causal else f
+
+    @property
+    def cu_seqlens(self):
+        out = [0]
+        for d in self.docs:
+            out.append(out[-1] + d)
+        return out
+
+
+def doc_lengths(total, n, lo, hi, seed):
+    """Seeded document lengths for a pack: n - 1 lengths drawn uniformly from
+    [lo, hi), the last one taking the rest of ``total`` (the draws are cut
+    short if they already reach it)."""
+    g = torch.Generator().manual_seed(seed)
+    out = []
+    for _ in range(n - 1):
+        d = int(torch.randint(lo, hi, (1,), generator=g).item())
+        if sum(out) + d >= total:
+            break
+        out.append(d)
+    out.append(total - sum(out))
+    return tuple(out)
 
 
 WORKLOADS = {
@@ -70,6 +95,11 @@ WORKLOADS = {
     # The 32k / cp=4 step with 8 key/value heads shared by 32 query heads (GQA).
     "bf16_L32000_cp4_gqa8_fwdbwd": Workload("bf16_L32000_cp4_gqa8_fwdbwd", "bf16", 1, 32, 32000, 128, True, 4,
                                             LAYOUT_HEAD_TAIL, 1.0, True, H_kv=8),
+    # A 32,000-token pack of 24 documents (23 drawn from 64..2599 tokens, the last
+    # taking the rest) laid out per
+    # document (packed sequences), cp=4 head-tail, causal within documents.
+    "bf16_L32000_cp4_varlen_fwdbwd": Workload("bf16_L32000_cp4_varlen_fwdbwd", "bf16", 1, 32, 32000, 128, True, 4,
+                                              LAYOUT_HEAD_TAIL, 1.0, True, docs=doc_lengths(32000, 24, 64, 2600, 7)),
     # The 32k / cp=4 step with RoPE fused into the permute of Q, K and the
     # unpermute of dQ, dK.
     "bf16_L32000_cp4_rope_fwdbwd": Workload("bf16_L32000_cp4_rope_fwdbwd", "bf16", 1, 32, 32000, 128, True, 4,

@@ -139,6 +139,63 @@ rattn_status cp_layout_unpermute_rope_grad(const void* dy, void* dx,
                                            rattn_dtype dtype, int cp_size, rattn_layout layout,
                                            double rope_base, rattn_rope_style style, void* stream);
 
+/* Packed sequences (varlen). [Megatron-CP] "Symmetric chunk assignment":
+ * packed-sequence metadata must follow the pairing structure. Each sequence of
+ * the pack (boundaries cu_seqlens [nseq + 1], host, starting at 0 and
+ * non-decreasing) is laid out on its own: padded to its own multiple (2 *
+ * cp_size for HEAD_TAIL, cp_size otherwise) and permuted as
+ * cp_layout_permute would permute it alone; rank r's slice then holds rank
+ * r's share of every sequence, sequences in pack order. Host only; no device
+ * work. Writes Tp (the permuted pack length, a multiple of cp_size) and, when
+ * the pointers are non-NULL, per slot [Tp] (host arrays):
+ *   src   index into the unpadded pack, or -1 for a pad slot;
+ *   pos   position inside the sequence (what RoPE uses; pads continue it);
+ *   segid 2 * (sequence index) for real tokens, 2 * (sequence index) + 1 for
+ *         pads: non-decreasing along every rank slice;
+ *   gkey  offset of the sequence in the padded pack + pos: increasing along
+ *         every rank slice.
+ * Call once with the array pointers NULL to learn Tp. Returns
+ * RATTN_ERR_INVALID_ARG on bad boundaries, cp_size < 1, unknown layout or a
+ * pack longer than INT32_MAX slots. */
+rattn_status cp_layout_varlen_plan(const int32_t* cu_seqlens, int nseq, int cp_size, rattn_layout layout,
+                                   int64_t* Tp, int32_t* src, int32_t* pos, int32_t* segid, int32_t* gkey);
+
+/* Row gather for the varlen layout: y [B,H,T_out,D] with
+ * y[:, :, i] = x[:, :, src[i]] for src[i] >= 0 and zero rows where
+ * src[i] < 0; src is a device int32 array [T_out] with entries < T_in
+ * (cp_layout_varlen_plan's src, copied to the device). Bit-exact copy; rows
+ * a multiple of 16 bytes and at most 4 KB. x and y must not overlap. */
+rattn_status cp_layout_gather(const void* x, void* y, const int32_t* src, int B, int H, int64_t T_in,
+                              int64_t T_out, int D, rattn_dtype dtype, void* stream);
+
+/* Inverse of cp_layout_gather for a src whose non-negative entries are
+ * distinct: x[:, :, src[i]] = y[:, :, i] for src[i] >= 0 (pad rows of y are
+ * dropped; rows of x that no entry names are left untouched). y [B,H,T_y,D],
+ * x [B,H,T_x,D], src device int32 [T_y]. */
+rattn_status cp_layout_scatter(const void* y, void* x, const int32_t* src, int B, int H, int64_t T_y,
+                               int64_t T_x, int D, rattn_dtype dtype, void* stream);
+
+/* Ring forward over a packed (varlen) layout: q [B,H,Tp,D], k and v
+ * [B,H_kv,Tp,D] (H a multiple of H_kv, as rattn_ring_fwd_gqa) in the order
+ * cp_layout_varlen_plan describes, with its gkey and segid arrays (device
+ * int32 [Tp]). A key is visible to a query iff both carry the same even
+ * segid (same sequence, not padding) and, when causal, gkey_key <= gkey_query.
+ * Outputs o [B,H,Tp,D] in `dtype` and lse fp32 [B,H,Tp]; rows of pad slots
+ * have lse = -inf and o = 0. Tp must be a multiple of cp_size. */
+rattn_status rattn_ring_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* gkey,
+                                   const int32_t* segid, int B, int H, int H_kv, int64_t Tp, int D,
+                                   rattn_dtype dtype, int cp_size, int causal, float scale, void* o, float* lse,
+                                   void* stream);
+
+/* Gradients of rattn_ring_fwd_varlen: dq [B,H,Tp,D]; dk, dv [B,H_kv,Tp,D].
+ * Inputs as rattn_ring_fwd_varlen plus o, dout (`dtype`) and lse; workspace as
+ * rattn_ring_bwd (rattn_ring_bwd_workspace_size(B, H, Tp, D) bytes). */
+rattn_status rattn_ring_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                   const float* lse, const int32_t* gkey, const int32_t* segid, int B, int H,
+                                   int H_kv, int64_t Tp, int D, rattn_dtype dtype, int cp_size, int causal,
+                                   float scale, void* dq, void* dk, void* dv, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* [CP-glossary], [Ring-page]: one partial attention of local queries against
  * one K/V block. q [B,H,Lq,D], k and v [B,H,Lk,D] in `dtype`; q_pos int32
  * [Lq] and kv_pos int32 [Lk] (either may be NULL, meaning 0,1,2,...);

@@ -5,7 +5,9 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
+import torch
 
 from tests.gpu_common import load_rattn
 
@@ -164,3 +166,49 @@ def test_bwd_rejects_bad_arguments_and_sizes_workspace(rattn):
     assert bwd(ws=FAKE + 16) == rattn.ERR_INVALID_ARG   # workspace must be 256-byte aligned
     assert bwd(ws=None) == rattn.ERR_INVALID_ARG
     assert bwd(dv=None) == rattn.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("layout", [0, 1, 2])
+@pytest.mark.parametrize("cp", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("cu", [[0, 5, 16, 16, 23], [0, 64], [0], [0, 1, 2, 3], [0, 4000, 4001, 9000, 32000]])
+def test_varlen_plan_matches_oracle(rattn, layout, cp, cu):
+    """The library's host-side packed layout against the oracle's, slot by slot;
+    the kernels' segid is 2 * sequence (+1 for padding)."""
+    import oracle
+    plan = rattn.cp_layout_varlen_plan(cu, cp, layout)
+    Tp, src, pos, seg, gkey = oracle.varlen_index(cu, cp, layout)
+    assert plan["Tp"] == Tp
+    assert np.array_equal(plan["src"].numpy(), src)
+    assert np.array_equal(plan["pos"].numpy(), pos)
+    assert np.array_equal(plan["gkey"].numpy(), gkey)
+    seq = np.repeat(np.arange(len(cu) - 1), [oracle.padded_len(b - a, cp, layout) for a, b in zip(cu, cu[1:])])
+    # every pad slot belongs to its sequence's block: recover the sequence of each slot from gkey
+    offsets = np.cumsum([0] + [oracle.padded_len(b - a, cp, layout) for a, b in zip(cu, cu[1:])])
+    slot_seq = np.searchsorted(offsets, gkey, side="right") - 1 if Tp else np.zeros(0, int)
+    assert np.array_equal(plan["segid"].numpy(), 2 * slot_seq + (src < 0))
+    assert np.array_equal(np.where(src >= 0, slot_seq, -1), seg)
+    assert len(seq) == Tp
+
+
+def test_varlen_calls_reject_bad_arguments(rattn):
+    L = rattn.lib
+    tp = ctypes.c_int64(0)
+    bad = torch.tensor([0, 5, 3], dtype=torch.int32)
+    assert L.cp_layout_varlen_plan(bad.data_ptr(), 2, 2, 1, ctypes.byref(tp), None, None, None, None) == \
+        rattn.ERR_INVALID_ARG
+    start = torch.tensor([1, 5], dtype=torch.int32)
+    assert L.cp_layout_varlen_plan(start.data_ptr(), 1, 2, 1, ctypes.byref(tp), None, None, None, None) == \
+        rattn.ERR_INVALID_ARG
+    ok = torch.tensor([0, 5], dtype=torch.int32)
+    assert L.cp_layout_varlen_plan(ok.data_ptr(), 1, 0, 1, ctypes.byref(tp), None, None, None, None) == \
+        rattn.ERR_INVALID_ARG
+    assert L.cp_layout_gather(FAKE, FAKE, FAKE, 1, 1, 16, 16, 3, 1, None) == rattn.ERR_UNSUPPORTED
+    assert L.cp_layout_gather(FAKE, MIS, FAKE, 1, 1, 16, 16, 64, 1, None) == rattn.ERR_INVALID_ARG
+    assert L.cp_layout_gather(FAKE, FAKE, FAKE, 1, 1, 16, 0, 64, 1, None) == rattn.OK
+    assert L.cp_layout_scatter(FAKE, FAKE, None, 1, 1, 16, 16, 64, 1, None) == rattn.ERR_INVALID_ARG
+    fv = L.rattn_ring_fwd_varlen(FAKE, FAKE, FAKE, FAKE, None, 1, 2, 2, 256, 64, 1, 2, 1, ctypes.c_float(0.125),
+                                 FAKE, FAKE, None)
+    assert fv == rattn.ERR_INVALID_ARG            # segid required
+    fv = L.rattn_ring_fwd_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 255, 64, 1, 2, 1, ctypes.c_float(0.125),
+                                 FAKE, FAKE, None)
+    assert fv == rattn.ERR_INVALID_ARG            # Tp not a multiple of cp
