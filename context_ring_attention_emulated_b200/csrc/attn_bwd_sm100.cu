@@ -26,6 +26,7 @@
 // TMEM columns: A [0,128) S^T; warpgroup g then overwrites its own columns
 // [64g, 64g+64) with P^T (bf16, [64g, 64g+32)) and dS^T ([64g+32, 64g+64));
 // B [128,256) dP^T, then dQ; dV [256,256+D); dK [256+D,256+2D).
+#include <limits.h>
 #include <math.h>
 
 #include "internal.h"
@@ -401,29 +402,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        // query columns of this tile that see this key: [first, last)
+        // query columns of this tile that see this key: [first, last). The
+        // tile's query positions and segids are spread over the warp (four
+        // per lane) and searched through shuffles (all lanes, eight steps).
         int first = 0, last = BQ;
-        if (key_dead) {
-          first = BQ;
-        } else if (!s_full[st]) {
+        if (!s_full[st]) {  // the same for the whole warp
           const int n = min(BQ, p.Lseg - i * BQ);
+          const long long qbase = static_cast<long long>(r) * p.Lseg + i * BQ;
+          int qp4[4], qs4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int idx = 4 * lane + e;
+            qp4[e] = idx < n ? __ldg(p.pos + qbase + idx) : INT_MAX;
+            qs4[e] = (p.seg && idx < n) ? __ldg(p.seg + qbase + idx) : INT_MAX;
+          }
           int lo = 0, hi = n;
-          while (lo < hi) {  // first query at or after this key (same sequence when packed)
+#pragma unroll 1
+          for (int step = 0; step < 8; ++step) {  // first query at or after this key (same sequence when packed)
             const int mid = (lo + hi) >> 1;
-            const bool past = p.causal ? posat(p, r, i * BQ + mid) >= my_kpos
-                                       : (!p.seg || segat(p, r, i * BQ + mid) >= my_seg);
-            if (past) hi = mid; else lo = mid + 1;
+            const int qp = warp_elem128(qp4, mid);
+            const int qs = p.seg ? warp_elem128(qs4, mid) : 0;
+            const bool past = p.causal ? qp >= my_kpos : (!p.seg || qs >= my_seg);
+            if (lo < hi) {
+              if (past) hi = mid; else lo = mid + 1;
+            }
           }
           first = lo;
           if (p.seg) {
             hi = n;
-            while (lo < hi) {  // first query of a later sequence
+#pragma unroll 1
+            for (int step = 0; step < 8; ++step) {  // first query of a later sequence
               const int mid = (lo + hi) >> 1;
-              if (segat(p, r, i * BQ + mid) > my_seg) hi = mid; else lo = mid + 1;
+              const int qs = warp_elem128(qs4, mid);
+              if (lo < hi) {
+                if (qs > my_seg) hi = mid; else lo = mid + 1;
+              }
             }
             last = lo;
           }
         }
+        if (key_dead) first = BQ;
         first -= qc0;  // relative to this warpgroup's columns
         last -= qc0;
         uint32_t sr[2][32];

@@ -28,6 +28,7 @@
 // written over the first 64 columns of its own score buffer. The MMA that
 // next overwrites that buffer (S_{g+3}) is issued only after the PV MMA
 // reading P_g has completed.
+#include <limits.h>
 #include <math.h>
 
 #include "internal.h"
@@ -366,24 +367,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if (j < f_lo || j >= f_hi) {
           // Masked tile: the visible keys of this row form a contiguous run
-          // [klo, khi) of the tile (a prefix without packed sequences).
+          // [klo, khi) of the tile (a prefix without packed sequences). The
+          // tile's key positions and segids are spread over the warp (four
+          // per lane, coalesced loads) and every row's bounds come from
+          // binary searches over them through shuffles (eight steps cover 128
+          // keys; all lanes take every step).
           const int n = min(BN, p.Lk_seg - j * BN);
+          const long long kbase = static_cast<long long>(s) * p.Lk_seg + j * BN;
+          int kp4[4], ks4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int idx = 4 * lane + e;
+            kp4[e] = idx < n ? (p.kv_pos ? __ldg(p.kv_pos + kbase + idx) : j * BN + idx) : INT_MAX;
+            ks4[e] = (p.seg && idx < n) ? __ldg(p.seg + kbase + idx) : INT_MAX;
+          }
           int klo = 0;
           if (p.seg) {
             int lo = 0, hi = n;
-            while (lo < hi) {
+#pragma unroll 1
+            for (int step = 0; step < 8; ++step) {
               const int mid = (lo + hi) >> 1;
-              if (segat(p, s, j * BN + mid) >= my_seg) hi = mid; else lo = mid + 1;
+              const int sg = warp_elem128(ks4, mid);
+              if (lo < hi) {
+                if (sg >= my_seg) hi = mid; else lo = mid + 1;
+              }
             }
             klo = (my_seg & 1) ? n : lo;
           }
           int lo = klo, hi = n;
-          while (lo < hi) {
+#pragma unroll 1
+          for (int step = 0; step < 8; ++step) {
             const int mid = (lo + hi) >> 1;
-            const long long kp = kpos(p, s, j * BN + mid);
-            const bool vis = kp < p.kv_valid && (!p.causal || kp <= my_pos) &&
-                             (!p.seg || segat(p, s, j * BN + mid) == my_seg);
-            if (vis) lo = mid + 1; else hi = mid;
+            const long long kp = warp_elem128(kp4, mid);
+            const int sg = p.seg ? warp_elem128(ks4, mid) : 0;
+            const bool vis = kp < p.kv_valid && (!p.causal || kp <= my_pos) && (!p.seg || sg == my_seg);
+            if (lo < hi) {
+              if (vis) lo = mid + 1; else hi = mid;
+            }
           }
           const int khi = lo;
 #pragma unroll

@@ -46,6 +46,19 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
                : "memory");
 }
 
+// Element idx (0..127) of a 128-entry array spread over a warp, four
+// consecutive entries per lane (lane l holds entries 4l..4l+3 in v[0..3]).
+// Every lane of the warp must call it (each may ask for a different idx).
+__device__ __forceinline__ int warp_elem128(const int (&v)[4], int idx) {
+  const int src = (idx >> 2) & 31;
+  const int a = __shfl_sync(0xffffffffu, v[0], src);
+  const int b = __shfl_sync(0xffffffffu, v[1], src);
+  const int c = __shfl_sync(0xffffffffu, v[2], src);
+  const int d = __shfl_sync(0xffffffffu, v[3], src);
+  const int e = idx & 3;
+  return e == 0 ? a : (e == 1 ? b : (e == 2 ? c : d));
+}
+
 // -------------------------------------------------------------- mbarrier ---
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
