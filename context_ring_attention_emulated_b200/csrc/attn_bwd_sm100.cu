@@ -133,7 +133,7 @@ __device__ __forceinline__ void transpose_reduce(uint32_t (&v)[32], float* dst, 
                  __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
 }
 
-template <int D>
+template <int D, bool SEG>  // SEG: packed sequences (segid array present)
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
@@ -153,7 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);       // per hop: visible query tiles [x, y)
+  // per hop: x = first visible query tile; y = end of the visible tiles for
+  // packed sequences, else the first tile with no masked element (the visible
+  // tiles then run to the last tile)
+  int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
   volatile int* s_full = reinterpret_cast<volatile int*>(smem + C::OFF_FULL);  // per Q/dO stage
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* s_delta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
@@ -205,8 +208,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // sequences) are non-decreasing in a segment, so both ends are found by
   // binary search; without packed sequences end_vis = nq_tiles.
   const bool live = k_min < p.kv_valid;
-  const int sk_lo = p.seg ? segat(p, s, k0) : 0;
-  const int sk_hi = p.seg ? segat(p, s, k0 + k_rows - 1) : 0;
+  const int sk_lo = SEG ? segat(p, s, k0) : 0;
+  const int sk_hi = SEG ? segat(p, s, k0 + k_rows - 1) : 0;
   for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
     const int r = (s + t) % p.nseg;
     int first_vis = p.nq_tiles, end_vis = p.nq_tiles;
@@ -215,18 +218,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (lo < hi) {  // first tile whose last query may see a key of this tile
         const int mid = (lo + hi) >> 1;
         const int last = min((mid + 1) * BQ, p.Lseg) - 1;
-        const bool reach = (!p.causal || posat(p, r, last) >= k_min) && (!p.seg || segat(p, r, last) >= sk_lo);
+        const bool reach = (!p.causal || posat(p, r, last) >= k_min) && (!SEG || segat(p, r, last) >= sk_lo);
         if (reach) hi = mid; else lo = mid + 1;
       }
       first_vis = lo;
-      if (p.seg) {
-        hi = p.nq_tiles;
+      hi = p.nq_tiles;
+      if (SEG) {
         while (lo < hi) {  // first tile wholly past the key tile's last segment
           const int mid = (lo + hi) >> 1;
           if (segat(p, r, mid * BQ) > sk_hi) hi = mid; else lo = mid + 1;
         }
-        end_vis = lo;
+      } else if (p.causal) {
+        while (lo < hi) {  // first tile whose first query sees every key
+          const int mid = (lo + hi) >> 1;
+          if (posat(p, r, mid * BQ) >= k_max) hi = mid; else lo = mid + 1;
+        }
+      } else {
+        lo = first_vis;  // non-causal: every visible tile is unmasked
       }
+      end_vis = lo;
     }
     s_hop[t] = make_int2(first_vis, end_vis);
   }
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   int NIT = 0;
-  for (int t = 0; t < p.nseg; ++t) NIT += s_hop[t].y - s_hop[t].x;
+  for (int t = 0; t < p.nseg; ++t) NIT += (SEG ? s_hop[t].y : p.nq_tiles) - s_hop[t].x;
   NIT *= p.group;  // the same tiles for every query head of the group
 
   int issued_q = 0;
@@ -262,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int bh = kvh * p.group + hq;  // (batch, query head)
       for (int t = 0; t < p.nseg && ok; ++t) {
         const int r = (s + t) % p.nseg;
-        for (int i = s_hop[t].x; i < s_hop[t].y; ++i, ++it) {
+        const int i_end = SEG ? s_hop[t].y : p.nq_tiles;
+        for (int i = s_hop[t].x; i < i_end; ++i, ++it) {
           const int st = it % C::NSQ;
           const uint32_t u = it / C::NSQ;
           if (u > 0 && !warp_wait(&bar_q_empty[st], (u - 1) & 1, s_abort, p.wait_ns)) {
@@ -286,12 +297,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (lane == 0) {
             // No element of this tile pair is masked when every query sees
-            // every key: all in one real sequence (packed) and, when causal,
-            // the first query at or after the last key.
-            const int qa = i * BQ, qb = min(qa + BQ, p.Lseg) - 1;
-            bool full = !p.causal || posat(p, r, qa) >= k_max;
-            if (p.seg)
-              full = full && sk_lo == sk_hi && (sk_lo & 1) == 0 && segat(p, r, qa) == sk_lo && segat(p, r, qb) == sk_lo;
+            // every key. Without packed sequences that is the tiles from the
+            // hop table's y on; packed, all in one real sequence and, when
+            // causal, the first query at or after the last key.
+            bool full = i >= s_hop[t].y;
+            if (SEG) {
+              const int qa = i * BQ, qb = min(qa + BQ, p.Lseg) - 1;
+              full = (!p.causal || posat(p, r, qa) >= k_max) && sk_lo == sk_hi && (sk_lo & 1) == 0 &&
+                     segat(p, r, qa) == sk_lo && segat(p, r, qb) == sk_lo;
+            }
             s_full[st] = full ? 1 : 0;
           }
           __syncwarp();
@@ -378,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = row < k_rows;
     const long long my_kpos = key_ok ? posat(p, s, k0 + row) : k_max;
-    const int my_seg = (p.seg && key_ok) ? segat(p, s, k0 + row) : 0;
+    const int my_seg = (SEG && key_ok) ? segat(p, s, k0 + row) : 0;
     const bool key_dead = !key_ok || my_kpos >= p.kv_valid || (my_seg & 1);  // odd segid: padding
     const float sl2 = p.scale_log2;
     const int qc0 = wg * 64;              // first query column of this warpgroup
@@ -391,22 +405,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < p.nseg && ok; ++t) {
       const int r = (s + t) % p.nseg;
       const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
-      for (int i = s_hop[t].x; i < s_hop[t].y; ++i, ++it) {
+      const int i_end = SEG ? s_hop[t].y : p.nq_tiles;
+      for (int i = s_hop[t].x; i < i_end; ++i, ++it) {
         const int st = it % C::NSQ;
         const float* lse2 = s_lse + st * 128 + qc0;
         const float* dlt = s_delta + st * 128 + qc0;
-        if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns) ||
-            !warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
-          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // query columns of this tile that see this key: [first, last). The
-        // tile's query positions and segids are spread over the warp (four
-        // per lane) and searched through shuffles (all lanes, eight steps).
+        // Query columns of this tile that see this key: [first, last).
+        // Without packed sequences the hop table says which tiles need a
+        // search, which then runs per thread before the wait for the tile's
+        // scores; packed, the tile's query positions and segids are spread
+        // over the warp (four per lane) and searched through shuffles (all
+        // lanes, eight steps) once the tile's flag is known.
         int first = 0, last = BQ;
-        if (!s_full[st]) {  // the same for the whole warp
+        auto search = [&]() {
           const int n = min(BQ, p.Lseg - i * BQ);
           const long long qbase = static_cast<long long>(r) * p.Lseg + i * BQ;
           int qp4[4], qs4[4];
@@ -414,21 +425,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int idx = 4 * lane + e;
             qp4[e] = idx < n ? __ldg(p.pos + qbase + idx) : INT_MAX;
-            qs4[e] = (p.seg && idx < n) ? __ldg(p.seg + qbase + idx) : INT_MAX;
+            qs4[e] = (SEG && idx < n) ? __ldg(p.seg + qbase + idx) : INT_MAX;
           }
           int lo = 0, hi = n;
 #pragma unroll 1
           for (int step = 0; step < 8; ++step) {  // first query at or after this key (same sequence when packed)
             const int mid = (lo + hi) >> 1;
             const int qp = warp_elem128(qp4, mid);
-            const int qs = p.seg ? warp_elem128(qs4, mid) : 0;
-            const bool past = p.causal ? qp >= my_kpos : (!p.seg || qs >= my_seg);
+            const int qs = SEG ? warp_elem128(qs4, mid) : 0;
+            const bool past = p.causal ? qp >= my_kpos : (!SEG || qs >= my_seg);
             if (lo < hi) {
               if (past) hi = mid; else lo = mid + 1;
             }
           }
           first = lo;
-          if (p.seg) {
+          if (SEG) {
             hi = n;
 #pragma unroll 1
             for (int step = 0; step < 8; ++step) {  // first query of a later sequence
@@ -440,7 +451,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             last = lo;
           }
+        };
+        if (!SEG && !key_dead && i < s_hop[t].y) {
+          // first query column at or after this key (the visible suffix)
+          int lo = 0, hi = min(BQ, p.Lseg - i * BQ);
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (posat(p, r, i * BQ + mid) >= my_kpos) hi = mid; else lo = mid + 1;
+          }
+          first = lo;
         }
+        if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns) ||
+            !warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
+          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (SEG && !s_full[st]) search();  // the same for the whole warp
         if (key_dead) first = BQ;
         first -= qc0;  // relative to this warpgroup's columns
         last -= qc0;
@@ -456,8 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c0 = 2 * e;
             float a = ex2_approx(fmaf(__uint_as_float(sr[c0 >> 5][c0 & 31]), sl2, -lse2[c0]));
             float b = ex2_approx(fmaf(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), sl2, -lse2[c0 + 1]));
-            a = (c0 >= first && c0 < last) ? a : 0.f;
-            b = (c0 + 1 >= first && c0 + 1 < last) ? b : 0.f;
+            if (SEG) {  // visible run [first, last)
+              a = (c0 >= first && c0 < last) ? a : 0.f;
+              b = (c0 + 1 >= first && c0 + 1 < last) ? b : 0.f;
+            } else {      // visible suffix from first
+              a = c0 >= first ? a : 0.f;
+              b = c0 + 1 >= first ? b : 0.f;
+            }
             sr[c0 >> 5][c0 & 31] = __float_as_uint(a);
             sr[(c0 + 1) >> 5][(c0 + 1) & 31] = __float_as_uint(b);
             pk[e] = pack_bf16x2(a, b);
@@ -660,7 +693,9 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
-  if ((st = set_smem_attr(reinterpret_cast<const void*>(&bwd_kernel<D>), C::SMEM)) != RATTN_OK) return st;
+  const void* kfn = a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true>)
+                         : reinterpret_cast<const void*>(&bwd_kernel<D, false>);
+  if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
   Params p;
   p.lse = a.lse;
   p.delta = a.delta;
@@ -681,7 +716,10 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.dv = a.dv;
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
-  bwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+  if (a.seg)
+    bwd_kernel<D, true><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+  else
+    bwd_kernel<D, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   const long long n4 = rows * D / 4;
   dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),

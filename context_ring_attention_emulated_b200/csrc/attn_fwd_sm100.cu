@@ -104,7 +104,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
 }
 
-template <int D>
+template <int D, bool SEG>  // SEG: packed sequences (segid array present)
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -178,10 +178,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // visible tiles are a prefix.
   for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
     const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-    const int sq_lo = p.seg ? segat(p, r, q0) : 0;
-    const int sq_hi = p.seg ? segat(p, r, q0 + q_rows - 1) : 0;
+    const int sq_lo = SEG ? segat(p, r, q0) : 0;
+    const int sq_hi = SEG ? segat(p, r, q0 + q_rows - 1) : 0;
     int first = 0;
-    if (p.seg) {  // first tile whose last key is in the query tile's first segment or later
+    if (SEG) {  // first tile whose last key is in the query tile's first segment or later
       int lo = 0, hi = nk_tiles;
       while (lo < hi) {
         const int mid = (lo + hi) >> 1;
@@ -193,15 +193,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
       const long long kmin = kpos(p, s, mid * BN);
-      const bool vis = kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!p.seg || segat(p, s, mid * BN) <= sq_hi);
+      const bool vis = kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!SEG || segat(p, s, mid * BN) <= sq_hi);
       if (vis) lo = mid + 1; else hi = mid;
     }
     const int n_vis = lo;
     int f_lo = first, f_hi = first;
-    const bool one_seg = !p.seg || (sq_lo == sq_hi && (sq_lo & 1) == 0);
+    const bool one_seg = !SEG || (sq_lo == sq_hi && (sq_lo & 1) == 0);
     if (one_seg && first < n_vis) {
       int a = first, b = n_vis;
-      if (p.seg) {  // tiles lying wholly in the query tile's segment: [a, b)
+      if (SEG) {  // tiles lying wholly in the query tile's segment: [a, b)
         lo = first;
         hi = n_vis;
         while (lo < hi) {
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool row_valid = row < q_rows;
     const long long my_pos = row_valid ? qpos(p, r, q0 + row) : q_max;
-    const int my_seg = (p.seg && row_valid) ? segat(p, r, q0 + row) : 1;  // odd: sees nothing
+    const int my_seg = (SEG && row_valid) ? segat(p, r, q0 + row) : 1;  // odd: sees nothing
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -379,10 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int idx = 4 * lane + e;
             kp4[e] = idx < n ? (p.kv_pos ? __ldg(p.kv_pos + kbase + idx) : j * BN + idx) : INT_MAX;
-            ks4[e] = (p.seg && idx < n) ? __ldg(p.seg + kbase + idx) : INT_MAX;
+            ks4[e] = (SEG && idx < n) ? __ldg(p.seg + kbase + idx) : INT_MAX;
           }
           int klo = 0;
-          if (p.seg) {
+          if (SEG) {
             int lo = 0, hi = n;
 #pragma unroll 1
             for (int step = 0; step < 8; ++step) {
@@ -399,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int step = 0; step < 8; ++step) {
             const int mid = (lo + hi) >> 1;
             const long long kp = warp_elem128(kp4, mid);
-            const int sg = p.seg ? warp_elem128(ks4, mid) : 0;
-            const bool vis = kp < p.kv_valid && (!p.causal || kp <= my_pos) && (!p.seg || sg == my_seg);
+            const int sg = SEG ? warp_elem128(ks4, mid) : 0;
+            const bool vis = kp < p.kv_valid && (!p.causal || kp <= my_pos) && (!SEG || sg == my_seg);
             if (lo < hi) {
               if (vis) lo = mid + 1; else hi = mid;
             }
@@ -564,7 +564,9 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
   if (a.group < 1 || a.BH % a.group) return RATTN_ERR_INVALID_ARG;
   if ((st = make_tmap_bf16(&tk, a.k, D, a.Lk_seg, a.nseg, a.BH / a.group, BN)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lk_seg, a.nseg, a.BH / a.group, BN)) != RATTN_OK) return st;
-  if ((st = set_smem_attr(reinterpret_cast<const void*>(&fwd_kernel<D>), C::SMEM)) != RATTN_OK) return st;
+  const void* kfn = a.seg ? reinterpret_cast<const void*>(&fwd_kernel<D, true>)
+                         : reinterpret_cast<const void*>(&fwd_kernel<D, false>);
+  if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
   Params p;
   p.q_pos = a.q_pos;
   p.kv_pos = a.kv_pos;
@@ -583,7 +585,10 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
   p.lse = a.lse;
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
-  fwd_kernel<D><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, p);
+  if (a.seg)
+    fwd_kernel<D, true><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, p);
+  else
+    fwd_kernel<D, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
