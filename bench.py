@@ -37,7 +37,7 @@ ROPE_BASE = 10000.0  # rotary base of the RoPE workloads (RoFormer's value)
 # launch by sequence length (traffic grows with the tensors). Source:
 # profiles/bwd_kernel_bf16_H32_L16000_cp4.md. Set to None when the kernel
 # changes until it is captured again.
-NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": (792.5e6 + 479.2e6) * 2}
+NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": (792.6e6 + 480.4e6) * 2}
 
 
 def peaks():
