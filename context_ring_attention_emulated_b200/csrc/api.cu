@@ -61,6 +61,9 @@ int64_t chunks_of(int cp, rattn_layout layout) {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Kernels index (batch, head) pairs with 32-bit integers.
+bool bh_fits(int B, int H) { return static_cast<int64_t>(B) * H <= INT32_MAX; }
+
 }  // namespace
 
 rattn_status get_dev_ctx(DevCtx* out) {
@@ -138,7 +141,7 @@ rattn_status cp_layout_permute(const void* x, void* y, int32_t* pos, int B, int 
   if (!es || B < 1 || H < 1 || D < 1 || L < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1)
     return RATTN_ERR_INVALID_ARG;
   if (Lp != cp_layout_padded_len(L, cp_size, layout)) return RATTN_ERR_INVALID_ARG;
-  if (Lp > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if (Lp > INT32_MAX || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
   if ((static_cast<int64_t>(D) * es) % 16) return RATTN_ERR_UNSUPPORTED;
   if (Lp == 0) return RATTN_OK;
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16) || (pos && !aligned(pos, 4))) return RATTN_ERR_INVALID_ARG;
@@ -151,7 +154,7 @@ rattn_status cp_layout_unpermute(const void* y, void* x, int B, int H, int64_t L
   if (!es || B < 1 || H < 1 || D < 1 || L < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1)
     return RATTN_ERR_INVALID_ARG;
   if (Lp != cp_layout_padded_len(L, cp_size, layout)) return RATTN_ERR_INVALID_ARG;
-  if (Lp > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if (Lp > INT32_MAX || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
   if ((static_cast<int64_t>(D) * es) % 16) return RATTN_ERR_UNSUPPORTED;
   if (L == 0) return RATTN_OK;
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return RATTN_ERR_INVALID_ARG;
@@ -200,7 +203,7 @@ static rattn_status check_gather(const void* a, const void* b, const int32_t* sr
                                  int64_t Tb, int D, rattn_dtype dtype) {
   const int es = elem_size(dtype);
   if (!es || B < 1 || H < 1 || D < 1 || Ta < 0 || Tb < 0) return RATTN_ERR_INVALID_ARG;
-  if (Ta > INT32_MAX || Tb > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if (Ta > INT32_MAX || Tb > INT32_MAX || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(D) * es;
   if (row % 16 || row > 4096) return RATTN_ERR_UNSUPPORTED;
   return RATTN_OK;
@@ -232,7 +235,7 @@ static rattn_status check_rope(int B, int H, int64_t L, int64_t Lp, int D, rattn
   if (!(base > 0.0 && base < INFINITY)) return RATTN_ERR_INVALID_ARG;
   if (style != RATTN_ROPE_HALF && style != RATTN_ROPE_INTERLEAVED) return RATTN_ERR_INVALID_ARG;
   if (Lp != cp_layout_padded_len(L, cp_size, layout)) return RATTN_ERR_INVALID_ARG;
-  if (Lp > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if (Lp > INT32_MAX || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
   const int64_t row = static_cast<int64_t>(D) * es;
   if (D % 2 || row % 16 || row > 4096) return RATTN_ERR_UNSUPPORTED;
   if (style == RATTN_ROPE_HALF && (row / 2) % 16) return RATTN_ERR_UNSUPPORTED;
@@ -269,7 +272,7 @@ rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v, cons
     return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_attn_d(D, dtype);
   if (st != RATTN_OK) return st;
-  if (Lq > INT32_MAX - 256 || Lk > INT32_MAX - 256) return RATTN_ERR_UNSUPPORTED;
+  if (Lq > INT32_MAX - 256 || Lk > INT32_MAX - 256 || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
   if (Lq == 0) return RATTN_OK;
   if (!q || !o || !lse || !aligned(q, 16) || !aligned(o, 16) || !aligned(lse, 4)) return RATTN_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return RATTN_ERR_INVALID_ARG;
@@ -321,7 +324,7 @@ static rattn_status check_ring(const void* q, const void* k, const void* v, cons
   if (n < 1 || Lp % n) return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_attn_d(D, dtype);
   if (st != RATTN_OK) return st;
-  if (cp_size > 64) return RATTN_ERR_UNSUPPORTED;
+  if (cp_size > 64 || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
   if (Lp > INT32_MAX - 256) return RATTN_ERR_UNSUPPORTED;
   if (Lp == 0) return RATTN_OK;
   if (!q || !k || !v || !pos || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(pos, 4))

@@ -25,6 +25,8 @@
  *     the caller. The library never allocates device memory; scratch space is
  *     passed in by the caller (rattn_ring_bwd's workspace).
  *   - Data pointers must be 16-byte aligned. Position arrays are int32.
+ *     B * H must fit in 32 bits and sequence lengths in 31 bits (larger
+ *     requests return RATTN_ERR_UNSUPPORTED).
  *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream). Arguments are validated on the host first;
  *     a violation returns RATTN_ERR_INVALID_ARG or RATTN_ERR_UNSUPPORTED and

@@ -212,3 +212,13 @@ def test_varlen_calls_reject_bad_arguments(rattn):
     fv = L.rattn_ring_fwd_varlen(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 255, 64, 1, 2, 1, ctypes.c_float(0.125),
                                  FAKE, FAKE, None)
     assert fv == rattn.ERR_INVALID_ARG            # Tp not a multiple of cp
+
+
+def test_batch_times_heads_beyond_int32_is_unsupported(rattn):
+    L = rattn.lib
+    big = 1 << 16
+    assert L.cp_layout_permute(FAKE, FAKE, FAKE, big, big, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_UNSUPPORTED
+    assert L.cp_layout_unpermute(FAKE, FAKE, big, big, 16, 16, 64, 1, 4, 1, None) == rattn.ERR_UNSUPPORTED
+    assert L.cp_layout_gather(FAKE, FAKE, FAKE, big, big, 16, 16, 64, 1, None) == rattn.ERR_UNSUPPORTED
+    assert L.rattn_ring_fwd(FAKE, FAKE, FAKE, FAKE, big, big, 256, 64, 1, 2, 1, 1, ctypes.c_float(0.125), 256,
+                            FAKE, FAKE, None) == rattn.ERR_UNSUPPORTED
