@@ -26,6 +26,12 @@
 // TMEM columns: A [0,128) S^T; warpgroup g then overwrites its own columns
 // [64g, 64g+64) with P^T (bf16, [64g, 64g+32)) and dS^T ([64g+32, 64g+64));
 // B [128,256) dP^T, then dQ; dV [256,256+D); dK [256+D,256+2D).
+//
+// Grouped key/value heads: the CTA of a K/V tile walks the query tiles of
+// every query head of its group, so dK/dV sum over the group in TMEM. Packed
+// sequences (the SEG instantiation): a key is visible only to queries with
+// the same even segid; the producer flags per query tile whether any element
+// needs masking.
 #include <limits.h>
 #include <math.h>
 

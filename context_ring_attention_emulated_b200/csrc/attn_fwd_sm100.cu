@@ -28,6 +28,12 @@
 // written over the first 64 columns of its own score buffer. The MMA that
 // next overwrites that buffer (S_{g+3}) is issued only after the PV MMA
 // reading P_g has completed.
+//
+// Grouped key/value heads: query head h reads the K/V of head h / group.
+// Packed sequences (the SEG instantiation; ring calls use the other one): a
+// key is visible only to queries carrying the same even segid, so the visible
+// tiles of a hop form a range rather than a prefix, and masked rows keep a
+// contiguous run of keys.
 #include <limits.h>
 #include <math.h>
 
