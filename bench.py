@@ -54,6 +54,16 @@ def step_flops(w):
     return fwd * (3.5 if w.bwd else 1.0), fwd
 
 
+def physical_gpu(local):
+    """nvidia-smi index of this process's CUDA device ``local``: the entry of
+    CUDA_VISIBLE_DEVICES it maps to, when that variable lists plain indices."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    if ids and local < len(ids) and ids[local].isdigit():
+        return int(ids[local])
+    return local
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -61,7 +71,7 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
-        self.index = index
+        self.index = physical_gpu(index)
         self.proc = None
 
     def __enter__(self):
@@ -119,7 +129,10 @@ def dist_setup(n):
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
-        dist.barrier()
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
 
 
 def max_over_ranks(x, world, device="cuda"):

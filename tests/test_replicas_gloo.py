@@ -22,6 +22,7 @@ def _rank(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         local_ms = [120.0, 150.0][rank]
+        bench.barrier(world)                              # the bench's barrier on a non-NCCL group
         ms = bench.max_over_ranks(local_ms, world, device="cpu")
         out[rank] = (ms, bench.aggregate_tflops(1e12, 10, world, ms))
     finally:
@@ -43,3 +44,13 @@ def test_two_replicas_agree_on_max_time_and_aggregate():
 def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(7.5, 1) == 7.5
     assert bench.dist_setup(1) == (0, 1, 0) or "RANK" in os.environ
+
+
+def test_physical_gpu_index_follows_visible_devices(monkeypatch):
+    import bench
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "4,5,6,7")
+    assert bench.physical_gpu(0) == 4 and bench.physical_gpu(3) == 7
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "")
+    assert bench.physical_gpu(2) == 2
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-1234abcd")
+    assert bench.physical_gpu(0) == 0
