@@ -31,12 +31,13 @@ rank/chunk table). No function is "parity unpinned".
 from .layout import (CONTIGUOUS, HEAD_TAIL, STRIPED, padded_len, perm_index, permute, unpermute, rank_chunks,
                      varlen_index, varlen_permute, varlen_unpermute)
 from .attn import (attention, merge, ring_emulate, blockwise_attention,
-                        attention_bwd, visible_mask, causal_pairs_per_rank, gqa_expand, gqa_reduce)
+                        attention_bwd, attention_bwd_block, visible_mask, causal_pairs_per_rank, gqa_expand,
+                   gqa_reduce)
 from .rotary import HALF as ROPE_HALF, INTERLEAVED as ROPE_INTERLEAVED, rope, rope_grad
 
 __all__ = [
     "CONTIGUOUS", "HEAD_TAIL", "STRIPED", "padded_len", "perm_index", "permute", "unpermute", "rank_chunks",
     "varlen_index", "varlen_permute", "varlen_unpermute",
-    "attention", "merge", "ring_emulate", "blockwise_attention", "attention_bwd", "visible_mask",
+    "attention", "merge", "ring_emulate", "blockwise_attention", "attention_bwd", "attention_bwd_block", "visible_mask",
     "causal_pairs_per_rank", "gqa_expand", "gqa_reduce", "ROPE_HALF", "ROPE_INTERLEAVED", "rope", "rope_grad",
 ]

@@ -204,6 +204,38 @@ def attention_bwd(q, k, v, do, scale, causal, q_pos=None, kv_pos=None, kv_valid=
     return dq.reshape(q.shape), dk.reshape(k.shape), dv.reshape(v.shape)
 
 
+def attention_bwd_block(q, k, v, do, lse, delta, scale, causal, q_pos=None, kv_pos=None, kv_valid=None):
+    """One key block's share of the attention gradient, float64: what a rank
+    computes at one hop of the ring backward, where the softmax of a query row
+    spans every block but only this one is at hand. The row's final LSE and
+    delta_i = sum_d dO_id O_id (O the final output) stand in for the rest:
+      P_ij = exp(scale q_i.k_j - LSE_i) on visible pairs, 0 elsewhere,
+      dV = P^T dO, dP = dO V^T, dS_ij = P_ij (dP_ij - delta_i),
+      dQ = scale dS K (this block's part), dK = scale dS^T Q, dV as above.
+    Since sum_j P_ij dP_ij = sum_d dO_id O_id, the shares summed over a
+    partition of the keys are ``attention_bwd``. lse [..., Lq], delta
+    [..., Lq]; returns dq [..., Lq, D], dk, dv [..., Lk, D]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
+    delta = np.asarray(delta, dtype=np.float64)
+    Lq, Lk = q.shape[-2], k.shape[-2]
+    q_pos = _default_pos(Lq) if q_pos is None else np.asarray(q_pos, dtype=np.int64)
+    kv_pos = _default_pos(Lk) if kv_pos is None else np.asarray(kv_pos, dtype=np.int64)
+    mask = visible_mask(q_pos, kv_pos, causal, kv_valid)
+    s = scale * np.einsum("...id,...jd->...ij", q, k)
+    with np.errstate(over="ignore", invalid="ignore"):
+        p = np.where(mask, np.exp(s - lse[..., :, None]), 0.0)
+    dv = np.einsum("...ij,...id->...jd", p, do)
+    dp = np.einsum("...id,...jd->...ij", do, v)
+    ds = p * (dp - delta[..., :, None])
+    dq = scale * np.einsum("...ij,...jd->...id", ds, k)
+    dk = scale * np.einsum("...ij,...id->...jd", ds, q)
+    return dq, dk, dv
+
+
 def causal_pairs_per_rank(L, cp, layout):
     """Brute-force count of visible causal (query, key) pairs per rank.
 

@@ -304,3 +304,97 @@ def test_empty_key_block_sees_nothing():
     assert o.shape == (2, 3, 4, 5) and np.all(o == 0.0) and np.all(np.isneginf(lse))
     dq, dk, dv = oracle.attention_bwd(q, k, k, q, 0.5, True)
     assert np.all(dq == 0.0) and dk.shape == k.shape and dv.shape == k.shape
+
+
+# ---- one hop of the ring backward -------------------------------------------
+
+def _block_bwd_case(seed, causal, kv_valid):
+    """Random rows with shuffled (not monotone) positions, the final O / LSE of
+    the whole key set, and a random split of the keys into blocks."""
+    r = np.random.default_rng(seed)
+    B, H, Lq, Lk, D = 2, 2, 11, 13, 4
+    q, do = r.standard_normal((B, H, Lq, D)), r.standard_normal((B, H, Lq, D))
+    k, v = r.standard_normal((B, H, Lk, D)), r.standard_normal((B, H, Lk, D))
+    q_pos = r.permutation(Lq) + 3
+    kv_pos = r.permutation(Lk)
+    cuts = np.sort(r.choice(np.arange(1, Lk), size=3, replace=False))
+    perm = r.permutation(Lk)
+    blocks = [np.sort(b) for b in np.split(perm, cuts)]
+    o, lse = oracle.attention(q, k, v, 0.45, causal, q_pos, kv_pos, kv_valid, row_block=4)
+    delta = (do * o).sum(-1)
+    return q, k, v, do, lse, delta, q_pos, kv_pos, blocks
+
+
+def _sum_of_block_shares(case, causal, kv_valid, block_fn=None):
+    q, k, v, do, lse, delta, q_pos, kv_pos, blocks = case
+    fn = block_fn or oracle.attention_bwd_block
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for idx in blocks:
+        gq, gk, gv = fn(q, k[..., idx, :], v[..., idx, :], do, lse, delta, 0.45, causal, q_pos, kv_pos[idx],
+                        kv_valid)
+        dq += gq
+        dk[..., idx, :] = gk
+        dv[..., idx, :] = gv
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("causal,kv_valid", [(True, None), (False, None), (True, 9), (False, 7)])
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_block_bwd_shares_sum_to_the_gradient(causal, kv_valid, seed):
+    """Summed over any split of the keys (and keys of each block written back
+    in place), the per-block shares are the full gradient (pinned above by
+    finite differences and torch autograd): sum_j P_ij dP_ij = delta_i."""
+    case = _block_bwd_case(seed, causal, kv_valid)
+    q, k, v, do, lse, delta, q_pos, kv_pos, _ = case
+    ref = oracle.attention_bwd(q, k, v, do, 0.45, causal, q_pos, kv_pos, kv_valid, row_block=4)
+    for got, want in zip(_sum_of_block_shares(case, causal, kv_valid), ref):
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_block_bwd_single_block_matches_finite_differences():
+    r = np.random.default_rng(5)
+    q, k, v, do = (r.standard_normal((6, 3)) for _ in range(4))
+    pos = np.arange(6)
+    o, lse = oracle.attention(q, k, v, 0.6, True, pos, pos)
+    got = oracle.attention_bwd_block(q, k, v, do, lse, (do * o).sum(-1), 0.6, True, pos, pos)
+    for g, ref in zip(got, _fd_grads(q, k, v, do, 0.6, True, pos, pos)):
+        np.testing.assert_allclose(g, ref, rtol=1e-7, atol=1e-8)
+
+
+def test_block_bwd_block_without_visible_keys_is_zero():
+    """A block that lies wholly in the future of every query adds nothing."""
+    r = np.random.default_rng(6)
+    q, do = r.standard_normal((1, 4, 2)), r.standard_normal((1, 4, 2))
+    k, v = r.standard_normal((1, 3, 2)), r.standard_normal((1, 3, 2))
+    lse = r.standard_normal((1, 4))
+    dq, dk, dv = oracle.attention_bwd_block(q, k, v, do, lse, r.standard_normal((1, 4)), 0.5, True,
+                                            np.arange(4), np.arange(10, 13))
+    assert not dq.any() and not dk.any() and not dv.any()
+
+
+def _delta_dropped(q, k, v, do, lse, delta, *a):
+    return oracle.attention_bwd_block(q, k, v, do, lse, np.zeros_like(delta), *a)
+
+
+def _lse_base2(q, k, v, do, lse, delta, *a):
+    return oracle.attention_bwd_block(q, k, v, do, lse / math.log(2.0), delta, *a)
+
+
+def _v_for_k(q, k, v, do, lse, delta, *a):
+    return oracle.attention_bwd_block(q, v, v, do, lse, delta, *a)
+
+
+def _scale_squared(q, k, v, do, lse, delta, scale, *a):
+    dq, dk, dv = oracle.attention_bwd_block(q, k, v, do, lse, delta, scale, *a)
+    return scale * dq, scale * dk, dv
+
+
+@pytest.mark.parametrize("mutant", [_delta_dropped, _lse_base2, _v_for_k, _scale_squared])
+def test_block_bwd_pin_rejects_planted_mistakes(mutant):
+    case = _block_bwd_case(11, True, None)
+    q, k, v, do, lse, delta, q_pos, kv_pos, _ = case
+    ref = oracle.attention_bwd(q, k, v, do, 0.45, True, q_pos, kv_pos, row_block=4)
+    got = _sum_of_block_shares(case, True, None, block_fn=mutant)
+    assert not all(np.allclose(g, w, atol=1e-12) for g, w in zip(got, ref))
