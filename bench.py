@@ -10,8 +10,8 @@ D=128, bf16, causal). Metric: causal-adjusted TFLOP/s of fwd + bwd
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 Under torchrun (N > 1) every rank runs an independent replica of the
-workload (the path has no cross-GPU exchange in this build); value is the
-work of all ranks over the max-over-ranks device time.
+workload (each emulates all CP ranks on its own GPU, so no data crosses
+GPUs); value is the work of all ranks over the max-over-ranks device time.
 """
 import argparse
 import json

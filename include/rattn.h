@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
   RATTN_OK = 0,
   RATTN_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or enum       */
-  RATTN_ERR_UNSUPPORTED = 2,   /* valid request this build does not handle   */
+  RATTN_ERR_UNSUPPORTED = 2,   /* valid request the library does not handle  */
   RATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
   RATTN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up         */
 } rattn_status;
