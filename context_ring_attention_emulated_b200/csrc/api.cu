@@ -473,6 +473,74 @@ rattn_status rattn_ring_bwd_varlen(const void* q, const void* k, const void* v, 
                        stream);
 }
 
+rattn_status rattn_bwd_prep(const void* o, const void* dout, int B, int H, int64_t L, int D, rattn_dtype dtype,
+                            float* delta, float* dq_acc, void* stream) {
+  if (B < 1 || H < 1 || L < 0) return RATTN_ERR_INVALID_ARG;
+  rattn_status st = check_attn_d(D, dtype);
+  if (st != RATTN_OK) return st;
+  if (dtype != RATTN_BF16 || !bh_fits(B, H) || L > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if (L == 0) return RATTN_OK;
+  if (!o || !dout || !delta || !aligned(o, 16) || !aligned(dout, 16) || !aligned(delta, 4) ||
+      (dq_acc && !aligned(dq_acc, 16)))
+    return RATTN_ERR_INVALID_ARG;
+  return launch_bwd_prep_sm100(o, dout, static_cast<long long>(B) * H * L, D, delta, dq_acc,
+                               static_cast<cudaStream_t>(stream));
+}
+
+rattn_status rattn_partial_bwd(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                               const float* delta, const int32_t* q_pos, const int32_t* kv_pos, int B, int H,
+                               int H_kv, int64_t Lq, int64_t Lk, int D, rattn_dtype dtype, float scale, int causal,
+                               int64_t kv_valid, float* dq_acc, float* dk, float* dv, int accumulate,
+                               void* stream) {
+  if (B < 1 || H < 1 || H_kv < 1 || H % H_kv || Lq < 0 || Lk < 0 || (causal != 0 && causal != 1) ||
+      (accumulate != 0 && accumulate != 1) || !(scale > 0.f && scale < INFINITY))
+    return RATTN_ERR_INVALID_ARG;
+  rattn_status st = check_attn_d(D, dtype);
+  if (st != RATTN_OK) return st;
+  if (dtype != RATTN_BF16) return RATTN_ERR_UNSUPPORTED;
+  if (Lq > INT32_MAX - 256 || Lk > INT32_MAX - 256 || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
+  if (Lk == 0) return RATTN_OK;
+  if (!k || !v || !kv_pos || !dk || !dv || !aligned(k, 16) || !aligned(v, 16) || !aligned(kv_pos, 4) ||
+      !aligned(dk, 16) || !aligned(dv, 16))
+    return RATTN_ERR_INVALID_ARG;
+  if (Lq > 0 && (!q || !dout || !lse || !delta || !q_pos || !dq_acc || !aligned(q, 16) || !aligned(dout, 16) ||
+                 !aligned(lse, 4) || !aligned(delta, 4) || !aligned(q_pos, 4) || !aligned(dq_acc, 16)))
+    return RATTN_ERR_INVALID_ARG;
+  PartialBwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.lse = lse;
+  a.delta = delta;
+  a.q_pos = q_pos;
+  a.kv_pos = kv_pos;
+  a.BH = B * H;
+  a.group = H / H_kv;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.D = D;
+  a.dtype = dtype;
+  a.scale = scale;
+  a.causal = causal;
+  a.kv_valid = kv_valid;
+  a.dq_acc = dq_acc;
+  a.dk = dk;
+  a.dv = dv;
+  a.accumulate = accumulate;
+  a.stream = static_cast<cudaStream_t>(stream);
+  DevCtx ctx;
+  if ((st = get_dev_ctx(&ctx)) != RATTN_OK) return st;
+  return launch_partial_bwd_sm100(a, ctx);
+}
+
+rattn_status rattn_grad_fold(float* acc, const float* blk, int64_t n, void* stream) {
+  if (n < 0 || n % 4) return RATTN_ERR_INVALID_ARG;
+  if (n == 0) return RATTN_OK;
+  if (!acc || !blk || !aligned(acc, 16) || !aligned(blk, 16)) return RATTN_ERR_INVALID_ARG;
+  return launch_grad_fold(acc, blk, n, static_cast<cudaStream_t>(stream));
+}
+
 rattn_status rattn_get_device_error(int* site) {
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_err_word, sizeof(int)) != cudaSuccess) return RATTN_ERR_CUDA;

@@ -32,6 +32,13 @@
 // sequences (the SEG instantiation): a key is visible only to queries with
 // the same even segid; the producer flags per query tile whether any element
 // needs masking.
+//
+// One hop across processes (the SPLIT instantiation, rattn_partial_bwd): the
+// query rows belong to one rank and the key rows to another, so each side
+// has its own length and position array; a single segment, no preparation
+// pass (the caller hands in Delta and owns the fp32 dQ accumulator, which
+// receives scale * dS K directly), and dK, dV leave as fp32 shares that are
+// written or added to the caller's buffers.
 #include <limits.h>
 #include <math.h>
 
@@ -84,6 +91,11 @@ struct Params {
   void* dv;
   int* err;
   unsigned long long wait_ns;
+  // SPLIT only
+  const int32_t* q_pos;   // query positions [Lq]
+  const int32_t* kv_pos;  // key positions [Lk]
+  int Lq, Lk;             // query and key rows (the ring uses Lseg for both)
+  int accumulate;         // 1 adds the dK, dV shares to the outputs, 0 writes them
 };
 
 __device__ __forceinline__ int segat(const Params& p, int rank, int row) {
@@ -92,6 +104,30 @@ __device__ __forceinline__ int segat(const Params& p, int rank, int row) {
 
 __device__ __forceinline__ long long posat(const Params& p, int seg, int row) {
   return static_cast<long long>(__ldg(p.pos + static_cast<long long>(seg) * p.Lseg + row));
+}
+
+// Query-side and key-side lengths and positions: one array of Lseg rows per
+// segment for the ring, separate arrays for a SPLIT hop.
+template <bool SPLIT>
+__device__ __forceinline__ int q_len(const Params& p) {
+  return SPLIT ? p.Lq : p.Lseg;
+}
+
+template <bool SPLIT>
+__device__ __forceinline__ int k_len(const Params& p) {
+  return SPLIT ? p.Lk : p.Lseg;
+}
+
+template <bool SPLIT>
+__device__ __forceinline__ long long qposat(const Params& p, int seg, int row) {
+  if constexpr (SPLIT) return static_cast<long long>(__ldg(p.q_pos + static_cast<long long>(seg) * p.Lq + row));
+  else return posat(p, seg, row);
+}
+
+template <bool SPLIT>
+__device__ __forceinline__ long long kposat(const Params& p, int seg, int row) {
+  if constexpr (SPLIT) return static_cast<long long>(__ldg(p.kv_pos + static_cast<long long>(seg) * p.Lk + row));
+  else return posat(p, seg, row);
 }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -139,7 +175,7 @@ __device__ __forceinline__ void transpose_reduce(uint32_t (&v)[32], float* dst, 
                  __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
 }
 
-template <int D, bool SEG>  // SEG: packed sequences (segid array present)
+template <int D, bool SEG, bool SPLIT>  // SEG: packed sequences; SPLIT: one hop across processes
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
@@ -184,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt = item % p.nk_tiles;
   const int kvh = item / p.nk_tiles;  // (batch, key/value head); its query heads are kvh * group + j
   const int k0 = kt * BK;
-  const int k_rows = min(BK, p.Lseg - k0);
-  const long long k_min = posat(p, s, k0);
-  const long long k_max = posat(p, s, k0 + k_rows - 1);
+  const int k_rows = min(BK, k_len<SPLIT>(p) - k0);
+  const long long k_min = kposat<SPLIT>(p, s, k0);
+  const long long k_max = kposat<SPLIT>(p, s, k0 + k_rows - 1);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
@@ -223,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int lo = 0, hi = p.nq_tiles;
       while (lo < hi) {  // first tile whose last query may see a key of this tile
         const int mid = (lo + hi) >> 1;
-        const int last = min((mid + 1) * BQ, p.Lseg) - 1;
-        const bool reach = (!p.causal || posat(p, r, last) >= k_min) && (!SEG || segat(p, r, last) >= sk_lo);
+        const int last = min((mid + 1) * BQ, q_len<SPLIT>(p)) - 1;
+        const bool reach = (!p.causal || qposat<SPLIT>(p, r, last) >= k_min) && (!SEG || segat(p, r, last) >= sk_lo);
         if (reach) hi = mid; else lo = mid + 1;
       }
       first_vis = lo;
@@ -237,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (p.causal) {
         while (lo < hi) {  // first tile whose first query sees every key
           const int mid = (lo + hi) >> 1;
-          if (posat(p, r, mid * BQ) >= k_max) hi = mid; else lo = mid + 1;
+          if (qposat<SPLIT>(p, r, mid * BQ) >= k_max) hi = mid; else lo = mid + 1;
         }
       } else {
         lo = first_vis;  // non-causal: every visible tile is unmasked
@@ -287,13 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
+          const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * q_len<SPLIT>(p);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = lane * 4 + e;
             const int q = i * BQ + c;
             float l2 = INFINITY, dl = 0.f;
-            if (q < p.Lseg) {
+            if (q < q_len<SPLIT>(p)) {
               const float l = __ldg(p.lse + rowbase + q);
               l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
               dl = __ldg(p.delta + rowbase + q);
@@ -308,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // causal, the first query at or after the last key.
             bool full = i >= s_hop[t].y;
             if (SEG) {
-              const int qa = i * BQ, qb = min(qa + BQ, p.Lseg) - 1;
-              full = (!p.causal || posat(p, r, qa) >= k_max) && sk_lo == sk_hi && (sk_lo & 1) == 0 &&
+              const int qa = i * BQ, qb = min(qa + BQ, q_len<SPLIT>(p)) - 1;
+              full = (!p.causal || qposat<SPLIT>(p, r, qa) >= k_max) && sk_lo == sk_hi && (sk_lo & 1) == 0 &&
                      segat(p, r, qa) == sk_lo && segat(p, r, qb) == sk_lo;
             }
             s_full[st] = full ? 1 : 0;
@@ -397,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;  // key row for S^T/dP^T/dK/dV, query row for dQ
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = row < k_rows;
-    const long long my_kpos = key_ok ? posat(p, s, k0 + row) : k_max;
+    const long long my_kpos = key_ok ? kposat<SPLIT>(p, s, k0 + row) : k_max;
     const int my_seg = (SEG && key_ok) ? segat(p, s, k0 + row) : 0;
     const bool key_dead = !key_ok || my_kpos >= p.kv_valid || (my_seg & 1);  // odd segid: padding
     const float sl2 = p.scale_log2;
@@ -410,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bh = kvh * p.group + hq;  // (batch, query head)
     for (int t = 0; t < p.nseg && ok; ++t) {
       const int r = (s + t) % p.nseg;
-      const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * p.Lseg;
+      const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * q_len<SPLIT>(p);
       const int i_end = SEG ? s_hop[t].y : p.nq_tiles;
       for (int i = s_hop[t].x; i < i_end; ++i, ++it) {
         const int st = it % C::NSQ;
@@ -424,13 +460,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lanes, eight steps) once the tile's flag is known.
         int first = 0, last = BQ;
         auto search = [&]() {
-          const int n = min(BQ, p.Lseg - i * BQ);
-          const long long qbase = static_cast<long long>(r) * p.Lseg + i * BQ;
+          const int n = min(BQ, q_len<SPLIT>(p) - i * BQ);
+          const long long qbase = static_cast<long long>(r) * q_len<SPLIT>(p) + i * BQ;
           int qp4[4], qs4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int idx = 4 * lane + e;
-            qp4[e] = idx < n ? __ldg(p.pos + qbase + idx) : INT_MAX;
+            qp4[e] = idx < n ? __ldg((SPLIT ? p.q_pos : p.pos) + qbase + idx) : INT_MAX;
             qs4[e] = (SEG && idx < n) ? __ldg(p.seg + qbase + idx) : INT_MAX;
           }
           int lo = 0, hi = n;
@@ -460,10 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         if (!SEG && !key_dead && i < s_hop[t].y) {
           // first query column at or after this key (the visible suffix)
-          int lo = 0, hi = min(BQ, p.Lseg - i * BQ);
+          int lo = 0, hi = min(BQ, q_len<SPLIT>(p) - i * BQ);
           while (lo < hi) {
             const int mid = (lo + hi) >> 1;
-            if (posat(p, r, i * BQ + mid) >= my_kpos) hi = mid; else lo = mid + 1;
+            if (qposat<SPLIT>(p, r, i * BQ + mid) >= my_kpos) hi = mid; else lo = mid + 1;
           }
           first = lo;
         }
@@ -555,11 +591,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int gi = lane >> 3, gj = lane & 7;
           float* dst0 = p.dq_acc + (rowbase + static_cast<long long>(i) * BQ + quarter * 32 + gi * 8) * D +
                         wg * (D / 2) + gj * 4;
-          const int rows_left = p.Lseg - (i * BQ + quarter * 32 + gi * 8);
+          const int rows_left = q_len<SPLIT>(p) - (i * BQ + quarter * 32 + gi * 8);
           uint32_t g0[32], g1[32];
           tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2), g0);
           if constexpr (D == 128) tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + 32, g1);
           tmem_wait_ld();
+          if constexpr (SPLIT) {  // the caller's accumulator holds dQ itself
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              g0[e] = __float_as_uint(__uint_as_float(g0[e]) * p.scale);
+              if constexpr (D == 128) g1[e] = __float_as_uint(__uint_as_float(g1[e]) * p.scale);
+            }
+          }
           transpose_reduce<D>(g0, dst0, rows_left);
           if constexpr (D == 128) transpose_reduce<D>(g1, dst0 + 32, rows_left);
         }
@@ -577,9 +620,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       if (NIT > 0) tc_fence_after();
-      const long long krow = (static_cast<long long>(kvh) * p.nseg + s) * p.Lseg + k0 + row;
+      const long long krow = (static_cast<long long>(kvh) * p.nseg + s) * k_len<SPLIT>(p) + k0 + row;
       __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + krow * D + wg * (D / 2);
       __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + krow * D + wg * (D / 2);
+      float* dk32 = static_cast<float*>(p.dk) + krow * D + wg * (D / 2);
+      float* dv32 = static_cast<float*>(p.dv) + krow * D + wg * (D / 2);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t gk[32], gv[32];
@@ -591,7 +636,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) gk[e] = gv[e] = 0u;
         }
-        if (key_ok) {
+        if (SPLIT && key_ok) {  // fp32 shares, written or added (this thread owns these elements)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float4 wk = make_float4(__uint_as_float(gk[4 * e + 0]) * p.scale, __uint_as_float(gk[4 * e + 1]) * p.scale,
+                                    __uint_as_float(gk[4 * e + 2]) * p.scale, __uint_as_float(gk[4 * e + 3]) * p.scale);
+            float4 wv = make_float4(__uint_as_float(gv[4 * e + 0]), __uint_as_float(gv[4 * e + 1]),
+                                    __uint_as_float(gv[4 * e + 2]), __uint_as_float(gv[4 * e + 3]));
+            float4* pk = reinterpret_cast<float4*>(dk32 + c * 32) + e;
+            float4* pv = reinterpret_cast<float4*>(dv32 + c * 32) + e;
+            if (p.accumulate) {
+              const float4 ok4 = *pk, ov4 = *pv;
+              wk.x += ok4.x; wk.y += ok4.y; wk.z += ok4.z; wk.w += ok4.w;
+              wv.x += ov4.x; wv.y += ov4.y; wv.z += ov4.z; wv.w += ov4.w;
+            }
+            *pk = wk;
+            *pv = wv;
+          }
+        } else if (key_ok) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             uint4 wk, wv;
@@ -630,9 +692,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Delta_i = dO_i . O_i (fp32) and zeroing of the dQ accumulator rows: one
-// 16-lane group per row, 16-byte loads.
-template <int D>
+// Delta_i = dO_i . O_i (fp32) and (ZERO_DQ) zeroing of the dQ accumulator
+// rows: one 16-lane group per row, 16-byte loads.
+template <int D, bool ZERO_DQ>
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                                 float* __restrict__ delta, float* __restrict__ dq_acc, long long rows) {
   constexpr int V = D / 8;  // 16-byte vectors per bf16 row
@@ -654,8 +716,10 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_
         s = fmaf(fa.y, fb.y, s);
       }
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
-    for (int e = l; e < D / 4; e += 16) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (ZERO_DQ) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + row * D);
+      for (int e = l; e < D / 4; e += 16) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
@@ -690,7 +754,7 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   const long long grid = static_cast<long long>(a.BH / a.group) * a.nseg * nt;  // one CTA per key/value tile
   if (grid == 0) return RATTN_OK;
   if (grid > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
-  bwd_prep_kernel<D><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
+  bwd_prep_kernel<D, true><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   CUtensorMap tq, tk, tv, tdo;
@@ -699,14 +763,18 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
-  const void* kfn = a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true>)
-                         : reinterpret_cast<const void*>(&bwd_kernel<D, false>);
+  const void* kfn = a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true, false>)
+                         : reinterpret_cast<const void*>(&bwd_kernel<D, false, false>);
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
   Params p;
   p.lse = a.lse;
   p.delta = a.delta;
   p.pos = a.pos;
   p.seg = a.seg;
+  p.q_pos = nullptr;
+  p.kv_pos = nullptr;
+  p.Lq = p.Lk = 0;
+  p.accumulate = 0;
   p.BH = a.BH;
   p.group = a.group;
   p.nseg = a.nseg;
@@ -723,13 +791,81 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
   if (a.seg)
-    bwd_kernel<D, true><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+    bwd_kernel<D, true, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
   else
-    bwd_kernel<D, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+    bwd_kernel<D, false, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   const long long n4 = rows * D / 4;
   dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
                                                             static_cast<uint2*>(a.dq), a.scale, n4);
+  return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
+}
+
+template <int D>
+rattn_status launch_split(const PartialBwdArgs& a, const DevCtx& ctx) {
+  using C = Cfg<D>;
+  if (a.Lq > INT32_MAX - BQ || a.Lk > INT32_MAX - BK) return RATTN_ERR_UNSUPPORTED;
+  if (a.group < 1 || a.BH % a.group) return RATTN_ERR_INVALID_ARG;
+  const int nqt = static_cast<int>((a.Lq + BQ - 1) / BQ);
+  const int nkt = static_cast<int>((a.Lk + BK - 1) / BK);
+  const long long grid = static_cast<long long>(a.BH / a.group) * nkt;  // one CTA per key/value tile
+  if (grid == 0) return RATTN_OK;                                       // no key rows: nothing to add
+  if (grid > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
+  if (a.Lq == 0) {  // no query rows: the shares are zero
+    if (a.accumulate) return RATTN_OK;
+    const size_t bytes = static_cast<size_t>(a.BH / a.group) * static_cast<size_t>(a.Lk) * D * sizeof(float);
+    if (cudaMemsetAsync(a.dk, 0, bytes, a.stream) != cudaSuccess ||
+        cudaMemsetAsync(a.dv, 0, bytes, a.stream) != cudaSuccess)
+      return RATTN_ERR_CUDA;
+    return RATTN_OK;
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  rattn_status st;
+  if ((st = make_tmap_bf16(&tq, a.q, D, a.Lq, 1, a.BH, BQ)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tk, a.k, D, a.Lk, 1, a.BH / a.group, BK)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tv, a.v, D, a.Lk, 1, a.BH / a.group, BK)) != RATTN_OK) return st;
+  if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lq, 1, a.BH, BQ)) != RATTN_OK) return st;
+  const void* kfn = reinterpret_cast<const void*>(&bwd_kernel<D, false, true>);
+  if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
+  Params p;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.pos = nullptr;
+  p.seg = nullptr;
+  p.q_pos = a.q_pos;
+  p.kv_pos = a.kv_pos;
+  p.BH = a.BH;
+  p.group = a.group;
+  p.nseg = 1;
+  p.Lseg = 0;
+  p.nq_tiles = nqt;
+  p.nk_tiles = nkt;
+  p.causal = a.causal;
+  p.Lq = static_cast<int>(a.Lq);
+  p.Lk = static_cast<int>(a.Lk);
+  p.accumulate = a.accumulate;
+  p.kv_valid = a.kv_valid;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.dq_acc = a.dq_acc;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.err = ctx.err_word;
+  p.wait_ns = ctx.wait_ns;
+  bwd_kernel<D, false, true><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
+}
+
+template <int D>
+rattn_status launch_prep(const void* o, const void* dout, long long rows, float* delta, float* dq_acc,
+                         cudaStream_t stream) {
+  const unsigned grid = static_cast<unsigned>((rows * 16 + 255) / 256);
+  if (dq_acc)
+    bwd_prep_kernel<D, true><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                      static_cast<const __nv_bfloat16*>(dout), delta, dq_acc, rows);
+  else
+    bwd_prep_kernel<D, false><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                       static_cast<const __nv_bfloat16*>(dout), delta, dq_acc, rows);
   return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
@@ -739,6 +875,22 @@ rattn_status launch_bwd_sm100(const BwdArgs& a, const DevCtx& ctx) {
   if (a.dtype != RATTN_BF16) return RATTN_ERR_UNSUPPORTED;
   if (a.D == 128) return launch<128>(a, ctx);
   if (a.D == 64) return launch<64>(a, ctx);
+  return RATTN_ERR_UNSUPPORTED;
+}
+
+rattn_status launch_partial_bwd_sm100(const PartialBwdArgs& a, const DevCtx& ctx) {
+  if (a.dtype != RATTN_BF16) return RATTN_ERR_UNSUPPORTED;
+  if (a.D == 128) return launch_split<128>(a, ctx);
+  if (a.D == 64) return launch_split<64>(a, ctx);
+  return RATTN_ERR_UNSUPPORTED;
+}
+
+rattn_status launch_bwd_prep_sm100(const void* o, const void* dout, long long rows, int D, float* delta,
+                                   float* dq_acc, cudaStream_t stream) {
+  if (rows == 0) return RATTN_OK;
+  if (rows > (static_cast<long long>(INT_MAX) * 256 - 255) / 16) return RATTN_ERR_UNSUPPORTED;  // grid.x limit
+  if (D == 128) return launch_prep<128>(o, dout, rows, delta, dq_acc, stream);
+  if (D == 64) return launch_prep<64>(o, dout, rows, delta, dq_acc, stream);
   return RATTN_ERR_UNSUPPORTED;
 }
 

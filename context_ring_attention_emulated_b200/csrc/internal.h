@@ -97,6 +97,41 @@ struct BwdArgs {
   cudaStream_t stream;
 };
 rattn_status launch_bwd_sm100(const BwdArgs& a, const DevCtx& ctx);
+
+// One hop of the ring backward with query rows of one rank and key rows of
+// another: q, dout [BH][Lq][D], lse, delta [BH][Lq], q_pos [Lq]; k, v
+// [BH/group][Lk][D], kv_pos [Lk]. dq_acc (fp32 [BH][Lq][D]) receives
+// scale * dS K added; dk, dv (fp32 [BH/group][Lk][D]) receive the block's
+// shares, written (accumulate = 0) or added (1).
+struct PartialBwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;
+  const float* lse;
+  const float* delta;
+  const int32_t* q_pos;
+  const int32_t* kv_pos;
+  int BH;
+  int group;
+  int64_t Lq;
+  int64_t Lk;
+  int D;
+  rattn_dtype dtype;
+  float scale;
+  int causal;
+  int64_t kv_valid;
+  float* dq_acc;
+  float* dk;
+  float* dv;
+  int accumulate;
+  cudaStream_t stream;
+};
+rattn_status launch_partial_bwd_sm100(const PartialBwdArgs& a, const DevCtx& ctx);
+// Delta = rowsum(dO o O) over `rows` bf16 rows of D, and zeroing of dq_acc
+// (fp32, same rows) unless it is NULL.
+rattn_status launch_bwd_prep_sm100(const void* o, const void* dout, long long rows, int D, float* delta,
+                                   float* dq_acc, cudaStream_t stream);
 rattn_status launch_bwd_simt(const BwdArgs& a);
 
 rattn_status launch_permute(const void* x, void* y, int32_t* pos, int BH, int64_t L, int64_t Lp, int row_bytes,
@@ -112,6 +147,7 @@ rattn_status launch_permute_rope(const void* x, void* y, int32_t* pos, int BH, i
 rattn_status launch_unpermute_rope_grad(const void* dy, void* dx, int BH, int64_t L, int64_t Lp, int D,
                                         rattn_dtype dtype, int cp, int layout, double base, int style,
                                         cudaStream_t stream);
+rattn_status launch_grad_fold(float* acc, const float* blk, int64_t n, cudaStream_t stream);
 rattn_status launch_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, int64_t rows,
                           int D, cudaStream_t stream);
 

@@ -1,4 +1,5 @@
-// merge.cu -- standalone online-softmax fold (bandwidth kernel).
+// merge.cu -- standalone online-softmax fold and gradient fold (bandwidth
+// kernels).
 //
 // [Ring-page] "Technical insight": block results are combined through a
 // running max and running normaliser, earlier partial sums being rescaled when
@@ -66,7 +67,25 @@ unsigned grid_for(long long work, int threads) {
   return static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
+// acc += blk over n4 16-byte vectors (the running dK / dV sums of the ring
+// backward across processes).
+__global__ void grad_fold_kernel(float4* __restrict__ acc, const float4* __restrict__ blk, long long n4) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = acc[i];
+    const float4 b = __ldg(blk + i);
+    acc[i] = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+  }
+}
+
 }  // namespace
+
+rattn_status launch_grad_fold(float* acc, const float* blk, int64_t n, cudaStream_t stream) {
+  const long long n4 = n / 4;
+  grad_fold_kernel<<<grid_for(n4, 256), 256, 0, stream>>>(reinterpret_cast<float4*>(acc),
+                                                          reinterpret_cast<const float4*>(blk), n4);
+  return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
+}
 
 rattn_status launch_merge(float* o_acc, float* lse_acc, const float* o_blk, const float* lse_blk, int64_t rows, int D,
                           cudaStream_t stream) {

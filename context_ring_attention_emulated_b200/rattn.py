@@ -52,6 +52,10 @@ SIGNATURES = [
                                 _P, _P, _P, _P, ctypes.c_size_t, _P]),
     ("rattn_ring_bwd_noalloc", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64,
                                     _P, _P, _P, _P]),
+    ("rattn_bwd_prep", _I, [_P, _P, _I, _I, _I64, _I, _I, _P, _P, _P]),
+    ("rattn_partial_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I64, _I64, _I, _I, _F, _I, _I64,
+                               _P, _P, _P, _I, _P]),
+    ("rattn_grad_fold", _I, [_P, _P, _I64, _P]),
     ("rattn_get_device_error", _I, [ctypes.POINTER(_I)]),
     ("rattn_set_wait_limit_ns", _I, [ctypes.c_ulonglong]),
 ]
@@ -316,6 +320,56 @@ def rattn_ring_bwd(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL,
                                                  int(causal), float(scale), int(L_valid), _ptr(dq), _ptr(dk),
                                                  _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream)))
     return dq, dk, dv
+
+
+def rattn_bwd_prep(o, dout, dq_acc=True, delta=None, stream=None):
+    """Delta fp32 [B,H,L] = rowsum(dout * o) for the hop-by-hop backward, and
+    the zeroed fp32 dQ accumulator [B,H,L,D]. dq_acc: True allocates one,
+    a tensor is zeroed in place, None skips it. Returns (delta, dq_acc)."""
+    _need_cuda(o, dout)
+    B, H, L, D = o.shape
+    if dout.shape != o.shape:
+        raise ValueError("o and dout must share one [B, H, L, D] shape")
+    if dq_acc is True:
+        dq_acc = torch.empty(B, H, L, D, dtype=torch.float32, device=o.device)
+    if delta is None:
+        delta = torch.empty(B, H, L, dtype=torch.float32, device=o.device)
+    _need_cuda(dq_acc, delta)
+    _check("rattn_bwd_prep", lib.rattn_bwd_prep(_ptr(o), _ptr(dout), B, H, L, D, _dtype_code(o), _ptr(delta),
+                                                 _ptr(dq_acc), _stream(stream)))
+    return delta, dq_acc
+
+
+def rattn_partial_bwd(q, k, v, dout, lse, delta, q_pos, kv_pos, dq_acc, scale=None, causal=True, kv_valid=2**62,
+                      dk=None, dv=None, accumulate=False, stream=None):
+    """One hop of the backward: adds this K/V block's dQ share to dq_acc (fp32
+    [B,H,Lq,D]) and returns its dK, dV shares (fp32 [B,H_kv,Lk,D]), written
+    into dk / dv when given (added to them with accumulate=True)."""
+    _need_cuda(q, k, v, dout, lse, delta, q_pos, kv_pos, dq_acc, dk, dv)
+    B, H, Lq, D = q.shape
+    H_kv, Lk = k.shape[1], k.shape[2]
+    if k.shape != (B, H_kv, Lk, D) or v.shape != k.shape or dout.shape != q.shape:
+        raise ValueError("k, v must be [B, H_kv, Lk, D] and dout [B, H, Lq, D]")
+    scale = D ** -0.5 if scale is None else scale
+    if accumulate and (dk is None or dv is None):
+        raise ValueError("accumulate=True needs dk and dv to add to")
+    dk = torch.empty(B, H_kv, Lk, D, dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty(B, H_kv, Lk, D, dtype=torch.float32, device=q.device) if dv is None else dv
+    _check("rattn_partial_bwd", lib.rattn_partial_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse),
+                                                       _ptr(delta), _ptr(q_pos), _ptr(kv_pos), B, H, H_kv, Lq, Lk,
+                                                       D, _dtype_code(q), float(scale), int(causal), int(kv_valid),
+                                                       _ptr(dq_acc), _ptr(dk), _ptr(dv), int(bool(accumulate)),
+                                                       _stream(stream)))
+    return dk, dv
+
+
+def rattn_grad_fold(acc, blk, stream=None):
+    """acc += blk (fp32, same shape), in place; returns acc."""
+    _need_cuda(acc, blk)
+    if acc.shape != blk.shape or acc.dtype != torch.float32 or blk.dtype != torch.float32:
+        raise ValueError("acc and blk must be fp32 tensors of one shape")
+    _check("rattn_grad_fold", lib.rattn_grad_fold(_ptr(acc), _ptr(blk), acc.numel(), _stream(stream)))
+    return acc
 
 
 def rattn_ring_fwd_gqa(q, k, v, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None, L_valid=None,

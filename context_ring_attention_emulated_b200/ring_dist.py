@@ -50,15 +50,15 @@ Schedules (rank r of cp ranks; next = r+1, prev = r-1, mod cp):
                 every rank computes its share of dK, dV for all blocks, and
                 ``reduce_scatter_tensor`` returns the sum for its own block.
 
-Block arithmetic. By default (``KernelOps``) the forward of a block runs on this
-library's kernels: ``rattn_partial_fwd``, then ``rattn_merge`` for the fold. The
-results are O and LSE in fp32 (the fold's accumulator, not cast). The backward
-of one block pairs query rows of one rank with key rows of another rank, which
-has separate position arrays. No kernel of this library computes that yet, so
-``KernelOps.bwd`` raises. The schedules take an ``ops`` object with the same
-methods; their tests on CPU (gloo ranks) pass the fp64 reference arithmetic
-there. Only tensors and the exchange are handled here: no attention arithmetic
-lives in this module.
+Block arithmetic. By default (``KernelOps``) every block runs on this library's
+kernels: ``rattn_partial_fwd`` and ``rattn_merge`` in the forward (O and LSE
+come back in fp32, the fold's accumulator); ``rattn_bwd_prep`` (Delta and the
+zeroed fp32 dQ accumulator), ``rattn_partial_bwd`` (one block's dQ added in
+place, its dK, dV shares in fp32) and ``rattn_grad_fold`` (running sums) in
+the backward. The schedules take an ``ops`` object with the same methods; their
+tests on CPU (gloo ranks) pass the fp64 reference arithmetic there. Only
+tensors and the exchange are handled here: no attention arithmetic lives in
+this module.
 
 Failure handling. Every exchange is a ``torch.distributed`` call on the
 caller's process group; give the group a short timeout so that a rank that
@@ -111,7 +111,15 @@ class RingMembership:
 class KernelOps:
     """Block arithmetic on this library's CUDA kernels (contiguous CUDA
     tensors only; the library must be built: importing its binding raises
-    otherwise, and there is no other implementation)."""
+    otherwise, and there is no other implementation).
+
+    fwd(q, k, v, q_pos, kv_pos, scale, causal, kv_valid) -> (o, lse)
+    merge(o_acc, lse_acc, o_blk, lse_blk) -> (o_acc, lse_acc), in place
+    prep(o, do) -> (delta, dq_acc): Delta and a zeroed fp32 dQ accumulator
+    bwd(q, k, v, do, lse, delta, q_pos, kv_pos, scale, causal, kv_valid,
+        dq_acc, dk=None, dv=None) -> (dk, dv): adds the block's dQ share to
+        dq_acc; writes its dK, dV shares into dk, dv (new when None)
+    fold(acc, blk) -> acc: acc += blk, in place"""
 
     def __init__(self):
         from . import rattn
@@ -123,13 +131,15 @@ class KernelOps:
     def merge(self, o_acc, lse_acc, o_blk, lse_blk):
         return self._r.rattn_merge(o_acc, lse_acc, o_blk, lse_blk)
 
-    def delta(self, o, do):
-        raise NotImplementedError("the per-block backward kernels (query and key rows of different ranks, "
-                                  "separate positions) are not built in this library")
+    def prep(self, o, do):
+        return self._r.rattn_bwd_prep(o, do)
 
-    def bwd(self, q, k, v, do, lse, delta, q_pos, kv_pos, scale, causal, kv_valid):
-        raise NotImplementedError("the per-block backward kernels (query and key rows of different ranks, "
-                                  "separate positions) are not built in this library")
+    def bwd(self, q, k, v, do, lse, delta, q_pos, kv_pos, scale, causal, kv_valid, dq_acc, dk=None, dv=None):
+        return self._r.rattn_partial_bwd(q, k, v, do, lse, delta, q_pos, kv_pos, dq_acc, scale, causal, kv_valid,
+                                         dk, dv)
+
+    def fold(self, acc, blk):
+        return self._r.rattn_grad_fold(acc, blk)
 
 
 def ring_peers(group=None):
@@ -216,18 +226,18 @@ def ring_bwd(q, k, v, o, do, lse, pos, scale=None, causal=True, kv_valid=2 ** 62
     """Gradients of ``ring_fwd`` for this rank's rows: dQ of its queries and
     dK, dV of its own key/value rows, summed over every rank's queries.
 
-    q, k, v, do: [B, H, L_loc, D]; o, lse: the forward's outputs for the same
-    rows; pos as in ``ring_fwd``. The running dK, dV sums travel one hop behind
-    the K/V blocks. Returns (dq, dk, dv) in the accumulator precision of
-    ``ops``."""
+    q, k, v, do: [B, H, L_loc, D]; o: the forward output of these rows in the
+    inputs' dtype (as the model keeps it) and lse its fp32 LSE; pos as in
+    ``ring_fwd``. The running dK, dV sums travel one hop behind the K/V
+    blocks. Returns (dq, dk, dv) in the accumulator precision of ``ops``
+    (fp32 with ``KernelOps``)."""
     _check_local(q, k, v, pos)
     ops = KernelOps() if ops is None else ops
     scale = _scale(q, scale)
     rank, cp, nxt, prv = ring_peers(group)
-    delta = ops.delta(o, do)
+    delta, dq = ops.prep(o, do)
     kv_bufs = [[torch.empty_like(t) for t in (k, v, pos)] for _ in range(min(2, cp - 1))]
     cur = [k, v, pos]
-    dq = None
     shares = [None, None]          # this rank's (dk, dv) totals sent at hops t and t-1
     in_bufs = [None, None]         # running sums received for the next hop
     pending = None                 # the dK/dV exchange posted at the end of the previous hop
@@ -236,13 +246,14 @@ def ring_bwd(q, k, v, o, do, lse, pos, scale=None, causal=True, kv_valid=2 ** 62
         if t < cp - 1:
             recv = kv_bufs[t % 2]
             kv_reqs = _exchange(cur, recv, nxt, prv, _TAG_KV, group)
-        gq, gk, gv = ops.bwd(q, cur[0], cur[1], do, lse, delta, pos, cur[2], scale, causal, kv_valid)
-        dq = gq if dq is None else dq.add_(gq)
+        # the buffers of hop t-2, whose send completed at hop t-1's wait
+        reuse = shares[t % 2] if shares[t % 2] is not None else (None, None)
+        gk, gv = ops.bwd(q, cur[0], cur[1], do, lse, delta, pos, cur[2], scale, causal, kv_valid, dq, *reuse)
         if pending is not None:
             _wait(pending)
             dk_in, dv_in = in_bufs[(t - 1) % 2]
-            gk.add_(dk_in)
-            gv.add_(dv_in)
+            ops.fold(gk, dk_in)
+            ops.fold(gv, dv_in)
         shares[t % 2] = (gk, gv)
         if cp > 1:
             if in_bufs[t % 2] is None:
@@ -252,7 +263,7 @@ def ring_bwd(q, k, v, o, do, lse, pos, scale=None, causal=True, kv_valid=2 ** 62
             _wait(kv_reqs)
             cur = recv
     if cp == 1:
-        return dq, shares[0][0], shares[0][1]
+        return (dq,) + shares[0]
     _wait(pending)
     dk, dv = in_bufs[(cp - 1) % 2]
     return dq, dk, dv
@@ -295,20 +306,18 @@ def allgather_bwd(q, k, v, o, do, lse, pos, scale=None, causal=True, kv_valid=2 
     ops = KernelOps() if ops is None else ops
     scale = _scale(q, scale)
     rank, cp, _, _ = ring_peers(group)
-    delta = ops.delta(o, do)
+    delta, dq = ops.prep(o, do)
     if cp == 1:
-        return ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid)
+        return (dq,) + tuple(ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid, dq))
     (kg, wk), (vg, wv), (pg, wp) = (_gather(t, cp, group) for t in (k, v, pos))
-    dq, gk, gv = ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid)
-    dkg = torch.empty((cp,) + tuple(gk.shape), dtype=gk.dtype, device=gk.device)
+    dkg = torch.empty((cp,) + tuple(k.shape), dtype=dq.dtype, device=dq.device)   # every block's shares
     dvg = torch.empty_like(dkg)
-    dkg[rank], dvg[rank] = gk, gv
+    ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid, dq, dkg[rank], dvg[rank])
     _wait([wk, wv, wp])
     for t in range(1, cp):
         s = (rank - t) % cp
-        gq, dkg[s], dvg[s] = ops.bwd(q, kg[s], vg[s], do, lse, delta, pos, pg[s], scale, causal, kv_valid)
-        dq.add_(gq)
-    dk, dv = torch.empty_like(gk), torch.empty_like(gv)
+        ops.bwd(q, kg[s], vg[s], do, lse, delta, pos, pg[s], scale, causal, kv_valid, dq, dkg[s], dvg[s])
+    dk, dv = torch.empty_like(dkg[0]), torch.empty_like(dvg[0])
     for out, full in ((dk, dkg), (dv, dvg)):
         dist.reduce_scatter_tensor(out, full.view((cp * out.shape[0],) + tuple(out.shape[1:])), group=group)
     return dq, dk, dv

@@ -278,6 +278,49 @@ rattn_status rattn_ring_bwd_gqa(const void* q, const void* k, const void* v, con
                                 int64_t L_valid, void* dq, void* dk, void* dv,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* --- One hop at a time: the backward when CP ranks are separate processes.
+ *
+ * [CP-glossary] "How context parallelism works" (each device works on the
+ * K/V block it holds, then passes the block on) and [Megatron-CP] "CP vs SP"
+ * (K and V travel between ranks ring-style or by an all-gather): when every
+ * rank is its own process, each hop of the backward is one call on the
+ * rank's queries and the block in hand, and the dK, dV shares travel back to
+ * the block's owner. The pages show only `.backward()`; these calls split the
+ * plain softmax-attention gradient by key block: with the row's final LSE
+ * and Delta_i = sum_d dO_id O_id of the whole sequence,
+ *   P = exp(scale Q K^T - LSE) (masked),  dV = P^T dO,  dP = dO V^T,
+ *   dS = P o (dP - Delta),  dQ = scale dS K,  dK = scale dS^T Q,
+ * and the shares summed over all blocks are the gradient. bf16 only
+ * (RATTN_F32 returns RATTN_ERR_UNSUPPORTED). */
+
+/* Per-step preparation: delta fp32 [B,H,L] = rowsum(dout o o) of the bf16
+ * [B,H,L,D] forward output and its upstream gradient, and, unless dq_acc is
+ * NULL, zeroing of the fp32 dQ accumulator dq_acc [B,H,L,D]. */
+rattn_status rattn_bwd_prep(const void* o, const void* dout, int B, int H, int64_t L, int D,
+                            rattn_dtype dtype, float* delta, float* dq_acc, void* stream);
+
+/* One hop: the share of one K/V block in the gradient of queries that
+ * attend the whole sequence. q, dout [B,H,Lq,D] and lse, delta fp32 [B,H,Lq]
+ * (the rank's rows; lse as the forward returned it, delta from
+ * rattn_bwd_prep); k, v [B,H_kv,Lk,D] (the block; query head h reads
+ * key/value head h / (H / H_kv)); q_pos int32 [Lq], kv_pos int32 [Lk], both
+ * required and non-decreasing. A key is visible iff (!causal || kv_pos <=
+ * q_pos) and kv_pos < kv_valid. Outputs (fp32, caller-owned, 16-byte
+ * aligned): dq_acc [B,H,Lq,D] += this block's dQ; dk, dv [B,H_kv,Lk,D] =
+ * the block's dK, dV shares (summed over each group's query heads), or +=
+ * them when accumulate = 1. Lk = 0 does nothing; Lq = 0 writes zero shares
+ * (accumulate = 0) or nothing. */
+rattn_status rattn_partial_bwd(const void* q, const void* k, const void* v, const void* dout,
+                               const float* lse, const float* delta, const int32_t* q_pos,
+                               const int32_t* kv_pos, int B, int H, int H_kv, int64_t Lq, int64_t Lk,
+                               int D, rattn_dtype dtype, float scale, int causal, int64_t kv_valid,
+                               float* dq_acc, float* dk, float* dv, int accumulate, void* stream);
+
+/* acc[i] += blk[i] for n fp32 values (n a multiple of 4, both 16-byte
+ * aligned): the running dK / dV sums of a block as it travels back to its
+ * owner. */
+rattn_status rattn_grad_fold(float* acc, const float* blk, int64_t n, void* stream);
+
 /* Size of the device array rattn_ring_bwd_noalloc uses as scratch space. */
 #define RATTN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 

@@ -222,3 +222,41 @@ def test_batch_times_heads_beyond_int32_is_unsupported(rattn):
     assert L.cp_layout_gather(FAKE, FAKE, FAKE, big, big, 16, 16, 64, 1, None) == rattn.ERR_UNSUPPORTED
     assert L.rattn_ring_fwd(FAKE, FAKE, FAKE, FAKE, big, big, 256, 64, 1, 2, 1, 1, ctypes.c_float(0.125), 256,
                             FAKE, FAKE, None) == rattn.ERR_UNSUPPORTED
+
+
+def test_hop_backward_calls_reject_bad_arguments(rattn):
+    """rattn_bwd_prep, rattn_partial_bwd and rattn_grad_fold validate on the
+    host and launch nothing on a bad argument."""
+    L, E, U, OK = rattn.lib, rattn.ERR_INVALID_ARG, rattn.ERR_UNSUPPORTED, rattn.OK
+    BF16, F32 = rattn.BF16, rattn.F32
+    # prep: sizes, dtype, pointers; an empty sequence is a no-op
+    assert L.rattn_bwd_prep(FAKE, FAKE, 0, 1, 8, 64, BF16, FAKE, FAKE, None) == E
+    assert L.rattn_bwd_prep(FAKE, FAKE, 1, 1, 8, 64, F32, FAKE, FAKE, None) == U
+    assert L.rattn_bwd_prep(FAKE, FAKE, 1, 1, 8, 96, BF16, FAKE, FAKE, None) == U
+    assert L.rattn_bwd_prep(MIS, FAKE, 1, 1, 8, 64, BF16, FAKE, FAKE, None) == E
+    assert L.rattn_bwd_prep(FAKE, FAKE, 1, 1, 8, 64, BF16, None, FAKE, None) == E
+    assert L.rattn_bwd_prep(FAKE, FAKE, 1, 1, 8, 64, BF16, FAKE, MIS, None) == E
+    assert L.rattn_bwd_prep(FAKE, FAKE, 1, 1, 0, 64, BF16, FAKE, FAKE, None) == OK
+
+    def hop(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, dout=FAKE, lse=FAKE, delta=FAKE, q_pos=FAKE, kv_pos=FAKE, B=1, H=4, H_kv=2,
+                 Lq=256, Lk=256, D=128, dtype=BF16, scale=0.1, causal=1, kv_valid=2**62, dq=FAKE, dk=FAKE, dv=FAKE,
+                 acc=0)
+        a.update(kw)
+        return L.rattn_partial_bwd(a["q"], a["k"], a["v"], a["dout"], a["lse"], a["delta"], a["q_pos"],
+                                   a["kv_pos"], a["B"], a["H"], a["H_kv"], a["Lq"], a["Lk"], a["D"], a["dtype"],
+                                   a["scale"], a["causal"], a["kv_valid"], a["dq"], a["dk"], a["dv"], a["acc"], None)
+    assert hop(H_kv=3) == E                  # H not a multiple of H_kv
+    assert hop(acc=2) == E and hop(causal=2) == E and hop(scale=0.0) == E and hop(Lq=-1) == E
+    assert hop(dtype=F32, D=64) == U         # tensor-core path only
+    assert hop(D=96) == U
+    assert hop(kv_pos=None) == E and hop(q_pos=None) == E and hop(dk=MIS) == E and hop(dq=None) == E
+    assert hop(k=MIS) == E and hop(lse=0x10002) == E
+    assert hop(Lk=0) == OK                   # no keys: nothing to add
+    assert hop(B=2**16, H=2**16, H_kv=2**16) == U
+    # fold: n a multiple of 4, aligned pointers; n = 0 is a no-op
+    assert L.rattn_grad_fold(FAKE, FAKE, 6, None) == E
+    assert L.rattn_grad_fold(FAKE, FAKE, -4, None) == E
+    assert L.rattn_grad_fold(MIS, FAKE, 8, None) == E
+    assert L.rattn_grad_fold(FAKE, None, 8, None) == E
+    assert L.rattn_grad_fold(FAKE, FAKE, 0, None) == OK

@@ -24,7 +24,8 @@ from context_ring_attention_emulated_b200 import ring_dist
 
 
 class OracleOps:
-    """The block arithmetic of the schedules, from the fp64 oracle (tests only)."""
+    """The block arithmetic of the schedules, from the fp64 oracle (tests
+    only), with the interface of ``ring_dist.KernelOps``."""
 
     def fwd(self, q, k, v, q_pos, kv_pos, scale, causal, kv_valid):
         o, lse = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale, causal, q_pos.numpy(), kv_pos.numpy(),
@@ -35,13 +36,24 @@ class OracleOps:
         o, lse = oracle.merge(o_acc.numpy(), lse_acc.numpy(), o_blk.numpy(), lse_blk.numpy())
         return torch.from_numpy(o), torch.from_numpy(lse)
 
-    def delta(self, o, do):
-        return torch.from_numpy((o.numpy() * do.numpy()).sum(-1))
+    def prep(self, o, do):
+        delta = torch.from_numpy((o.numpy().astype(np.float64) * do.numpy()).sum(-1))
+        return delta, torch.zeros(do.shape, dtype=torch.float64)
 
-    def bwd(self, q, k, v, do, lse, delta, q_pos, kv_pos, scale, causal, kv_valid):
-        g = oracle.attention_bwd_block(q.numpy(), k.numpy(), v.numpy(), do.numpy(), lse.numpy(), delta.numpy(),
-                                       scale, causal, q_pos.numpy(), kv_pos.numpy(), kv_valid)
-        return tuple(torch.from_numpy(np.ascontiguousarray(x)) for x in g)
+    def bwd(self, q, k, v, do, lse, delta, q_pos, kv_pos, scale, causal, kv_valid, dq_acc, dk=None, dv=None):
+        gq, gk, gv = (torch.from_numpy(np.ascontiguousarray(x)) for x in oracle.attention_bwd_block(
+            q.numpy(), k.numpy(), v.numpy(), do.numpy(), lse.numpy(), delta.numpy(), scale, causal, q_pos.numpy(),
+            kv_pos.numpy(), kv_valid))
+        dq_acc += gq
+        if dk is None:
+            return gk, gv
+        dk.copy_(gk)
+        dv.copy_(gv)
+        return dk, dv
+
+    def fold(self, acc, blk):
+        acc += blk
+        return acc
 
 
 LAYOUTS = (oracle.CONTIGUOUS, oracle.HEAD_TAIL, oracle.STRIPED)
@@ -147,8 +159,7 @@ def test_single_rank_ring_is_the_local_attention():
 
 def test_kernel_ops_take_no_cpu_path():
     """The default block arithmetic is the library's CUDA kernels alone: CPU
-    tensors are refused, and the backward, whose per-block kernels are not
-    built, raises rather than running anything else."""
+    tensors are refused by every schedule, forward and backward."""
     port = _free_port()
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=0, world_size=1)
@@ -159,8 +170,10 @@ def test_kernel_ops_take_no_cpu_path():
             ring_dist.ring_fwd(q, k, v, pos)
         with pytest.raises(ValueError, match="CUDA"):
             ring_dist.allgather_fwd(q, k, v, pos)
-        with pytest.raises(NotImplementedError):
+        with pytest.raises(ValueError, match="CUDA"):
             ring_dist.ring_bwd(q, k, v, q, do, q[..., 0], pos)
+        with pytest.raises(ValueError, match="CUDA"):
+            ring_dist.allgather_bwd(q, k, v, q, do, q[..., 0], pos)
         with pytest.raises(ValueError, match="int32"):
             ring_dist.ring_fwd(q, k, v, pos.long(), ops=OracleOps())
         with pytest.raises(ValueError, match="shape"):
