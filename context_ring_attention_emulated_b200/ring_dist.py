@@ -36,11 +36,12 @@ Schedules (rank r of cp ranks; next = r+1, prev = r-1, mod cp):
   ring_bwd      (reading: the pages show only a call to ``.backward()``, so
                 this is the plain gradient of the forward's fold, hop by hop.)
                 delta = rowsum(dO * O) once; at hop t rank r adds block s's
-                share to dQ and computes its share of dK_s, dV_s in fresh fp32
-                buffers. Meanwhile the running sums of dK_s, dV_s arrive from
-                prev, which worked on block s at hop t-1. They are added and
-                the totals go on to next. After the last hop each block's sums
-                arrive at the block's owner.
+                share to dQ and writes its share of dK_s, dV_s into fp32
+                buffers of its own (two pairs, used in turn). Meanwhile the
+                running sums of dK_s, dV_s arrive from prev, which worked on
+                block s at hop t-1. They are folded in and the totals go on
+                to next. After the last hop each block's sums arrive at the
+                block's owner.
   allgather_fwd / allgather_bwd
                 the all-gather option of [Megatron-CP]: K, V and positions are
                 gathered once (the local block's arithmetic runs while the
