@@ -35,9 +35,12 @@ ROPE_BASE = 10000.0  # rotary base of the RoPE workloads (RoFormer's value)
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
 # capture of the current kernel on a half-length case, scaled to the full
 # launch by sequence length (traffic grows with the tensors). Source:
-# profiles/bwd_kernel_bf16_H32_L16000_cp4.md. Set to None when the kernel
-# changes until it is captured again.
-NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": (792.6e6 + 480.4e6) * 2}
+# profiles/bwd_kernel_bf16_H32_L16000_cp4.md. Empty while the kernel has
+# changed since its last capture: that capture (2.55 GB per 32k launch)
+# predates the per-hop instantiation, which changed the ring instantiation's
+# register allocation, so the traffic is reported as null until it is
+# captured again.
+NCU_TRAFFIC = {}
 
 
 def peaks():
