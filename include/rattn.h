@@ -36,7 +36,8 @@
  *     accumulation, D in {64, 128}); RATTN_F32 runs an exact-fp32 SIMT path
  *     (D a multiple of 4, at most 128).
  *   - Position arrays must be non-decreasing within every rank's slice (ring
- *     calls) or over the whole array (rattn_partial_fwd). The layouts produced
+ *     calls) or over the whole array (rattn_partial_fwd, rattn_partial_bwd:
+ *     each of q_pos and kv_pos). The layouts produced
  *     by cp_layout_permute satisfy this; kernels use it to skip and classify
  *     tiles. A key is visible to a query iff (!causal || kv_pos <= q_pos) and
  *     kv_pos < kv_valid (L_valid in ring calls).
