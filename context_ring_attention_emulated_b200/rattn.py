@@ -114,15 +114,69 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _dims(t, n, name):
+    if t.dim() != n:
+        raise ValueError(f"{name} must be {n}-D, got shape {tuple(t.shape)}")
+
+
+def _expect(t, shape, dtype, name):
+    """The library reads and writes whole [B, H, L, D] extents it cannot see:
+    every tensor handed to it must have exactly the shape and dtype the call
+    implies (checked here, before any launch)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _padded(L, cp_size, layout, fn):
+    Lp = cp_layout_padded_len(L, cp_size, layout)
+    if Lp < 0:
+        raise RattnError(fn, ERR_INVALID_ARG)
+    return Lp
+
+
+def _attn(q, k, v, fn, gqa=True, same_len=True):
+    """Shapes of an attention call: q [B,H,Lq,D]; k, v [B,H_kv,Lk,D] in q's
+    dtype; H_kv == H unless the call takes grouped heads, Lk == Lq for the
+    ring calls (one sequence). Returns B, H, Lq, D, H_kv, Lk."""
+    _dims(q, 4, "q")
+    _dims(k, 4, "k")
+    B, H, Lq, D = q.shape
+    H_kv, Lk = k.shape[1], k.shape[2]
+    if not gqa and H_kv != H:
+        raise ValueError(f"{fn}: k and v must have the {H} heads of q, got {H_kv} (grouped heads: the _gqa call)")
+    if same_len and Lk != Lq:
+        raise ValueError(f"{fn}: k and v must have the {Lq} rows of q, got {Lk}")
+    _expect(k, (B, H_kv, Lk, D), q.dtype, "k")
+    _expect(v, (B, H_kv, Lk, D), q.dtype, "v")
+    return B, H, Lq, D, H_kv, Lk
+
+
+def _bwd_io(q, k, o, dout, lse, dq, dk, dv):
+    B, H, L, D = q.shape
+    _expect(o, q.shape, q.dtype, "o")
+    _expect(dout, q.shape, q.dtype, "dout")
+    _expect(lse, (B, H, L), torch.float32, "lse")
+    _expect(dq, q.shape, q.dtype, "dq")
+    _expect(dk, k.shape, q.dtype, "dk")
+    _expect(dv, k.shape, q.dtype, "dv")
+
+
 def cp_layout_padded_len(L, cp_size, layout=LAYOUT_HEAD_TAIL):
     return int(lib.cp_layout_padded_len(int(L), int(cp_size), int(layout)))
 
 
 def cp_layout_permute(x, cp_size, layout=LAYOUT_HEAD_TAIL, y=None, pos=None, stream=None):
     """x [B,H,L,D] -> (y [B,H,Lp,D] rank-major, pos int32 [Lp])."""
-    _need_cuda(x)
+    _dims(x, 4, "x")
     B, H, L, D = x.shape
-    Lp = cp_layout_padded_len(L, cp_size, layout)
+    Lp = _padded(L, cp_size, layout, "cp_layout_permute")
+    _expect(y, (B, H, Lp, D), x.dtype, "y")
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _need_cuda(x)
     if y is None:
         y = torch.empty(B, H, Lp, D, dtype=x.dtype, device=x.device)
     if pos is None:
@@ -135,8 +189,10 @@ def cp_layout_permute(x, cp_size, layout=LAYOUT_HEAD_TAIL, y=None, pos=None, str
 
 def cp_layout_unpermute(y, L, cp_size, layout=LAYOUT_HEAD_TAIL, x=None, stream=None):
     """y [B,H,Lp,D] rank-major -> x [B,H,L,D] global order."""
-    _need_cuda(y)
+    _dims(y, 4, "y")
     B, H, Lp, D = y.shape
+    _expect(x, (B, H, L, D), y.dtype, "x")
+    _need_cuda(y)
     if x is None:
         x = torch.empty(B, H, L, D, dtype=y.dtype, device=y.device)
     _need_cuda(x)
@@ -149,9 +205,12 @@ def cp_layout_permute_rope(x, cp_size, layout=LAYOUT_HEAD_TAIL, rope_base=10000.
                            pos=None, stream=None):
     """x [B,H,L,D] -> (y [B,H,Lp,D] rank-major with RoPE at the global
     positions, pos int32 [Lp])."""
-    _need_cuda(x)
+    _dims(x, 4, "x")
     B, H, L, D = x.shape
-    Lp = cp_layout_padded_len(L, cp_size, layout)
+    Lp = _padded(L, cp_size, layout, "cp_layout_permute_rope")
+    _expect(y, (B, H, Lp, D), x.dtype, "y")
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _need_cuda(x)
     if y is None:
         y = torch.empty(B, H, Lp, D, dtype=x.dtype, device=x.device)
     if pos is None:
@@ -167,8 +226,10 @@ def cp_layout_unpermute_rope_grad(dy, L, cp_size, layout=LAYOUT_HEAD_TAIL, rope_
                                   dx=None, stream=None):
     """dy [B,H,Lp,D] rank-major (gradient w.r.t. the rotated tensor) ->
     dx [B,H,L,D] global order (gradient w.r.t. the un-rotated input)."""
-    _need_cuda(dy)
+    _dims(dy, 4, "dy")
     B, H, Lp, D = dy.shape
+    _expect(dx, (B, H, L, D), dy.dtype, "dx")
+    _need_cuda(dy)
     if dx is None:
         dx = torch.empty(B, H, L, D, dtype=dy.dtype, device=dy.device)
     _need_cuda(dx)
@@ -197,9 +258,13 @@ def cp_layout_varlen_plan(cu_seqlens, cp_size, layout=LAYOUT_HEAD_TAIL):
 
 def cp_layout_gather(x, src, y=None, stream=None):
     """y[:, :, i] = x[:, :, src[i]] (zero rows where src[i] < 0); src device int32."""
-    _need_cuda(x, src)
+    _dims(x, 4, "x")
+    _dims(src, 1, "src")
     B, H, T, D = x.shape
     T_out = src.numel()
+    _expect(src, (T_out,), torch.int32, "src")
+    _expect(y, (B, H, T_out, D), x.dtype, "y")
+    _need_cuda(x, src)
     if y is None:
         y = torch.empty(B, H, T_out, D, dtype=x.dtype, device=x.device)
     _need_cuda(y)
@@ -210,8 +275,11 @@ def cp_layout_gather(x, src, y=None, stream=None):
 
 def cp_layout_scatter(y, src, T_x, x=None, stream=None):
     """x[:, :, src[i]] = y[:, :, i] for src[i] >= 0; x [B, H, T_x, D]."""
-    _need_cuda(y, src)
+    _dims(y, 4, "y")
     B, H, T_y, D = y.shape
+    _expect(src, (T_y,), torch.int32, "src")
+    _expect(x, (B, H, T_x, D), y.dtype, "x")
+    _need_cuda(y, src)
     if x is None:
         x = torch.zeros(B, H, T_x, D, dtype=y.dtype, device=y.device)
     _need_cuda(x)
@@ -223,9 +291,12 @@ def cp_layout_scatter(y, src, T_x, x=None, stream=None):
 def rattn_ring_fwd_varlen(q, k, v, gkey, segid, cp_size, causal=True, scale=None, o=None, lse=None, stream=None):
     """Ring forward over a packed layout (cp_layout_varlen_plan order); gkey and
     segid device int32 [Tp]. Returns (O, LSE)."""
-    _need_cuda(q, k, v, gkey, segid)
-    B, H, Tp, D = q.shape
-    H_kv = k.shape[1]
+    B, H, Tp, D, H_kv, _ = _attn(q, k, v, "rattn_ring_fwd_varlen")
+    _expect(gkey, (Tp,), torch.int32, "gkey")
+    _expect(segid, (Tp,), torch.int32, "segid")
+    _expect(o, q.shape, q.dtype, "o")
+    _expect(lse, (B, H, Tp), torch.float32, "lse")
+    _need_cuda(q, k, v, gkey, segid, o, lse)
     scale = D ** -0.5 if scale is None else scale
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty(B, H, Tp, dtype=torch.float32, device=q.device) if lse is None else lse
@@ -238,9 +309,11 @@ def rattn_ring_fwd_varlen(q, k, v, gkey, segid, cp_size, causal=True, scale=None
 def rattn_ring_bwd_varlen(q, k, v, o, dout, lse, gkey, segid, cp_size, causal=True, scale=None, dq=None, dk=None,
                           dv=None, workspace=None, stream=None):
     """Gradients of rattn_ring_fwd_varlen: returns (dQ, dK, dV)."""
-    _need_cuda(q, k, v, o, dout, lse, gkey, segid)
-    B, H, Tp, D = q.shape
-    H_kv = k.shape[1]
+    B, H, Tp, D, H_kv, _ = _attn(q, k, v, "rattn_ring_bwd_varlen")
+    _expect(gkey, (Tp,), torch.int32, "gkey")
+    _expect(segid, (Tp,), torch.int32, "segid")
+    _bwd_io(q, k, o, dout, lse, dq, dk, dv)
+    _need_cuda(q, k, v, o, dout, lse, gkey, segid, dq, dk, dv, workspace)
     scale = D ** -0.5 if scale is None else scale
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
@@ -258,9 +331,12 @@ def rattn_ring_bwd_varlen(q, k, v, o, dout, lse, gkey, segid, cp_size, causal=Tr
 def rattn_partial_fwd(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True, kv_valid=2**62,
                       o=None, lse=None, stream=None):
     """One partial attention: returns (O fp32 [B,H,Lq,D], LSE fp32 [B,H,Lq])."""
-    _need_cuda(q, k, v, q_pos, kv_pos)
-    B, H, Lq, D = q.shape
-    Lk = k.shape[2]
+    B, H, Lq, D, _, Lk = _attn(q, k, v, "rattn_partial_fwd", gqa=False, same_len=False)
+    _expect(q_pos, (Lq,), torch.int32, "q_pos")
+    _expect(kv_pos, (Lk,), torch.int32, "kv_pos")
+    _expect(o, (B, H, Lq, D), torch.float32, "o")
+    _expect(lse, (B, H, Lq), torch.float32, "lse")
+    _need_cuda(q, k, v, q_pos, kv_pos, o, lse)
     scale = D ** -0.5 if scale is None else scale
     if o is None:
         o = torch.empty(B, H, Lq, D, dtype=torch.float32, device=q.device)
@@ -274,8 +350,13 @@ def rattn_partial_fwd(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True,
 
 def rattn_merge(o_acc, lse_acc, o_blk, lse_blk, stream=None):
     """In-place online-softmax fold of (o_blk, lse_blk) into (o_acc, lse_acc)."""
-    _need_cuda(o_acc, lse_acc, o_blk, lse_blk)
+    _dims(o_acc, 4, "o_acc")
     B, H, Lq, D = o_acc.shape
+    _expect(o_acc, (B, H, Lq, D), torch.float32, "o_acc")
+    _expect(o_blk, (B, H, Lq, D), torch.float32, "o_blk")
+    _expect(lse_acc, (B, H, Lq), torch.float32, "lse_acc")
+    _expect(lse_blk, (B, H, Lq), torch.float32, "lse_blk")
+    _need_cuda(o_acc, lse_acc, o_blk, lse_blk)
     _check("rattn_merge", lib.rattn_merge(_ptr(o_acc), _ptr(lse_acc), _ptr(o_blk), _ptr(lse_blk), B, H, Lq, D,
                                            _stream(stream)))
     return o_acc, lse_acc
@@ -284,8 +365,11 @@ def rattn_merge(o_acc, lse_acc, o_blk, lse_blk, stream=None):
 def rattn_ring_fwd(q, k, v, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None, L_valid=None,
                    o=None, lse=None, stream=None):
     """Emulated ring forward on rank-major q/k/v [B,H,Lp,D]: returns (O, LSE)."""
-    _need_cuda(q, k, v, pos)
-    B, H, Lp, D = q.shape
+    B, H, Lp, D, _, _ = _attn(q, k, v, "rattn_ring_fwd", gqa=False)
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _expect(o, q.shape, q.dtype, "o")
+    _expect(lse, (B, H, Lp), torch.float32, "lse")
+    _need_cuda(q, k, v, pos, o, lse)
     scale = D ** -0.5 if scale is None else scale
     L_valid = Lp if L_valid is None else L_valid
     if o is None:
@@ -305,8 +389,10 @@ def rattn_ring_bwd_workspace_size(B, H, Lp, D):
 def rattn_ring_bwd(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=True, scale=None,
                    L_valid=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
     """Gradients of the ring forward (rank-major): returns (dQ, dK, dV)."""
-    _need_cuda(q, k, v, o, dout, lse, pos)
-    B, H, Lp, D = q.shape
+    B, H, Lp, D, _, _ = _attn(q, k, v, "rattn_ring_bwd", gqa=False)
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _bwd_io(q, k, o, dout, lse, dq, dk, dv)
+    _need_cuda(q, k, v, o, dout, lse, pos, dq, dk, dv, workspace)
     scale = D ** -0.5 if scale is None else scale
     L_valid = Lp if L_valid is None else L_valid
     dq = torch.empty_like(q) if dq is None else dq
@@ -326,10 +412,13 @@ def rattn_bwd_prep(o, dout, dq_acc=True, delta=None, stream=None):
     """Delta fp32 [B,H,L] = rowsum(dout * o) for the hop-by-hop backward, and
     the zeroed fp32 dQ accumulator [B,H,L,D]. dq_acc: True allocates one,
     a tensor is zeroed in place, None skips it. Returns (delta, dq_acc)."""
-    _need_cuda(o, dout)
+    _dims(o, 4, "o")
     B, H, L, D = o.shape
-    if dout.shape != o.shape:
-        raise ValueError("o and dout must share one [B, H, L, D] shape")
+    _expect(dout, o.shape, o.dtype, "dout")
+    if dq_acc is not True:
+        _expect(dq_acc, (B, H, L, D), torch.float32, "dq_acc")
+    _expect(delta, (B, H, L), torch.float32, "delta")
+    _need_cuda(o, dout)
     if dq_acc is True:
         dq_acc = torch.empty(B, H, L, D, dtype=torch.float32, device=o.device)
     if delta is None:
@@ -345,11 +434,16 @@ def rattn_partial_bwd(q, k, v, dout, lse, delta, q_pos, kv_pos, dq_acc, scale=No
     """One hop of the backward: adds this K/V block's dQ share to dq_acc (fp32
     [B,H,Lq,D]) and returns its dK, dV shares (fp32 [B,H_kv,Lk,D]), written
     into dk / dv when given (added to them with accumulate=True)."""
+    B, H, Lq, D, H_kv, Lk = _attn(q, k, v, "rattn_partial_bwd", same_len=False)
+    _expect(dout, q.shape, q.dtype, "dout")
+    for t, name, shape in ((lse, "lse", (B, H, Lq)), (delta, "delta", (B, H, Lq)), (q_pos, "q_pos", (Lq,)),
+                           (kv_pos, "kv_pos", (Lk,)), (dq_acc, "dq_acc", (B, H, Lq, D))):
+        if t is None:
+            raise ValueError(f"rattn_partial_bwd: {name} is required")
+        _expect(t, shape, torch.int32 if name.endswith("pos") else torch.float32, name)
+    _expect(dk, (B, H_kv, Lk, D), torch.float32, "dk")
+    _expect(dv, (B, H_kv, Lk, D), torch.float32, "dv")
     _need_cuda(q, k, v, dout, lse, delta, q_pos, kv_pos, dq_acc, dk, dv)
-    B, H, Lq, D = q.shape
-    H_kv, Lk = k.shape[1], k.shape[2]
-    if k.shape != (B, H_kv, Lk, D) or v.shape != k.shape or dout.shape != q.shape:
-        raise ValueError("k, v must be [B, H_kv, Lk, D] and dout [B, H, Lq, D]")
     scale = D ** -0.5 if scale is None else scale
     if accumulate and (dk is None or dv is None):
         raise ValueError("accumulate=True needs dk and dv to add to")
@@ -365,9 +459,9 @@ def rattn_partial_bwd(q, k, v, dout, lse, delta, q_pos, kv_pos, dq_acc, scale=No
 
 def rattn_grad_fold(acc, blk, stream=None):
     """acc += blk (fp32, same shape), in place; returns acc."""
-    _need_cuda(acc, blk)
     if acc.shape != blk.shape or acc.dtype != torch.float32 or blk.dtype != torch.float32:
         raise ValueError("acc and blk must be fp32 tensors of one shape")
+    _need_cuda(acc, blk)
     _check("rattn_grad_fold", lib.rattn_grad_fold(_ptr(acc), _ptr(blk), acc.numel(), _stream(stream)))
     return acc
 
@@ -376,11 +470,11 @@ def rattn_ring_fwd_gqa(q, k, v, pos, cp_size, layout=LAYOUT_HEAD_TAIL, causal=Tr
                        o=None, lse=None, stream=None):
     """Ring forward with grouped key/value heads: q [B,H,Lp,D], k/v
     [B,H_kv,Lp,D] (H_kv from k's shape); returns (O [B,H,Lp,D], LSE)."""
-    _need_cuda(q, k, v, pos)
-    B, H, Lp, D = q.shape
-    H_kv = k.shape[1]
-    if k.shape != (B, H_kv, Lp, D) or v.shape != k.shape:
-        raise ValueError("k and v must be [B, H_kv, Lp, D] matching q")
+    B, H, Lp, D, H_kv, _ = _attn(q, k, v, "rattn_ring_fwd_gqa")
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _expect(o, q.shape, q.dtype, "o")
+    _expect(lse, (B, H, Lp), torch.float32, "lse")
+    _need_cuda(q, k, v, pos, o, lse)
     scale = D ** -0.5 if scale is None else scale
     L_valid = Lp if L_valid is None else L_valid
     if o is None:
@@ -397,11 +491,10 @@ def rattn_ring_bwd_gqa(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HEAD_T
                        L_valid=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
     """Gradients of rattn_ring_fwd_gqa: returns (dQ [B,H,Lp,D], dK, dV
     [B,H_kv,Lp,D], each summed over its group of query heads)."""
-    _need_cuda(q, k, v, o, dout, lse, pos)
-    B, H, Lp, D = q.shape
-    H_kv = k.shape[1]
-    if k.shape != (B, H_kv, Lp, D) or v.shape != k.shape:
-        raise ValueError("k and v must be [B, H_kv, Lp, D] matching q")
+    B, H, Lp, D, H_kv, _ = _attn(q, k, v, "rattn_ring_bwd_gqa")
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _bwd_io(q, k, o, dout, lse, dq, dk, dv)
+    _need_cuda(q, k, v, o, dout, lse, pos, dq, dk, dv, workspace)
     scale = D ** -0.5 if scale is None else scale
     L_valid = Lp if L_valid is None else L_valid
     dq = torch.empty_like(q) if dq is None else dq
@@ -421,8 +514,10 @@ def rattn_ring_bwd_noalloc(q, k, v, o, dout, lse, pos, cp_size, layout=LAYOUT_HE
                            L_valid=None, dq=None, dk=None, dv=None, stream=None):
     """rattn_ring_bwd without a workspace: scratch comes from the library's own
     fixed device array (for callers that cannot allocate device memory)."""
-    _need_cuda(q, k, v, o, dout, lse, pos)
-    B, H, Lp, D = q.shape
+    B, H, Lp, D, _, _ = _attn(q, k, v, "rattn_ring_bwd_noalloc", gqa=False)
+    _expect(pos, (Lp,), torch.int32, "pos")
+    _bwd_io(q, k, o, dout, lse, dq, dk, dv)
+    _need_cuda(q, k, v, o, dout, lse, pos, dq, dk, dv)
     scale = D ** -0.5 if scale is None else scale
     L_valid = Lp if L_valid is None else L_valid
     dq = torch.empty_like(q) if dq is None else dq

@@ -260,3 +260,58 @@ def test_hop_backward_calls_reject_bad_arguments(rattn):
     assert L.rattn_grad_fold(MIS, FAKE, 8, None) == E
     assert L.rattn_grad_fold(FAKE, None, 8, None) == E
     assert L.rattn_grad_fold(FAKE, FAKE, 0, None) == OK
+
+
+def test_binding_checks_shapes_and_dtypes_before_any_launch(rattn):
+    """The library cannot see tensor extents: the binding refuses tensors whose
+    shape or dtype does not match the call (before its CUDA check, so this runs
+    here on CPU tensors), and lets matching ones through to that check."""
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    t = lambda *s, d=bf: torch.zeros(*s, dtype=d)
+    q, kv, pos = t(1, 4, 16, 64), t(1, 4, 16, 64), t(16, d=i32)
+    bad = [
+        lambda: rattn.cp_layout_permute(q, 2, y=t(1, 4, 8, 64)),
+        lambda: rattn.cp_layout_permute(q, 2, pos=t(16, d=torch.int64)),
+        lambda: rattn.cp_layout_unpermute(q, 16, 2, x=t(1, 4, 16, 64, d=f32)),
+        lambda: rattn.cp_layout_gather(q, t(16, d=torch.int64)),
+        lambda: rattn.cp_layout_gather(q, pos, y=t(1, 4, 15, 64)),
+        lambda: rattn.cp_layout_scatter(q, t(15, d=i32), 16),
+        lambda: rattn.rattn_ring_fwd(q, t(1, 2, 16, 64), t(1, 2, 16, 64), pos, 2),     # grouped heads: _gqa call
+        lambda: rattn.rattn_ring_fwd(q, kv, kv, t(15, d=i32), 2),
+        lambda: rattn.rattn_ring_fwd(q, kv, kv, pos, 2, o=t(1, 4, 16, 64, d=f32)),
+        lambda: rattn.rattn_ring_fwd(q, kv, kv, pos, 2, lse=t(1, 4, 16)),
+        lambda: rattn.rattn_ring_fwd(q, kv.float(), kv, pos, 2),
+        lambda: rattn.rattn_ring_bwd(q, kv, kv, q, q.float(), t(1, 4, 16, d=f32), pos, 2),
+        lambda: rattn.rattn_ring_bwd(q, kv, kv, q, q, t(1, 4, 16, d=f32), pos, 2, dk=t(1, 4, 8, 64)),
+        lambda: rattn.rattn_ring_fwd_gqa(q, t(1, 2, 16, 64), t(1, 4, 16, 64), pos, 2),
+        lambda: rattn.rattn_ring_bwd_noalloc(q, kv, kv, q, q, t(1, 4, 15, d=f32), pos, 2),
+        lambda: rattn.rattn_partial_fwd(q, t(1, 2, 9, 64), t(1, 2, 9, 64)),
+        lambda: rattn.rattn_partial_fwd(q, t(1, 4, 9, 64), t(1, 4, 9, 64), q_pos=t(9, d=i32)),
+        lambda: rattn.rattn_merge(t(1, 4, 16, 64, d=f32), t(1, 4, 16, d=f32), q, t(1, 4, 16, d=f32)),
+        lambda: rattn.rattn_bwd_prep(q, q, dq_acc=t(1, 4, 16, 64)),
+        lambda: rattn.rattn_bwd_prep(q, q, delta=t(1, 4, 15, d=f32)),
+        lambda: rattn.rattn_partial_bwd(q, kv, kv, q, t(1, 4, 16, d=f32), t(1, 4, 16, d=f32), None, pos,
+                                        t(1, 4, 16, 64, d=f32)),
+        lambda: rattn.rattn_partial_bwd(q, kv, kv, q, t(1, 4, 16, d=f32), t(1, 4, 16, d=f32), pos, pos,
+                                        t(1, 4, 16, 64, d=f32), dk=t(1, 4, 16, 64)),
+        lambda: rattn.rattn_grad_fold(t(8, d=f32), t(8)),
+        lambda: rattn.rattn_ring_fwd_varlen(q, kv, kv, t(15, d=i32), pos, 2),
+    ]
+    for i, call in enumerate(bad):
+        with pytest.raises(ValueError) as e:
+            call()
+        assert "CUDA" not in str(e.value), f"case {i} reached the CUDA check: {e.value}"
+    with pytest.raises(rattn.RattnError):
+        rattn.cp_layout_permute(q, 0)                   # no padded length for cp = 0
+    good = [
+        lambda: rattn.cp_layout_permute(q, 2),
+        lambda: rattn.rattn_ring_fwd(q, kv, kv, pos, 2),
+        lambda: rattn.rattn_ring_fwd_gqa(q, t(1, 2, 16, 64), t(1, 2, 16, 64), pos, 2),
+        lambda: rattn.rattn_partial_fwd(q, t(1, 4, 9, 64), t(1, 4, 9, 64), t(16, d=i32), t(9, d=i32)),
+        lambda: rattn.rattn_partial_bwd(q, t(1, 2, 9, 64), t(1, 2, 9, 64), q, t(1, 4, 16, d=f32),
+                                        t(1, 4, 16, d=f32), pos, t(9, d=i32), t(1, 4, 16, 64, d=f32)),
+        lambda: rattn.rattn_bwd_prep(q, q),
+    ]
+    for call in good:
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
