@@ -139,6 +139,43 @@ def test_ring_and_allgather_match_full_attention(world):
             np.testing.assert_allclose(ag, ref, rtol=0, atol=1e-12)
 
 
+def _subgroup_main(rank, world, port, out):
+    """Two rings at once on four processes: {0, 2} and {1, 3} (CP groups
+    inside a larger job); each must exchange only within its own group."""
+    _init(rank, world, port)
+    try:
+        groups = [dist.new_group([0, 2]), dist.new_group([1, 3])]
+        g = groups[rank % 2]
+        cp, gr = 2, dist.get_rank(g)
+        L = 10
+        q, k, v, do = _inputs(L, 700 + rank % 2)           # each ring its own sequence
+        Lp, _, pos = oracle.perm_index(L, cp, oracle.HEAD_TAIL)
+        qp, kp, vp, dop = (torch.from_numpy(oracle.permute(x, cp, oracle.HEAD_TAIL)[0]) for x in (q, k, v, do))
+        pl = ring_dist.rank_slice(torch.from_numpy(np.asarray(pos, dtype=np.int32)), gr, cp)
+        ql, kl, vl, dol = (ring_dist.rank_slice(x, gr, cp) for x in (qp, kp, vp, dop))
+        o, lse = ring_dist.ring_fwd(ql, kl, vl, pl, SCALE, True, L, group=g, ops=OracleOps())
+        dq, dk, dv = ring_dist.ring_bwd(ql, kl, vl, o, dol, lse, pl, SCALE, True, L, group=g, ops=OracleOps())
+        out[rank] = dict(gr=gr, o=o.numpy(), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rings_on_subgroups_exchange_within_their_group():
+    world, port = 4, _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_subgroup_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for ring, members in ((0, (0, 2)), (1, (1, 3))):
+        q, k, v, do = _inputs(10, 700 + ring)
+        parts = sorted((res[r]["gr"], res[r]) for r in members)
+        o = _assemble([p["o"] for _, p in parts], 10, 2, oracle.HEAD_TAIL)
+        np.testing.assert_allclose(o, oracle.attention(q, k, v, SCALE, True)[0], rtol=0, atol=1e-12)
+        for name, ref in zip(("dq", "dk", "dv"), oracle.attention_bwd(q, k, v, do, SCALE, True)):
+            got = _assemble([p[name] for _, p in parts], 10, 2, oracle.HEAD_TAIL)
+            np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
 def test_single_rank_ring_is_the_local_attention():
     port = _free_port()
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
