@@ -61,6 +61,11 @@ tests on CPU (gloo ranks) pass the fp64 reference arithmetic there. Only
 tensors and the exchange are handled here: no attention arithmetic lives in
 this module.
 
+With NCCL, set each process's device (``torch.cuda.set_device``) before the
+first call: batched point-to-point operations need it, and every rank of the
+group takes part in each exchange (all ranks call the same schedule with the
+same cp, shapes and dtypes).
+
 Failure handling. Every exchange is a ``torch.distributed`` call on the
 caller's process group; give the group a short timeout so that a rank that
 stops answering ends the others' next exchange with an error rather than a
