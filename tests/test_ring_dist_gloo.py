@@ -295,3 +295,15 @@ def test_exchange_with_a_dead_peer_raises_instead_of_hanging():
     assert not alive, "a rank hung on the exchange"
     assert res[1] == "exited"
     assert res[0].startswith("error"), res[0]
+
+
+def test_test_ops_mirror_the_kernel_ops_interface():
+    """The schedules tested here with OracleOps run on the GPU with KernelOps:
+    both must offer the same methods with the same parameters."""
+    import inspect
+    names = [n for n in vars(ring_dist.KernelOps) if not n.startswith("_")]
+    assert sorted(names) == ["bwd", "fold", "fwd", "merge", "prep"]
+    for n in names:
+        a = inspect.signature(getattr(ring_dist.KernelOps, n))
+        b = inspect.signature(getattr(OracleOps, n))
+        assert list(a.parameters) == list(b.parameters), n
