@@ -324,7 +324,6 @@ def cpu_sample_run(w, min_seconds=0.0):
     """The oracle as it stands on a bounded sample: the first 8000 tokens (one
     emulated rank's worth) of one head, causal fwd (+ bwd), fp64 on the host;
     further heads are added until at least ``min_seconds`` of CPU work ran."""
-    import numpy as np
     import oracle
     Ls = min(8000, w.L)
     g = torch.Generator().manual_seed(0)

@@ -1,6 +1,5 @@
 """GPU parity of the ring backward (dQ, dK, dV from the saved LSE) against
 the oracle's textbook softmax-attention gradient, in fp64."""
-import numpy as np
 import pytest
 import torch
 

@@ -19,7 +19,7 @@ import pytest
 import torch
 
 import oracle
-from context_ring_attention_emulated_b200.workloads import WORKLOADS, make_qkv, make_tensor
+from context_ring_attention_emulated_b200.workloads import WORKLOADS, make_tensor
 from tests.gpu_common import check_grad, check_lse, check_o, load_rattn, to64
 
 pytestmark = pytest.mark.gpu

@@ -4,7 +4,6 @@ shards into independent replicas: no data-path collective exists)."""
 import os
 import socket
 
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
