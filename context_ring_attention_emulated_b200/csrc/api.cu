@@ -199,8 +199,9 @@ rattn_status cp_layout_varlen_plan(const int32_t* cu_seqlens, int nseq, int cp_s
   return RATTN_OK;
 }
 
-static rattn_status check_gather(const void* a, const void* b, const int32_t* src, int B, int H, int64_t Ta,
-                                 int64_t Tb, int D, rattn_dtype dtype) {
+// Sizes of a packed-layout gather or scatter (pointers are checked by the callers,
+// which know which of them an empty side leaves unused).
+static rattn_status check_gather(int B, int H, int64_t Ta, int64_t Tb, int D, rattn_dtype dtype) {
   const int es = elem_size(dtype);
   if (!es || B < 1 || H < 1 || D < 1 || Ta < 0 || Tb < 0) return RATTN_ERR_INVALID_ARG;
   if (Ta > INT32_MAX || Tb > INT32_MAX || !bh_fits(B, H)) return RATTN_ERR_UNSUPPORTED;
@@ -211,7 +212,7 @@ static rattn_status check_gather(const void* a, const void* b, const int32_t* sr
 
 rattn_status cp_layout_gather(const void* x, void* y, const int32_t* src, int B, int H, int64_t T_in,
                               int64_t T_out, int D, rattn_dtype dtype, void* stream) {
-  rattn_status st = check_gather(x, y, src, B, H, T_in, T_out, D, dtype);
+  rattn_status st = check_gather(B, H, T_in, T_out, D, dtype);
   if (st != RATTN_OK || T_out == 0) return st;
   if (!y || !src || !aligned(y, 16) || !aligned(src, 4) || (T_in > 0 && (!x || !aligned(x, 16))))
     return RATTN_ERR_INVALID_ARG;
@@ -221,7 +222,7 @@ rattn_status cp_layout_gather(const void* x, void* y, const int32_t* src, int B,
 
 rattn_status cp_layout_scatter(const void* y, void* x, const int32_t* src, int B, int H, int64_t T_y,
                                int64_t T_x, int D, rattn_dtype dtype, void* stream) {
-  rattn_status st = check_gather(y, x, src, B, H, T_y, T_x, D, dtype);
+  rattn_status st = check_gather(B, H, T_y, T_x, D, dtype);
   if (st != RATTN_OK || T_y == 0 || T_x == 0) return st;
   if (!x || !y || !src || !aligned(x, 16) || !aligned(y, 16) || !aligned(src, 4)) return RATTN_ERR_INVALID_ARG;
   return launch_scatter(y, x, src, B * H, T_y, T_x, D * elem_size(dtype), static_cast<cudaStream_t>(stream));
