@@ -14,6 +14,8 @@ workload (each emulates all CP ranks on its own GPU, so no data crosses
 GPUs); value is the work of all ranks over the max-over-ranks device time.
 """
 import argparse
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -32,15 +34,14 @@ METRIC = "ring-attn fwd/bwd TFLOP/s (causal FLOPs) on 1 B200; % of BF16 tensor p
 DEFAULT = "bf16_L32000_cp4_fwdbwd"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROPE_BASE = 10000.0  # rotary base of the RoPE workloads (RoFormer's value)
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
-# capture of the current kernel on a half-length case, scaled to the full
-# launch by sequence length (traffic grows with the tensors). Source:
-# profiles/bwd_kernel_bf16_H32_L16000_cp4.md. Empty while the kernel has
-# changed since its last capture: that capture (2.55 GB per 32k launch)
-# predates the per-hop instantiation, which changed the ring instantiation's
-# register allocation, so the traffic is reported as null until it is
-# captured again.
+# DRAM bytes (read + write) per launch of the dominant kernel from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the kernel as it
+# stands, taken on a smaller case and scaled to the workload's launch by the
+# sequence length. Empty while the kernel has changed since its last capture.
 NCU_TRAFFIC = {}
+# Dense bf16 tensor rate of one SM: a 128x128x16 MMA every 64 cycles.
+SM_COUNT = 148
+TENSOR_FLOP_PER_CLK_SM = 8192
 
 
 def peaks():
@@ -80,7 +81,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -316,30 +317,173 @@ def run_ours(args, w, rank, world, local):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # Rows 0..Ls-1 of the first heads, inputs and results of the last timed
+    # step: under a causal mask they depend on nothing past row Ls, so the
+    # oracle can recompute them from this prefix alone.
+    sample = None
+    if w.causal and not w.docs and Hkv == H:
+        Ls, nh = min(8000, L), min(8, B * H)
+        pick = lambda t: t.reshape(B * H, L, D)[:nh, :Ls].float().cpu()
+        sample = {"q": pick(q), "k": pick(k), "v": pick(v), "do": pick(do), "o": pick(out["o"]),
+                  "dq": pick(out["dq"]) if w.bwd else None, "rows": Ls}
     return {"ms": ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
-            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps}
+            "h2d": h2d, "d2h": d2h, "launches": launches_per_step * args.steps, "sample": sample}
 
 
-def cpu_sample_run(w, min_seconds=0.0):
+def median_event_ms(fn, reps, warmup, stream):
+    """Median CUDA-event time of ``fn`` on ``stream`` over ``reps`` calls after
+    ``warmup`` untimed ones."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
+def tensor_rate_at(sm_mhz):
+    """Dense bf16 tensor-core FLOP/s of the whole GPU at an SM clock (MHz)."""
+    return SM_COUNT * TENSOR_FLOP_PER_CLK_SM * sm_mhz * 1e6 if sm_mhz else None
+
+
+def extra_measurements(local, pk):
+    """Kernels the default step does not time, each measured on its own after
+    the step's timed regions: the 1M-token causal ring forward (8 heads, cp=8
+    head-tail), and the bandwidth kernels (merge, permute, unpermute) at the
+    32k and 1M sizes. Inputs are larger than L2 in every case."""
+    from context_ring_attention_emulated_b200 import rattn
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    res = {}
+
+    w = WORKLOADS["bf16_L1M_cp8"]
+    q, k, v = make_qkv(w, dev, seed=0)
+    Lp = rattn.cp_layout_padded_len(w.L, w.cp, w.layout)
+    qp, pos = rattn.cp_layout_permute(q, w.cp, w.layout)
+    kp, _ = rattn.cp_layout_permute(k, w.cp, w.layout)
+    vp, _ = rattn.cp_layout_permute(v, w.cp, w.layout)
+    o = torch.empty_like(qp)
+    lse = torch.empty(w.B, w.H, Lp, dtype=torch.float32, device=dev)
+    fwd = lambda: rattn.rattn_ring_fwd(qp, kp, vp, pos, w.cp, w.layout, True, w.scale, L_valid=w.L, o=o, lse=lse)
+    with ClockSampler(local) as clk:
+        ms = median_event_ms(fwd, 3, 1, stream)
+    c = clk.summary()
+    tf = w.causal_flops_fwd() / (ms / 1e3) / 1e12
+    at_clk = tensor_rate_at(c["sm_mhz"])
+    res["ring_fwd_" + w.name] = {"ms": ms, "tflops": tf, "frac_of_burst": tf / burst,
+                                 "frac_at_clock": tf * 1e12 / at_clk if at_clk else None, "clocks": c,
+                                 "reps": "median of 3 after 1 warm-up"}
+
+    def bw_entry(name, fn, nbytes, reps=10):
+        ms_ = median_event_ms(fn, reps, 3, stream)
+        gbs = nbytes / (ms_ / 1e3) / 1e9
+        res[name] = {"ms": ms_, "GB_per_s": gbs, "frac_of_hbm": gbs / hbm, "bytes": nbytes}
+
+    es = 2
+    n1m = w.B * w.H * w.L * w.D * es
+    bw_entry("permute_" + w.name, lambda: rattn.cp_layout_permute(q, w.cp, w.layout, y=qp, pos=pos), 2 * n1m + 4 * Lp)
+    bw_entry("unpermute_" + w.name, lambda: rattn.cp_layout_unpermute(qp, w.L, w.cp, w.layout, x=q), 2 * n1m)
+    del q, k, v, qp, kp, vp, o, lse, pos
+    torch.cuda.empty_cache()
+
+    w = WORKLOADS["bf16_L32000_cp4"]
+    x = make_qkv(w, dev, seed=0)[0]
+    Lp = rattn.cp_layout_padded_len(w.L, w.cp, w.layout)
+    y = torch.empty(w.B, w.H, Lp, w.D, dtype=x.dtype, device=dev)
+    pos = torch.empty(Lp, dtype=torch.int32, device=dev)
+    n32 = w.B * w.H * w.L * w.D * es
+    bw_entry("permute_" + w.name, lambda: rattn.cp_layout_permute(x, w.cp, w.layout, y=y, pos=pos), 2 * n32 + 4 * Lp)
+    bw_entry("unpermute_" + w.name, lambda: rattn.cp_layout_unpermute(y, w.L, w.cp, w.layout, x=x), 2 * n32)
+    rows = w.B * w.H * w.L
+    o_acc = torch.randn(w.B, w.H, w.L, w.D, device=dev)
+    o_blk = torch.randn(w.B, w.H, w.L, w.D, device=dev)
+    l_acc = torch.randn(w.B, w.H, w.L, device=dev)
+    l_blk = torch.randn(w.B, w.H, w.L, device=dev)
+    bw_entry("merge_" + w.name, lambda: rattn.rattn_merge(o_acc, l_acc, o_blk, l_blk), rows * (12 * w.D + 12))
+    err, site = rattn.rattn_get_device_error()
+    if err != rattn.OK:
+        raise RuntimeError(f"device-side wait timed out at site {site}")
+    return res
+
+
+def source_digest():
+    """Commit of the checkout when git can tell, and a digest of the library
+    sources and this file (which identifies the code when no .git travels)."""
+    sha = None
+    try:
+        r = subprocess.run(["git", "rev-parse", "HEAD"], cwd=ROOT, capture_output=True, text=True, timeout=10)
+        if r.returncode == 0:
+            sha = r.stdout.strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "context_ring_attention_emulated_b200")
+    files = sorted(glob.glob(os.path.join(pkg, "csrc", "*")) + glob.glob(os.path.join(ROOT, "include", "*.h")) +
+                   [os.path.join(pkg, "rattn.py"), os.path.abspath(__file__)])
+    for f in files:
+        h.update(os.path.relpath(f, ROOT).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return {"git": sha, "src_sha256": h.hexdigest()[:16]}
+
+
+def cpu_sample_run(w, min_seconds=0.0, sample=None):
     """The oracle as it stands on a bounded sample: the first 8000 tokens (one
     emulated rank's worth) of one head, causal fwd (+ bwd), fp64 on the host;
-    further heads are added until at least ``min_seconds`` of CPU work ran."""
+    further heads are added until at least ``min_seconds`` of CPU work ran.
+
+    With ``sample`` (rows 0..Ls-1 of the first heads of the GPU run: inputs,
+    O and dQ), the oracle runs on exactly those inputs, and the GPU's O and dQ
+    on those rows are compared with its results (a causal prefix depends on
+    nothing after it), giving the line a parity record."""
+    import numpy as np
+
     import oracle
-    Ls = min(8000, w.L)
+    Ls = sample["rows"] if sample else min(8000, w.L)
+    n_avail = sample["q"].shape[0] if sample else w.B * w.H
     g = torch.Generator().manual_seed(0)
     heads, dt = 0, 0.0
-    while heads < w.B * w.H and (heads == 0 or dt < min_seconds):
-        q, k, v, do = (torch.randn(Ls, w.D, generator=g).to(w.torch_dtype).double().numpy() for _ in range(4))
+    err = {"o_max_abs": 0.0, "o_viol": 0, "dq_max_abs": 0.0, "dq_ref_max": 0.0}
+    while heads < n_avail and (heads == 0 or dt < min_seconds):
+        if sample:
+            q, k, v, do = (sample[n][heads].double().numpy() for n in ("q", "k", "v", "do"))
+        else:
+            q, k, v, do = (torch.randn(Ls, w.D, generator=g).to(w.torch_dtype).double().numpy() for _ in range(4))
         t0 = time.perf_counter()
-        oracle.attention(q, k, v, w.scale, w.causal, row_block=1000)
-        if w.bwd:
-            oracle.attention_bwd(q, k, v, do, w.scale, w.causal, row_block=1000)
+        o_ref, _ = oracle.attention(q, k, v, w.scale, w.causal, row_block=1000)
+        grads = oracle.attention_bwd(q, k, v, do, w.scale, w.causal, row_block=1000) if w.bwd else None
         dt += time.perf_counter() - t0
+        if sample:
+            e = np.abs(sample["o"][heads].double().numpy() - o_ref)
+            err["o_max_abs"] = max(err["o_max_abs"], float(e.max()))
+            err["o_viol"] += int((e > 2e-2 + 1e-2 * np.abs(o_ref)).sum())
+            if grads is not None and sample["dq"] is not None:
+                err["dq_max_abs"] = max(err["dq_max_abs"],
+                                        float(np.abs(sample["dq"][heads].double().numpy() - grads[0]).max()))
+                err["dq_ref_max"] = max(err["dq_ref_max"], float(np.abs(grads[0]).max()))
         heads += 1
     fl = heads * 4.0 * w.D * Ls * Ls * (0.5 if w.causal else 1.0) * (3.5 if w.bwd else 1.0)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{heads} head(s) x first {Ls} tokens, {'fwd+bwd' if w.bwd else 'fwd'}, numpy fp64 "
-                      f"BLAS, {dt:.2f} s"}
+    out = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": f"{heads} head(s) x first {Ls} tokens{' of the GPU run' if sample else ''}, "
+                     f"{'fwd+bwd' if w.bwd else 'fwd'}, numpy fp64 BLAS, {dt:.2f} s"}
+    if sample:
+        par = {"rows": f"heads 0..{heads - 1}, global rows 0..{Ls - 1} of the last timed step",
+               "o_max_abs": err["o_max_abs"], "o_elements_outside_tol": err["o_viol"],
+               "tolerance": "O: |x-ref| <= 2e-2 + 1e-2|ref|; dQ: 3e-2 max-abs"}
+        if w.bwd:
+            par["dq_max_abs"] = err["dq_max_abs"]
+            par["dq_max_abs_over_ref_max"] = err["dq_max_abs"] / err["dq_ref_max"] if err["dq_ref_max"] else None
+        par["pass"] = err["o_viol"] == 0 and (not w.bwd or err["dq_max_abs"] <= 3e-2)
+        out["parity"] = par
+    return out
 
 
 def blas_threads():
@@ -361,6 +505,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the per-kernel measurements after the step")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     flops_step, fwd_flops = step_flops(w)
@@ -402,6 +547,8 @@ def main():
     sustained = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     achieved = kflops / (kms / 1e3) / 1e12
+    at_clk = tensor_rate_at(r["clocks"]["sm_mhz"])
+    traffic = NCU_TRAFFIC.get(w.name) if w.bwd else None
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -411,18 +558,24 @@ def main():
         "kernels": {"ring_fwd": {"ms": r["fwd_ms"], "tflops": fwd_flops / (r["fwd_ms"] / 1e3) / 1e12},
                     "ring_bwd": ({"ms": r["bwd_ms"], "tflops": 2.5 * fwd_flops / (r["bwd_ms"] / 1e3) / 1e12}
                                  if r["bwd_ms"] else None)},
-        "roofline": {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": sustained,
-                     "peak_kind": f"bf16_tflops_sustained ({pk_kind}); timed inside a long step",
-                     "unit": "TFLOP/s", "frac": achieved / sustained, "frac_of_burst": achieved / burst,
-                     "traffic": NCU_TRAFFIC.get(w.name) if w.bwd else None},
+        "roofline": {"kernel": kname, "bound": "tensor", "achieved": achieved, "peak": burst,
+                     "peak_kind": f"bf16_tflops burst ({pk_kind})", "unit": "TFLOP/s", "frac": achieved / burst,
+                     "frac_of_sustained": achieved / sustained,
+                     "tensor_rate_at_clock": at_clk / 1e12 if at_clk else None,
+                     "frac_at_clock": achieved * 1e12 / at_clk if at_clk else None,
+                     "traffic": traffic["bytes"] if traffic else None,
+                     "traffic_over_algorithmic": traffic["ratio"] if traffic else None},
         "clocks": r["clocks"],
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
+        "source": source_digest(),
     }
+    if rank == 0 and world == 1:
+        if not args.no_extra and w.name == DEFAULT:
+            line["extra"] = extra_measurements(local, pk)
+        line["cpu_baseline"] = cpu_sample_run(w, min_seconds=10.0, sample=r["sample"])
     if rank == 0:
-        if world == 1:
-            line["cpu_baseline"] = cpu_sample_run(w, min_seconds=10.0)
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist

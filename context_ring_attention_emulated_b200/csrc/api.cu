@@ -110,6 +110,22 @@ rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t r
   return r == CUDA_SUCCESS ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
+rattn_status make_tmap_f32_acc(CUtensorMap* map, void* base, int D, int64_t rows, int nseg, int64_t outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return RATTN_ERR_CUDA;
+  if (rows < 1) rows = 1;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(nseg), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(rows) * D * 4,
+                                 static_cast<cuuint64_t>(nseg) * rows * D * 4};
+  const cuuint32_t box[4] = {32u, 128u, 1u, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RATTN_OK : RATTN_ERR_CUDA;
+}
+
 }  // namespace rattn
 
 using namespace rattn;
@@ -269,7 +285,16 @@ rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v, cons
                                const int32_t* kv_pos, int B, int H, int64_t Lq, int64_t Lk, int D,
                                rattn_dtype dtype, float scale, int causal, int64_t kv_valid, float* o, float* lse,
                                void* stream) {
-  if (B < 1 || H < 1 || Lq < 0 || Lk < 0 || (causal != 0 && causal != 1) || !(scale > 0.f && scale < INFINITY))
+  return rattn_partial_fwd_gqa(q, k, v, q_pos, kv_pos, B, H, H, Lq, Lk, D, dtype, scale, causal, kv_valid, o, lse,
+                               stream);
+}
+
+rattn_status rattn_partial_fwd_gqa(const void* q, const void* k, const void* v, const int32_t* q_pos,
+                                   const int32_t* kv_pos, int B, int H, int H_kv, int64_t Lq, int64_t Lk, int D,
+                                   rattn_dtype dtype, float scale, int causal, int64_t kv_valid, float* o,
+                                   float* lse, void* stream) {
+  if (B < 1 || H < 1 || H_kv < 1 || H % H_kv || Lq < 0 || Lk < 0 || (causal != 0 && causal != 1) ||
+      !(scale > 0.f && scale < INFINITY))
     return RATTN_ERR_INVALID_ARG;
   rattn_status st = check_attn_d(D, dtype);
   if (st != RATTN_OK) return st;
@@ -285,6 +310,7 @@ rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v, cons
   a.q_pos = q_pos;
   a.kv_pos = kv_pos;
   a.BH = B * H;
+  a.group = H / H_kv;
   a.nseg = 1;
   a.Lq_seg = Lq;
   a.Lk_seg = Lk;

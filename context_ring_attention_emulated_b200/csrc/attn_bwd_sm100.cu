@@ -10,22 +10,25 @@
 // (r - s) mod cp) and its dK/dV travel with it; here one CTA keeps one
 // 128-key K/V tile of rank s resident and walks every rank's query tiles in
 // that hop order, skipping tiles the causal relation fully masks. dK and dV
-// accumulate in TMEM; each query tile's dQ contribution is transposed
-// within 8-lane groups by shuffles and added into an fp32 workspace with
-// coalesced vector reductions (whole 128-byte lines per warp instruction),
-// converted to the output dtype at the end.
+// accumulate in TMEM. Each query tile's dQ contribution is read out of TMEM
+// by a warpgroup of its own and added into an fp32 workspace by TMA tile
+// reduce-adds from shared memory, which proceed in the background while the
+// next tiles are computed; the workspace is converted to the output dtype at
+// the end.
 //
-// Warp roles (320 threads):
-//   warp 0      producer: K, V once; per query tile Q, dO by TMA and the
-//               tile's LSE (pre-scaled by log2 e) and Delta into shared memory;
-//   warp 1      TMEM allocation and tcgen05.mma issue (one thread);
-//   warps 2..9  two warpgroups, one thread per TMEM lane each: P^T and dS^T
-//               for its key row over the warpgroup's 64 query columns, then
-//               the dQ read-out for its query row over half of D, finally
-//               half of dK/dV.
-// TMEM columns: A [0,128) S^T; warpgroup g then overwrites its own columns
-// [64g, 64g+64) with P^T (bf16, [64g, 64g+32)) and dS^T ([64g+32, 64g+64));
-// B [128,256) dP^T, then dQ; dV [256,256+D); dK [256+D,256+2D).
+// Warp roles (448 threads):
+//   warps 0..3   dQ read-out: one thread per query row, 32-column chunks
+//                staged 128-byte swizzled, one thread issues the reduce-adds;
+//   warps 4..11  two warpgroups, one thread per key row (TMEM lane) each:
+//                P^T and dS^T over the warpgroup's 64 query columns, finally
+//                half of dK/dV each;
+//   warp 12      producer: K, V once; per query tile Q and dO by TMA and the
+//                tile's LSE (pre-scaled by log2 e) and Delta into shared memory;
+//   warp 13      TMEM allocation and tcgen05.mma issue (one thread).
+// TMEM columns: [0,128) S^T, then P^T (bf16, warpgroup g at [64g, 64g+32));
+// [128,256) dP^T, then dS^T (bf16, at 128 + [64g, 64g+32)), then dQ;
+// dV [256,256+D); dK [256+D,256+2D). dS also goes to a swizzled shared tile,
+// the A operand of dQ = dS K.
 //
 // Grouped key/value heads: the CTA of a K/V tile walks the query tiles of
 // every query head of its group, so dK/dV sum over the group in TMEM. Packed
@@ -48,33 +51,48 @@
 namespace rattn {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int BQ = 128;   // query rows per tile
-constexpr int BK = 128;   // key rows per CTA
+constexpr int kThreads = 448;  // 14 warps
+constexpr int BQ = 128;        // query rows per tile
+constexpr int BK = 128;        // key rows per CTA
 constexpr int kMaxHops = 64;
+constexpr int kWarpProducer = 12;
+constexpr int kWarpMma = 13;
+constexpr int kWarpCompute0 = 4;  // warps 4..11: two compute warpgroups
+constexpr int kReduceBar = 1;     // named barrier of the dQ warpgroup (warps 0..3)
 
 template <int D>
 struct Cfg {
-  static constexpr int NSQ = (D == 128) ? 2 : 3;   // Q/dO stages
+  static constexpr int NSQ = 2;                   // Q stages (each with its LSE, Delta and mask flag)
+  static constexpr int NSO = (D == 128) ? 1 : 2;  // dO stages
   static constexpr int TILE = 128 * D * 2;
   static constexpr int NBOX = D / 64;
-  static constexpr int BOX = 128 * 128;            // one 128-row x 64-element box
-  static constexpr uint32_t T_A = 0, T_B = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr int BOX = 128 * 128;           // one 128-row x 64-element box
+  static constexpr int NCH = D / 32;              // 32-column chunks of a dQ tile
+  static constexpr int CHUNK = 128 * 32 * 4;      // one staged fp32 dQ chunk
+  static constexpr int NSTG = 2;                  // dQ staging buffers
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
   static constexpr uint32_t T_COLS = 512;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;                 // NSQ stages
-  static constexpr int OFF_DO = OFF_Q + NSQ * TILE;          // NSQ stages
-  static constexpr int OFF_DS = OFF_DO + NSQ * TILE;         // 128 x 128 bf16, two boxes
-  static constexpr int OFF_LSE = OFF_DS + 2 * BOX;           // NSQ x 128 floats
+  static constexpr int OFF_DO = OFF_Q + NSQ * TILE;          // NSO stages
+  static constexpr int OFF_DS = OFF_DO + NSO * TILE;         // 128 keys x 128 queries bf16, two boxes
+  static constexpr int OFF_STG = OFF_DS + 2 * BOX;           // NSTG staged dQ chunks
+  static constexpr int OFF_LSE = OFF_STG + NSTG * CHUNK;     // NSQ x 128 floats
   static constexpr int OFF_DELTA = OFF_LSE + NSQ * 128 * 4;  // NSQ x 128 floats
   static constexpr int OFF_BAR = OFF_DELTA + NSQ * 128 * 4;
-  static constexpr int NBAR = 1 + 2 * NSQ + 7;
+  // barrier indices
+  static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + NSQ, B_OF = B_QE + NSQ, B_OE = B_OF + NSO,
+                       B_SF = B_OE + NSO, B_PR = B_SF + 1, B_DPF = B_PR + 1, B_DSR = B_DPF + 1, B_DKD = B_DSR + 1,
+                       B_DVD = B_DKD + 1, B_DQF = B_DVD + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
+                       B_DRAIN = B_FIN + 1, NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_FULL = OFF_MISC + 16;            // NSQ ints: tile needs no masking
-  static constexpr int OFF_HOP = OFF_FULL + 16;             // int2 table
-  static_assert(OFF_HOP % 8 == 0 && OFF_BAR % 8 == 0, "shared-memory alignment");
+  static constexpr int OFF_FULL = OFF_MISC + 16;  // NSQ ints: tile needs no masking
+  static constexpr int OFF_HOP = OFF_FULL + 16;   // int2 table
   static constexpr int SMEM = OFF_HOP + kMaxHops * 8;
+  static_assert(OFF_STG % 1024 == 0 && OFF_DS % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_DO % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+  static_assert(OFF_HOP % 8 == 0 && OFF_BAR % 8 == 0 && NSQ <= 4, "shared-memory alignment");
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -86,7 +104,6 @@ struct Params {
   int BH, group, nseg, Lseg, nq_tiles, nk_tiles, causal;
   long long kv_valid;
   float scale, scale_log2;
-  float* dq_acc;
   void* dk;
   void* dv;
   int* err;
@@ -144,54 +161,57 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
 }
 
-// In: v = 32 consecutive fp32 values (8 float4 slots) of this lane's row.
-// Lanes 8g..8g+7 transpose their 8 x 8 float4 slots by xor shuffles (three
-// butterfly stages), after which lane (g, j) holds, in slot k, float4 j of
-// row 8g + k; then one reduction per slot adds four whole 128-byte rows per
-// warp instruction. dst = element (row 8g, column 4j) of this warp's rows;
-// only rows k < rows_left exist.
+// The dQ warpgroup's hand-off of one 128-row x 32-column fp32 chunk (this
+// thread's row in v) to the TMA: wait until the staging buffer's previous
+// reduce-add has read it, write the row 128-byte swizzled (16-byte piece j of
+// row r at piece j ^ (r mod 8): conflict-free for a warp's 32 rows), make the
+// writes visible to the async proxy, and let one thread issue the tile
+// reduce-add into the accumulator at (column c0, row r0) of segment `seg` of
+// (batch, head) `bh`.
 template <int D>
-__device__ __forceinline__ void transpose_reduce(uint32_t (&v)[32], float* dst, int rows_left) {
-  const int j = threadIdx.x & 7;
+__device__ __forceinline__ void stage_dq_chunk(const uint32_t (&v)[32], uint8_t* buf, int row, bool elected,
+                                               bool wait_buffer, const CUtensorMap* tm, int c0, int r0, int seg,
+                                               int bh) {
+  if (elected && wait_buffer) bulk_wait_group_read<Cfg<D>::NSTG - 1>();
+  bar_sync(kReduceBar, 128);
+  uint8_t* rowp = buf + row * 128;
 #pragma unroll
-  for (int sh = 4; sh >= 1; sh >>= 1) {
-    const bool hi = (j & sh) != 0;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      if (x & sh) continue;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t send = hi ? v[4 * x + e] : v[4 * (x | sh) + e];
-        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, sh);
-        if (hi) v[4 * x + e] = recv;
-        else v[4 * (x | sh) + e] = recv;
-      }
-    }
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(rowp + ((j ^ (row & 7)) << 4)) = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                                                                          v[4 * j + 3]);
+  fence_proxy_async_smem();
+  bar_sync(kReduceBar, 128);
+  if (elected) {
+    tma_reduce_add_4d(tm, buf, c0, r0, seg, bh);
+    bulk_commit_group();
   }
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    if (k < rows_left)
-      red_add_v4(dst + static_cast<long long>(k) * D, __uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
-                 __uint_as_float(v[4 * k + 2]), __uint_as_float(v[4 * k + 3]));
 }
 
+// 14 warps share an SM's four register-file partitions 4/4/3/3, so a thread
+// may hold at most 16,384 / (4 x 32) = 128 registers.
 template <int D, bool SEG, bool SPLIT>  // SEG: packed sequences; SPLIT: one hop across processes
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, const Params p) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const __grid_constant__ CUtensorMap tm_dq, const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* bar_kv_full = bars;
-  uint64_t* bar_q_full = bars + 1;
-  uint64_t* bar_q_empty = bar_q_full + C::NSQ;
-  uint64_t* bar_s_full = bar_q_empty + C::NSQ;
-  uint64_t* bar_dp_full = bar_s_full + 1;
-  uint64_t* bar_ds_ready = bar_dp_full + 1;
-  uint64_t* bar_a_free = bar_ds_ready + 1;
-  uint64_t* bar_dq_full = bar_a_free + 1;
-  uint64_t* bar_dq_free = bar_dq_full + 1;
-  uint64_t* bar_drain = bar_dq_free + 1;
+  uint64_t* bar_kv_full = bars + C::B_KV;
+  uint64_t* bar_q_full = bars + C::B_QF;
+  uint64_t* bar_q_empty = bars + C::B_QE;
+  uint64_t* bar_o_full = bars + C::B_OF;
+  uint64_t* bar_o_empty = bars + C::B_OE;
+  uint64_t* bar_s_full = bars + C::B_SF;      // S^T(j) in TMEM
+  uint64_t* bar_p_ready = bars + C::B_PR;     // P^T(j) written over it (one arrival per compute warp)
+  uint64_t* bar_dp_full = bars + C::B_DPF;    // dP^T(j) in TMEM
+  uint64_t* bar_ds_ready = bars + C::B_DSR;   // dS^T(j) over dP^T(j) and dS(j) in shared memory
+  uint64_t* bar_dk_done = bars + C::B_DKD;    // dK MMA of j completed (dS^T(j) consumed)
+  uint64_t* bar_dv_done = bars + C::B_DVD;    // dV MMA of j completed (P^T(j) consumed)
+  uint64_t* bar_dq_full = bars + C::B_DQF;    // dQ(j) in TMEM (dS(j) in shared memory consumed)
+  uint64_t* bar_dq_empty = bars + C::B_DQE;   // dQ(j) read out of TMEM (one arrival per dQ warp)
+  uint64_t* bar_fin = bars + C::B_FIN;        // every MMA completed
+  uint64_t* bar_drain = bars + C::B_DRAIN;
 
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -199,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // packed sequences, else the first tile with no masked element (the visible
   // tiles then run to the last tile)
   int2* s_hop = reinterpret_cast<int2*>(smem + C::OFF_HOP);
-  volatile int* s_full = reinterpret_cast<volatile int*>(smem + C::OFF_FULL);  // per Q/dO stage
+  volatile int* s_full = reinterpret_cast<volatile int*>(smem + C::OFF_FULL);  // per Q stage
   float* s_lse = reinterpret_cast<float*>(smem + C::OFF_LSE);
   float* s_delta = reinterpret_cast<float*>(smem + C::OFF_DELTA);
 
@@ -230,21 +250,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar_q_full[i], 1);
       mbar_init(&bar_q_empty[i], 1);
     }
+    for (int i = 0; i < C::NSO; ++i) {
+      mbar_init(&bar_o_full[i], 1);
+      mbar_init(&bar_o_empty[i], 1);
+    }
     mbar_init(bar_s_full, 1);
+    mbar_init(bar_p_ready, 8);
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_ds_ready, 8);
-    mbar_init(bar_a_free, 1);
+    mbar_init(bar_dk_done, 1);
+    mbar_init(bar_dv_done, 1);
     mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 8);
+    mbar_init(bar_dq_empty, 4);
+    mbar_init(bar_fin, 1);
     mbar_init(bar_drain, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(s_tmem, C::T_COLS);
+  if (warp == kWarpMma) tmem_alloc(s_tmem, C::T_COLS);
 
-  // Per hop t the query segment is r = (s + t) mod nseg. Visible query tiles
-  // form a suffix [first_vis, nq_tiles) and unmasked ones a suffix
-  // [first_full, nq_tiles), since positions are non-decreasing in a segment.
   // Per hop t the query segment is r = (s + t) mod nseg. Visible query tiles
   // form a range [first_vis, end_vis): positions (and segids for packed
   // sequences) are non-decreasing in a segment, so both ends are found by
@@ -290,10 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int t = 0; t < p.nseg; ++t) NIT += (SEG ? s_hop[t].y : p.nq_tiles) - s_hop[t].x;
   NIT *= p.group;  // the same tiles for every query head of the group
 
-  int issued_q = 0;
+  int issued_q = 0, issued_o = 0;
   bool kv_issued = false;
 
-  if (warp == 0) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     if (NIT > 0) {
       if (lane == 0) {
@@ -352,101 +376,151 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (lane == 0) {
-            mbar_arrive_expect_tx(&bar_q_full[st], 2 * C::TILE);
-            for (int b = 0; b < C::NBOX; ++b) {
+            mbar_arrive_expect_tx(&bar_q_full[st], C::TILE);
+            for (int b = 0; b < C::NBOX; ++b)
               tma_load_4d(smem + C::OFF_Q + st * C::TILE + b * C::BOX, &tm_q, &bar_q_full[st], b * 64, i * BQ, r,
                           bh);
-              tma_load_4d(smem + C::OFF_DO + st * C::TILE + b * C::BOX, &tm_do, &bar_q_full[st], b * 64, i * BQ,
-                          r, bh);
-            }
           }
           ++issued_q;
+          const int so = it % C::NSO;
+          const uint32_t uo = it / C::NSO;
+          if (uo > 0 && !warp_wait(&bar_o_empty[so], (uo - 1) & 1, s_abort, p.wait_ns)) {
+            if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_LOAD);
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&bar_o_full[so], C::TILE);
+            for (int b = 0; b < C::NBOX; ++b)
+              tma_load_4d(smem + C::OFF_DO + so * C::TILE + b * C::BOX, &tm_do, &bar_o_full[so], b * 64, i * BQ,
+                          r, bh);
+          }
+          ++issued_o;
         }
       }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ----------------------------------------------------------- MMA issue
+    // Per query tile j: S^T(j) = K Q^T, dP^T(j) = V dO^T, dV += P^T dO,
+    // dK += dS^T Q (dS^T read from TMEM over dP^T), dQ(j) = dS K (into the
+    // dP^T columns once dK(j) has read them). Issue order, steady state:
+    //   dK(i), dQ(i), dV(i+1), dP(i+1), S(i+2)
+    // so that the read-out of dQ(i) overlaps dV(i+1), and the softmax of
+    // tile i+2 and the dS of tile i+1 overlap dK / dQ and S.
     if (lane == 0 && NIT > 0) {
-      const uint32_t idesc_t = idesc_bf16_f32(BK, BQ, 0, 0);    // S^T, dP^T: K-major A and B
-      const uint32_t idesc_g = idesc_bf16_f32(BK, D, 0, 1);     // dV, dK: A in TMEM, B MN-major
-      const uint32_t idesc_q = idesc_bf16_f32(BQ, D, 1, 1);     // dQ: A (dS) and B (K) MN-major
+      const uint32_t idesc_t = idesc_bf16_f32(BK, BQ, 0, 0);  // S^T, dP^T: K-major A and B
+      const uint32_t idesc_g = idesc_bf16_f32(BK, D, 0, 1);   // dV, dK: A in TMEM, B MN-major
+      const uint32_t idesc_q = idesc_bf16_f32(BQ, D, 1, 1);   // dQ: A (dS) and B (K) MN-major
       const uint32_t sK = smem_u32(smem + C::OFF_K);
       const uint32_t sV = smem_u32(smem + C::OFF_V);
       const uint32_t sDS = smem_u32(smem + C::OFF_DS);
-      bool ok = mbar_wait(bar_kv_full, 0, s_abort, p.wait_ns);
-      for (int it = 0; it < NIT && ok; ++it) {
-        const int st = it % C::NSQ;
-        const uint32_t sQ = smem_u32(smem + C::OFF_Q + st * C::TILE);
-        const uint32_t sDO = smem_u32(smem + C::OFF_DO + st * C::TILE);
-        ok = mbar_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns);
-        if (ok && it > 0) ok = mbar_wait(bar_a_free, (it - 1) & 1, s_abort, p.wait_ns);
-        if (!ok) break;
+      auto sQ = [&](int j) { return smem_u32(smem + C::OFF_Q + (j % C::NSQ) * C::TILE); };
+      auto sDO = [&](int j) { return smem_u32(smem + C::OFF_DO + (j % C::NSO) * C::TILE); };
+      auto wt = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, s_abort, p.wait_ns); };
+
+      auto mma_s = [&](int j) -> bool {
+        if (!wt(&bar_q_full[j % C::NSQ], (j / C::NSQ) & 1)) return false;
+        if (j > 0 && !wt(bar_dv_done, (j - 1) & 1)) return false;  // P^T(j-1) consumed
         tc_fence_after();
+        const uint32_t q = sQ(j);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          umma_ss(tmem + C::T_A, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idesc_t,
+          umma_ss(tmem + C::T_S, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q + off, 16, 1024), idesc_t,
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full);
-        if (it > 0 && !(ok = mbar_wait(bar_dq_free, (it - 1) & 1, s_abort, p.wait_ns))) break;
+        return true;
+      };
+      auto mma_dp = [&](int j) -> bool {
+        if (!wt(&bar_o_full[j % C::NSO], (j / C::NSO) & 1)) return false;
+        if (j > 0 && !wt(bar_dq_empty, (j - 1) & 1)) return false;  // dQ(j-1) read out
         tc_fence_after();
+        const uint32_t o = sDO(j);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          umma_ss(tmem + C::T_B, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sDO + off, 16, 1024), idesc_t,
+          umma_ss(tmem + C::T_DP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(o + off, 16, 1024), idesc_t,
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_dp_full);
-        if (!(ok = mbar_wait(bar_ds_ready, it & 1, s_abort, p.wait_ns))) break;
+        umma_commit(&bar_o_empty[j % C::NSO]);  // dV(j) was issued before dP(j)
+        return true;
+      };
+      auto mma_dv = [&](int j) -> bool {
+        if (!wt(bar_p_ready, j & 1)) return false;
+        if (!wt(&bar_o_full[j % C::NSO], (j / C::NSO) & 1)) return false;
         tc_fence_after();
-        // dQ first, so its read-out and atomics overlap the dV / dK MMAs.
+        const uint32_t o = sDO(j);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {  // dQ = dS K
-          umma_ss(tmem + C::T_B, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t a_col = C::T_S + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s P^T
+          umma_ts(tmem + C::T_DV, tmem + a_col, sdesc_sw128(o + kk * 2048, C::BOX, 1024), idesc_g,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_dv_done);
+        return true;
+      };
+      auto mma_dk = [&](int j) -> bool {
+        if (!wt(bar_ds_ready, j & 1)) return false;
+        tc_fence_after();
+        const uint32_t q = sQ(j);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t a_col = C::T_DP + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s dS^T
+          umma_ts(tmem + C::T_DK, tmem + a_col, sdesc_sw128(q + kk * 2048, C::BOX, 1024), idesc_g,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_dk_done);
+        umma_commit(&bar_q_empty[j % C::NSQ]);  // S(j) and dK(j) were Q's readers
+        return true;
+      };
+      auto mma_dq = [&](int j) -> bool {
+        if (!wt(bar_dk_done, j & 1)) return false;  // dQ overwrites the dS^T columns dK(j) reads
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
                   sdesc_sw128(sK + kk * 2048, C::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
-        }
         umma_commit(bar_dq_full);
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {  // dV += P^T dO ; dK += dS^T Q
-          const uint64_t bdo = sdesc_sw128(sDO + kk * 2048, C::BOX, 1024);
-          const uint64_t bq = sdesc_sw128(sQ + kk * 2048, C::BOX, 1024);
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t a_col = C::T_A + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s columns
-          umma_ts(tmem + C::T_DV, tmem + a_col, bdo, idesc_g, acc);
-          umma_ts(tmem + C::T_DK, tmem + a_col + 32, bq, idesc_g, acc);
-        }
-        umma_commit(bar_a_free);
-        umma_commit(&bar_q_empty[st]);
+        return true;
+      };
+
+      bool ok = wt(bar_kv_full, 0);
+      ok = ok && mma_s(0) && mma_dv(0) && mma_dp(0) && (NIT < 2 || mma_s(1));
+      for (int i = 0; i < NIT && ok; ++i) {
+        ok = mma_dk(i) && mma_dq(i);
+        if (ok && i + 1 < NIT) ok = mma_dv(i + 1) && mma_dp(i + 1);
+        if (ok && i + 2 < NIT) ok = mma_s(i + 2);
       }
-      if (!ok) record_failure(s_abort, p.err, SITE_BWD_MMA);
+      if (ok) umma_commit(bar_fin);
+      else record_failure(s_abort, p.err, SITE_BWD_MMA);
     }
-  } else {
-    // ------------------------------------------------- per-lane gradients
+  } else if (warp >= kWarpCompute0) {
+    // ------------------------------------------------- P^T and dS^T per key
     // Two warpgroups; warpgroup wg owns query columns [64 wg, 64 wg + 64) of
-    // every tile (and D columns [wg D/2, (wg+1) D/2) of dQ, dK, dV). Each
-    // writes its P^T / dS^T only into TMEM columns it alone has read:
-    // P^T of its columns at T_A + 64 wg, dS^T at T_A + 64 wg + 32.
-    const int wg = (warp - 2) >> 2;
+    // every tile (and D columns [wg D/2, (wg+1) D/2) of dK, dV at the end).
+    // Each writes P^T / dS^T only into TMEM columns it alone has read: P^T of
+    // its columns at T_S + 64 wg, dS^T at T_DP + 64 wg (bf16 pairs).
+    const int wg = (warp - kWarpCompute0) >> 2;
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // key row for S^T/dP^T/dK/dV, query row for dQ
+    const int row = quarter * 32 + lane;  // key row
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = row < k_rows;
     const long long my_kpos = key_ok ? kposat<SPLIT>(p, s, k0 + row) : k_max;
     const int my_seg = (SEG && key_ok) ? segat(p, s, k0 + row) : 0;
     const bool key_dead = !key_ok || my_kpos >= p.kv_valid || (my_seg & 1);  // odd segid: padding
     const float sl2 = p.scale_log2;
-    const int qc0 = wg * 64;              // first query column of this warpgroup
-    const uint32_t t_a = tmem + lane_base + C::T_A + wg * 64;
+    const int qc0 = wg * 64;  // first query column of this warpgroup
+    const uint32_t t_s = tmem + lane_base + C::T_S + qc0;
+    const uint32_t t_dp = tmem + lane_base + C::T_DP + qc0;
     uint8_t* sds = smem + C::OFF_DS + wg * C::BOX;
     bool ok = true;
     int it = 0;
     for (int hq = 0; hq < p.group && ok; ++hq) {
-    const int bh = kvh * p.group + hq;  // (batch, query head)
     for (int t = 0; t < p.nseg && ok; ++t) {
       const int r = (s + t) % p.nseg;
-      const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * q_len<SPLIT>(p);
       const int i_end = SEG ? s_hop[t].y : p.nq_tiles;
       for (int i = s_hop[t].x; i < i_end; ++i, ++it) {
         const int st = it % C::NSQ;
@@ -515,17 +589,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         first -= qc0;  // relative to this warpgroup's columns
         last -= qc0;
         uint32_t sr[2][32];
-        tmem_ld32(t_a, sr[0]);
-        tmem_ld32(t_a + 32, sr[1]);
+        tmem_ld32(t_s, sr[0]);
+        tmem_ld32(t_s + 32, sr[1]);
         tmem_wait_ld();
-        // P^T (fp32, kept in sr) and its bf16 copy into TMEM
-        {
-          uint32_t pk[32];
+        // P^T (fp32, kept in sr) and its bf16 copy over its scores, 32 query
+        // columns at a time
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c0 = 2 * e;
-            float a = ex2_approx(fmaf(__uint_as_float(sr[c0 >> 5][c0 & 31]), sl2, -lse2[c0]));
-            float b = ex2_approx(fmaf(__uint_as_float(sr[(c0 + 1) >> 5][(c0 + 1) & 31]), sl2, -lse2[c0 + 1]));
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = 32 * h + 2 * e;
+            float a = ex2_approx(fmaf(__uint_as_float(sr[h][2 * e]), sl2, -lse2[c0]));
+            float b = ex2_approx(fmaf(__uint_as_float(sr[h][2 * e + 1]), sl2, -lse2[c0 + 1]));
             if (SEG) {  // visible run [first, last)
               a = (c0 >= first && c0 < last) ? a : 0.f;
               b = (c0 + 1 >= first && c0 + 1 < last) ? b : 0.f;
@@ -533,40 +609,47 @@ __global__ void __launch_bounds__(kThreads, 1)
               a = c0 >= first ? a : 0.f;
               b = c0 + 1 >= first ? b : 0.f;
             }
-            sr[c0 >> 5][c0 & 31] = __float_as_uint(a);
-            sr[(c0 + 1) >> 5][(c0 + 1) & 31] = __float_as_uint(b);
+            sr[h][2 * e] = __float_as_uint(a);
+            sr[h][2 * e + 1] = __float_as_uint(b);
             pk[e] = pack_bf16x2(a, b);
           }
-          tmem_st32(t_a, pk);
+          tmem_st16(t_s + 16 * h, pk);
         }
-        if (!warp_wait(bar_dp_full, it & 1, s_abort, p.wait_ns)) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p_ready);  // one arrival per warp
+        // dS(j) goes into the shared tile that dQ(j-1) reads: wait for it.
+        if (!warp_wait(bar_dp_full, it & 1, s_abort, p.wait_ns) ||
+            (it > 0 && !warp_wait(bar_dq_full, (it - 1) & 1, s_abort, p.wait_ns))) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
           ok = false;
           break;
         }
         tc_fence_after();
-        // dS^T = P^T o (dP^T - Delta): bf16 into TMEM and into the swizzled
-        // shared tile read by the dQ MMA (box wg, row = key).
-        uint32_t dp[2][32];
-        tmem_ld32(tmem + lane_base + C::T_B + qc0, dp[0]);
-        tmem_ld32(tmem + lane_base + C::T_B + qc0 + 32, dp[1]);
-        tmem_wait_ld();
-
+        // dS^T = P^T o (dP^T - Delta): bf16 over this warpgroup's dP^T
+        // columns in TMEM (read by dK) and into the swizzled shared tile read
+        // by dQ (box wg, row = key), 16 query columns at a time (the packed
+        // pairs of chunk c land on columns already read).
+        uint8_t* rowp = sds + row * 128;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dp[16];
+          tmem_ld16(t_dp + c * 16, dp);
+          tmem_wait_ld();
+          uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int q0 = c * 32 + 2 * e;
-            const float a = __uint_as_float(sr[c][2 * e]) * (__uint_as_float(dp[c][2 * e]) - dlt[q0]);
-            const float b = __uint_as_float(sr[c][2 * e + 1]) * (__uint_as_float(dp[c][2 * e + 1]) - dlt[q0 + 1]);
+          for (int e = 0; e < 8; ++e) {
+            const int q0 = c * 16 + 2 * e;
+            const float a = __uint_as_float(sr[c >> 1][(c & 1) * 16 + 2 * e]) * (__uint_as_float(dp[2 * e]) - dlt[q0]);
+            const float b =
+                __uint_as_float(sr[c >> 1][(c & 1) * 16 + 2 * e + 1]) * (__uint_as_float(dp[2 * e + 1]) - dlt[q0 + 1]);
             pk[e] = pack_bf16x2(a, b);
           }
-          tmem_st16(t_a + 32 + c * 16, pk);
-          uint8_t* rowp = sds + row * 128;
+          tmem_st8(t_dp + c * 8, pk);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int chunk = c * 4 + j;
+          for (int j = 0; j < 2; ++j) {
+            const int chunk = c * 2 + j;
             *reinterpret_cast<uint4*>(rowp + ((chunk ^ (row & 7)) << 4)) =
                 make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
@@ -576,45 +659,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_ds_ready);  // one arrival per warp
-        // dQ read-out: this lane's query row, this warpgroup's half of D, in
-        // 32-column chunks, transposed within 8-lane groups by shuffles so
-        // that one warp instruction covers four whole 128-byte rows of the
-        // fp32 accumulator (coalesced vector reductions; no shared-memory
-        // round trip, whose bandwidth the MMAs need).
-        if (!warp_wait(bar_dq_full, it & 1, s_abort, p.wait_ns)) {
-          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        {
-          const int gi = lane >> 3, gj = lane & 7;
-          float* dst0 = p.dq_acc + (rowbase + static_cast<long long>(i) * BQ + quarter * 32 + gi * 8) * D +
-                        wg * (D / 2) + gj * 4;
-          const int rows_left = q_len<SPLIT>(p) - (i * BQ + quarter * 32 + gi * 8);
-          uint32_t g0[32], g1[32];
-          tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2), g0);
-          if constexpr (D == 128) tmem_ld32(tmem + lane_base + C::T_B + wg * (D / 2) + 32, g1);
-          tmem_wait_ld();
-          if constexpr (SPLIT) {  // the caller's accumulator holds dQ itself
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              g0[e] = __float_as_uint(__uint_as_float(g0[e]) * p.scale);
-              if constexpr (D == 128) g1[e] = __float_as_uint(__uint_as_float(g1[e]) * p.scale);
-            }
-          }
-          transpose_reduce<D>(g0, dst0, rows_left);
-          if constexpr (D == 128) transpose_reduce<D>(g1, dst0 + 32, rows_left);
-        }
-        if (!ok) break;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_dq_free);  // one arrival per warp
       }
     }
     }
     // ------------------------------------------------------ dK, dV out
-    if (ok && NIT > 0 && !warp_wait(bar_a_free, (NIT - 1) & 1, s_abort, p.wait_ns)) {
+    if (ok && NIT > 0 && !warp_wait(bar_fin, 0, s_abort, p.wait_ns)) {
       if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_EPILOGUE);
       ok = false;
     }
@@ -671,21 +720,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+  } else {
+    // ------------------------------------------------------ dQ read-out
+    // Warps 0..3, one thread per query row (TMEM lane): each dQ(j) is read
+    // out of TMEM in 32-column chunks (the dP^T columns are released as soon
+    // as the last chunk is in registers), staged in shared memory and added
+    // into the fp32 accumulator by TMA tile reduce-adds, which run on in the
+    // background while the next tiles are computed. One thread issues the
+    // copies; named barriers keep the warpgroup in step, and every decision
+    // to stop is taken together (so no thread is left at a barrier).
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // query row
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool elected = threadIdx.x == 0;
+    uint8_t* stg = smem + C::OFF_STG;
+    int n_staged = 0;
+    bool ok = NIT > 0;
+    int it = 0;
+    for (int hq = 0; hq < p.group && ok; ++hq) {
+    const int bh = kvh * p.group + hq;  // (batch, query head)
+    for (int t = 0; t < p.nseg && ok; ++t) {
+      const int r = (s + t) % p.nseg;
+      const int i_end = SEG ? s_hop[t].y : p.nq_tiles;
+      for (int i = s_hop[t].x; i < i_end; ++i, ++it) {
+        const bool got = mbar_wait(bar_dq_full, it & 1, s_abort, p.wait_ns);
+        if (bar_any(kReduceBar, 128, !got)) {
+          if (elected) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < C::NCH / 2; ++h) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_base + C::T_DP + (2 * h) * 32, v0);
+          tmem_ld32(tmem + lane_base + C::T_DP + (2 * h + 1) * 32, v1);
+          tmem_wait_ld();
+          if (h == C::NCH / 2 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_dq_empty);  // one arrival per warp
+          }
+          if constexpr (SPLIT) {  // the caller's accumulator holds dQ itself
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              v0[e] = __float_as_uint(__uint_as_float(v0[e]) * p.scale);
+              v1[e] = __float_as_uint(__uint_as_float(v1[e]) * p.scale);
+            }
+          }
+          stage_dq_chunk<D>(v0, stg + (n_staged % C::NSTG) * C::CHUNK, row, elected, n_staged >= C::NSTG, &tm_dq,
+                            (2 * h) * 32, i * BQ, r, bh);
+          ++n_staged;
+          stage_dq_chunk<D>(v1, stg + (n_staged % C::NSTG) * C::CHUNK, row, elected, n_staged >= C::NSTG, &tm_dq,
+                            (2 * h + 1) * 32, i * BQ, r, bh);
+          ++n_staged;
+        }
+      }
+    }
+    }
+    if (elected) bulk_wait_all();  // the staged chunks are read before shared memory goes away
   }
 
   // ------------------------------------------------------------ teardown
-  if (warp == 0 && lane == 0) {
+  if (warp == kWarpProducer && lane == 0) {
     if (kv_issued) drain_wait(bar_kv_full, 0);
     for (int it = max(0, issued_q - C::NSQ); it < issued_q; ++it)
       drain_wait(&bar_q_full[it % C::NSQ], (it / C::NSQ) & 1);
+    for (int it = max(0, issued_o - C::NSO); it < issued_o; ++it)
+      drain_wait(&bar_o_full[it % C::NSO], (it / C::NSO) & 1);
   }
-  if (warp == 1 && lane == 0 && NIT > 0) {
+  if (warp == kWarpMma && lane == 0 && NIT > 0) {
     umma_commit(bar_drain);
     if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::T_COLS);
@@ -754,18 +864,20 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   const long long grid = static_cast<long long>(a.BH / a.group) * a.nseg * nt;  // one CTA per key/value tile
   if (grid == 0) return RATTN_OK;
   if (grid > INT32_MAX) return RATTN_ERR_UNSUPPORTED;
-  bwd_prep_kernel<D, true><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
-      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
-  if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
-  CUtensorMap tq, tk, tv, tdo;
+  // Everything that can fail on the host comes before the first launch.
+  CUtensorMap tq, tk, tv, tdo, tdq;
   rattn_status st;
   if ((st = make_tmap_bf16(&tq, a.q, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tk, a.k, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
+  if ((st = make_tmap_f32_acc(&tdq, a.dq_acc, D, a.Lseg, a.nseg, a.BH)) != RATTN_OK) return st;
   const void* kfn = a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true, false>)
                          : reinterpret_cast<const void*>(&bwd_kernel<D, false, false>);
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
+  bwd_prep_kernel<D, true><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
+      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
+  if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   Params p;
   p.lse = a.lse;
   p.delta = a.delta;
@@ -785,15 +897,16 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.kv_valid = a.kv_valid;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.dq_acc = a.dq_acc;
   p.dk = a.dk;
   p.dv = a.dv;
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
   if (a.seg)
-    bwd_kernel<D, true, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+    bwd_kernel<D, true, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq,
+                                                                                              p);
   else
-    bwd_kernel<D, false, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+    bwd_kernel<D, false, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq,
+                                                                                               p);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   const long long n4 = rows * D / 4;
   dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
@@ -819,12 +932,13 @@ rattn_status launch_split(const PartialBwdArgs& a, const DevCtx& ctx) {
       return RATTN_ERR_CUDA;
     return RATTN_OK;
   }
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   rattn_status st;
   if ((st = make_tmap_bf16(&tq, a.q, D, a.Lq, 1, a.BH, BQ)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tk, a.k, D, a.Lk, 1, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lk, 1, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lq, 1, a.BH, BQ)) != RATTN_OK) return st;
+  if ((st = make_tmap_f32_acc(&tdq, a.dq_acc, D, a.Lq, 1, a.BH)) != RATTN_OK) return st;
   const void* kfn = reinterpret_cast<const void*>(&bwd_kernel<D, false, true>);
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
   Params p;
@@ -847,12 +961,11 @@ rattn_status launch_split(const PartialBwdArgs& a, const DevCtx& ctx) {
   p.kv_valid = a.kv_valid;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.dq_acc = a.dq_acc;
   p.dk = a.dk;
   p.dv = a.dv;
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
-  bwd_kernel<D, false, true><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, p);
+  bwd_kernel<D, false, true><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? RATTN_OK : RATTN_ERR_CUDA;
 }
 

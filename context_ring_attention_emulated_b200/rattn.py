@@ -42,6 +42,8 @@ SIGNATURES = [
     ("cp_layout_permute_rope", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _D, _I, _P]),
     ("cp_layout_unpermute_rope_grad", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _D, _I, _P]),
     ("rattn_partial_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I, _I, _F, _I, _I64, _P, _P, _P]),
+    ("rattn_partial_fwd_gqa", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I64, _I, _I, _F, _I, _I64, _P, _P,
+                                   _P]),
     ("rattn_merge", _I, [_P, _P, _P, _P, _I, _I, _I64, _I, _P]),
     ("rattn_ring_fwd", _I, [_P, _P, _P, _P, _I, _I, _I64, _I, _I, _I, _I, _I, _F, _I64, _P, _P, _P]),
     ("rattn_ring_bwd_workspace_size", ctypes.c_size_t, [_I, _I, _I64, _I]),
@@ -345,6 +347,28 @@ def rattn_partial_fwd(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True,
     _check("rattn_partial_fwd", lib.rattn_partial_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(q_pos), _ptr(kv_pos), B, H,
                                                        Lq, Lk, D, _dtype_code(q), float(scale), int(causal),
                                                        int(kv_valid), _ptr(o), _ptr(lse), _stream(stream)))
+    return o, lse
+
+
+def rattn_partial_fwd_gqa(q, k, v, q_pos=None, kv_pos=None, scale=None, causal=True, kv_valid=2**62,
+                          o=None, lse=None, stream=None):
+    """rattn_partial_fwd with k, v [B,H_kv,Lk,D] shared by groups of H / H_kv
+    query heads: returns (O fp32 [B,H,Lq,D], LSE fp32 [B,H,Lq])."""
+    B, H, Lq, D, H_kv, Lk = _attn(q, k, v, "rattn_partial_fwd_gqa", same_len=False)
+    _expect(q_pos, (Lq,), torch.int32, "q_pos")
+    _expect(kv_pos, (Lk,), torch.int32, "kv_pos")
+    _expect(o, (B, H, Lq, D), torch.float32, "o")
+    _expect(lse, (B, H, Lq), torch.float32, "lse")
+    _need_cuda(q, k, v, q_pos, kv_pos, o, lse)
+    scale = D ** -0.5 if scale is None else scale
+    if o is None:
+        o = torch.empty(B, H, Lq, D, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, H, Lq, dtype=torch.float32, device=q.device)
+    _check("rattn_partial_fwd_gqa", lib.rattn_partial_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(q_pos), _ptr(kv_pos),
+                                                               B, H, H_kv, Lq, Lk, D, _dtype_code(q), float(scale),
+                                                               int(causal), int(kv_valid), _ptr(o), _ptr(lse),
+                                                               _stream(stream)))
     return o, lse
 
 

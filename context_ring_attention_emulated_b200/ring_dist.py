@@ -52,7 +52,7 @@ Schedules (rank r of cp ranks; next = r+1, prev = r-1, mod cp):
                 ``reduce_scatter_tensor`` returns the sum for its own block.
 
 Block arithmetic. By default (``KernelOps``) every block runs on this library's
-kernels: ``rattn_partial_fwd`` and ``rattn_merge`` in the forward (O and LSE
+kernels: ``rattn_partial_fwd_gqa`` and ``rattn_merge`` in the forward (O and LSE
 come back in fp32, the fold's accumulator); ``rattn_bwd_prep`` (Delta and the
 zeroed fp32 dQ accumulator), ``rattn_partial_bwd`` (one block's dQ added in
 place, its dK, dV shares in fp32) and ``rattn_grad_fold`` (running sums) in
@@ -64,7 +64,17 @@ this module.
 With NCCL, set each process's device (``torch.cuda.set_device``) before the
 first call: batched point-to-point operations need it, and every rank of the
 group takes part in each exchange (all ranks call the same schedule with the
-same cp, shapes and dtypes).
+same cp, shapes and dtypes). A group whose backend moves only host memory
+(gloo) can still carry CUDA blocks: each exchange then copies the blocks it
+sends into pinned host buffers, moves those, and copies what arrives back to
+the device on the current stream when the exchange is waited for.
+
+Grouped key/value heads: K and V may have H_kv heads with H a multiple of
+H_kv (query head h reads key/value head h / (H / H_kv)); only the H_kv heads
+travel, which is what makes the ring's traffic O(L H_kv) in [Megatron-CP].
+
+Each hop's work is bracketed by an NVTX range ("rattn hop t") when the
+tensors are on a GPU, so a profiler's timeline shows the hops.
 
 Failure handling. Every exchange is a ``torch.distributed`` call on the
 caller's process group; give the group a short timeout so that a rank that
@@ -132,7 +142,7 @@ class KernelOps:
         self._r = rattn
 
     def fwd(self, q, k, v, q_pos, kv_pos, scale, causal, kv_valid):
-        return self._r.rattn_partial_fwd(q, k, v, q_pos, kv_pos, scale, causal, kv_valid)
+        return self._r.rattn_partial_fwd_gqa(q, k, v, q_pos, kv_pos, scale, causal, kv_valid)
 
     def merge(self, o_acc, lse_acc, o_blk, lse_blk):
         return self._r.rattn_merge(o_acc, lse_acc, o_blk, lse_blk)
@@ -172,25 +182,86 @@ def rank_slice(x, rank, cp):
 
 
 def _check_local(q, k, v, pos):
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
-        raise ValueError(f"q, k, v must share one [B, H, L_loc, D] shape, got {tuple(q.shape)}, "
-                         f"{tuple(k.shape)}, {tuple(v.shape)}")
-    if pos.dim() != 1 or pos.shape[0] != q.shape[2] or pos.dtype != torch.int32:
-        raise ValueError(f"pos must be int32 [L_loc = {q.shape[2]}], got {pos.dtype} {tuple(pos.shape)}")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError(f"q must be [B, H, L_loc, D] and k, v one [B, H_kv, L_loc, D] shape, got "
+                         f"{tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    B, H, L_loc, D = q.shape
+    H_kv = k.shape[1]
+    if k.shape[0] != B or k.shape[2] != L_loc or k.shape[3] != D or H_kv < 1 or H % H_kv:
+        raise ValueError(f"k, v must be [B={B}, H_kv, L_loc={L_loc}, D={D}] with H={H} a multiple of H_kv, "
+                         f"got {tuple(k.shape)}")
+    if pos.dim() != 1 or pos.shape[0] != L_loc or pos.dtype != torch.int32:
+        raise ValueError(f"pos must be int32 [L_loc = {L_loc}], got {pos.dtype} {tuple(pos.shape)}")
     for t in (q, k, v, pos):
         if not t.is_contiguous() or t.device != q.device:
             raise ValueError("q, k, v and pos must be contiguous and on one device")
 
 
+def _host_staged(group, tensors):
+    """True when the group's backend moves host memory only (gloo) and some of
+    the tensors live on a GPU: they then travel through pinned host copies."""
+    return dist.get_backend(group) == "gloo" and any(t.is_cuda for t in tensors)
+
+
+def _to_host(t):
+    """Pinned host copy of a device tensor, complete when this returns."""
+    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h.copy_(t)
+    return h
+
+
+def _wire(t):
+    """The bytes of a contiguous tensor, as the exchange moves them."""
+    return t.reshape(-1).view(torch.uint8)
+
+
+class _Exchange:
+    """One posted exchange: ``sends`` go to rank ``nxt`` and ``recvs`` are
+    filled from rank ``prv``; ``wait()`` completes it."""
+
+    def __init__(self, sends, recvs, nxt, prv, tag, group):
+        self.recvs = recvs
+        self.host_recvs = None
+        if _host_staged(group, list(sends) + list(recvs)):
+            sends = [_to_host(t) for t in sends]
+            self.host_recvs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in recvs]
+            recvs = self.host_recvs
+        self._keep = sends
+        ops = [dist.P2POp(dist.isend, _wire(t), nxt, group, tag) for t in sends]
+        ops += [dist.P2POp(dist.irecv, _wire(t), prv, group, tag) for t in recvs]
+        self.reqs = dist.batch_isend_irecv(ops)
+
+    def wait(self):
+        for r in self.reqs:
+            r.wait()
+        if self.host_recvs is not None:
+            for d, h in zip(self.recvs, self.host_recvs):
+                d.copy_(h, non_blocking=True)
+            self.host_recvs = None
+
+
 def _exchange(sends, recvs, nxt, prv, tag, group):
-    ops = [dist.P2POp(dist.isend, t, nxt, group, tag) for t in sends]
-    ops += [dist.P2POp(dist.irecv, t, prv, group, tag) for t in recvs]
-    return dist.batch_isend_irecv(ops)
+    return _Exchange(sends, recvs, nxt, prv, tag, group)
 
 
 def _wait(reqs):
     for r in reqs:
         r.wait()
+
+
+class _hop:
+    """NVTX range around one hop's work when the tensors are on a GPU."""
+
+    def __init__(self, t, on_gpu):
+        self.t, self.on_gpu = t, on_gpu
+
+    def __enter__(self):
+        if self.on_gpu:
+            torch.cuda.nvtx.range_push(f"rattn hop {self.t}")
+
+    def __exit__(self, *a):
+        if self.on_gpu:
+            torch.cuda.nvtx.range_pop()
 
 
 def _scale(q, scale):
@@ -213,18 +284,19 @@ def ring_fwd(q, k, v, pos, scale=None, causal=True, kv_valid=2 ** 62, group=None
     cur = [k, v, pos]
     o = lse = None
     for t in range(cp):
-        reqs = None
-        if t < cp - 1:
-            recv = bufs[t % 2]
-            reqs = _exchange(cur, recv, nxt, prv, _TAG_KV, group)
-        ob, lb = ops.fwd(q, cur[0], cur[1], pos, cur[2], scale, causal, kv_valid)
-        if o is None:
-            o, lse = ob, lb
-        else:
-            o, lse = ops.merge(o, lse, ob, lb)
-        if reqs is not None:
-            _wait(reqs)
-            cur = recv
+        with _hop(t, q.is_cuda):
+            xch = None
+            if t < cp - 1:
+                recv = bufs[t % 2]
+                xch = _exchange(cur, recv, nxt, prv, _TAG_KV, group)
+            ob, lb = ops.fwd(q, cur[0], cur[1], pos, cur[2], scale, causal, kv_valid)
+            if o is None:
+                o, lse = ob, lb
+            else:
+                o, lse = ops.merge(o, lse, ob, lb)
+            if xch is not None:
+                xch.wait()
+                cur = recv
     return o, lse
 
 
@@ -248,38 +320,63 @@ def ring_bwd(q, k, v, o, do, lse, pos, scale=None, causal=True, kv_valid=2 ** 62
     in_bufs = [None, None]         # running sums received for the next hop
     pending = None                 # the dK/dV exchange posted at the end of the previous hop
     for t in range(cp):
-        kv_reqs = None
-        if t < cp - 1:
-            recv = kv_bufs[t % 2]
-            kv_reqs = _exchange(cur, recv, nxt, prv, _TAG_KV, group)
-        # the buffers of hop t-2, whose send completed at hop t-1's wait
-        reuse = shares[t % 2] if shares[t % 2] is not None else (None, None)
-        gk, gv = ops.bwd(q, cur[0], cur[1], do, lse, delta, pos, cur[2], scale, causal, kv_valid, dq, *reuse)
-        if pending is not None:
-            _wait(pending)
-            dk_in, dv_in = in_bufs[(t - 1) % 2]
-            ops.fold(gk, dk_in)
-            ops.fold(gv, dv_in)
-        shares[t % 2] = (gk, gv)
-        if cp > 1:
-            if in_bufs[t % 2] is None:
-                in_bufs[t % 2] = (torch.empty_like(gk), torch.empty_like(gv))
-            pending = _exchange([gk, gv], list(in_bufs[t % 2]), nxt, prv, _TAG_DKV, group)
-        if kv_reqs is not None:
-            _wait(kv_reqs)
-            cur = recv
+        with _hop(t, q.is_cuda):
+            kv_xch = None
+            if t < cp - 1:
+                recv = kv_bufs[t % 2]
+                kv_xch = _exchange(cur, recv, nxt, prv, _TAG_KV, group)
+            # the buffers of hop t-2, whose send completed at hop t-1's wait
+            reuse = shares[t % 2] if shares[t % 2] is not None else (None, None)
+            gk, gv = ops.bwd(q, cur[0], cur[1], do, lse, delta, pos, cur[2], scale, causal, kv_valid, dq, *reuse)
+            if pending is not None:
+                pending.wait()
+                dk_in, dv_in = in_bufs[(t - 1) % 2]
+                ops.fold(gk, dk_in)
+                ops.fold(gv, dv_in)
+            shares[t % 2] = (gk, gv)
+            if cp > 1:
+                if in_bufs[t % 2] is None:
+                    in_bufs[t % 2] = (torch.empty_like(gk), torch.empty_like(gv))
+                pending = _exchange([gk, gv], list(in_bufs[t % 2]), nxt, prv, _TAG_DKV, group)
+            if kv_xch is not None:
+                kv_xch.wait()
+                cur = recv
     if cp == 1:
         return (dq,) + shares[0]
-    _wait(pending)
+    pending.wait()
     dk, dv = in_bufs[(cp - 1) % 2]
     return dq, dk, dv
 
 
-def _gather(x, cp, group):
-    out = torch.empty((cp,) + tuple(x.shape), dtype=x.dtype, device=x.device)
-    flat = out.view((cp * x.shape[0],) + tuple(x.shape[1:])) if x.dim() > 0 else out
-    work = dist.all_gather_into_tensor(flat, x, group=group, async_op=True)
-    return out, work
+class _Gather:
+    """All ranks' copies of ``x`` stacked as [cp, *x.shape], gathered
+    asynchronously; ``wait()`` completes it (host-staged on gloo)."""
+
+    def __init__(self, x, cp, group):
+        self.out = torch.empty((cp,) + tuple(x.shape), dtype=x.dtype, device=x.device)
+        self.host = None
+        src, dst = x, self.out
+        if _host_staged(group, [x]):
+            src = _to_host(x)
+            self.host = dst = torch.empty(self.out.shape, dtype=x.dtype, pin_memory=True)
+        self.work = dist.all_gather_into_tensor(_wire(dst), _wire(src), group=group, async_op=True)
+        self._keep = src
+
+    def wait(self):
+        self.work.wait()
+        if self.host is not None:
+            self.out.copy_(self.host, non_blocking=True)
+            self.host = None
+
+
+def _reduce_scatter(out, full, group):
+    """out = this rank's block of the sum over ranks of ``full`` [cp * n, ...]."""
+    if _host_staged(group, [out, full]):
+        h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dist.reduce_scatter_tensor(h, _to_host(full), group=group)
+        out.copy_(h, non_blocking=True)
+    else:
+        dist.reduce_scatter_tensor(out, full, group=group)
 
 
 def allgather_fwd(q, k, v, pos, scale=None, causal=True, kv_valid=2 ** 62, group=None, ops=None):
@@ -293,13 +390,16 @@ def allgather_fwd(q, k, v, pos, scale=None, causal=True, kv_valid=2 ** 62, group
     rank, cp, _, _ = ring_peers(group)
     if cp == 1:
         return ops.fwd(q, k, v, pos, pos, scale, causal, kv_valid)
-    (kg, wk), (vg, wv), (pg, wp) = (_gather(t, cp, group) for t in (k, v, pos))
-    o, lse = ops.fwd(q, k, v, pos, pos, scale, causal, kv_valid)
-    _wait([wk, wv, wp])
+    gathers = [_Gather(t, cp, group) for t in (k, v, pos)]
+    with _hop(0, q.is_cuda):
+        o, lse = ops.fwd(q, k, v, pos, pos, scale, causal, kv_valid)
+    _wait(gathers)
+    kg, vg, pg = (g.out for g in gathers)
     for t in range(1, cp):
         s = (rank - t) % cp
-        ob, lb = ops.fwd(q, kg[s], vg[s], pos, pg[s], scale, causal, kv_valid)
-        o, lse = ops.merge(o, lse, ob, lb)
+        with _hop(t, q.is_cuda):
+            ob, lb = ops.fwd(q, kg[s], vg[s], pos, pg[s], scale, causal, kv_valid)
+            o, lse = ops.merge(o, lse, ob, lb)
     return o, lse
 
 
@@ -315,15 +415,18 @@ def allgather_bwd(q, k, v, o, do, lse, pos, scale=None, causal=True, kv_valid=2 
     delta, dq = ops.prep(o, do)
     if cp == 1:
         return (dq,) + tuple(ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid, dq))
-    (kg, wk), (vg, wv), (pg, wp) = (_gather(t, cp, group) for t in (k, v, pos))
+    gathers = [_Gather(t, cp, group) for t in (k, v, pos)]
     dkg = torch.empty((cp,) + tuple(k.shape), dtype=dq.dtype, device=dq.device)   # every block's shares
     dvg = torch.empty_like(dkg)
-    ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid, dq, dkg[rank], dvg[rank])
-    _wait([wk, wv, wp])
+    with _hop(0, q.is_cuda):
+        ops.bwd(q, k, v, do, lse, delta, pos, pos, scale, causal, kv_valid, dq, dkg[rank], dvg[rank])
+    _wait(gathers)
+    kg, vg, pg = (g.out for g in gathers)
     for t in range(1, cp):
         s = (rank - t) % cp
-        ops.bwd(q, kg[s], vg[s], do, lse, delta, pos, pg[s], scale, causal, kv_valid, dq, dkg[s], dvg[s])
+        with _hop(t, q.is_cuda):
+            ops.bwd(q, kg[s], vg[s], do, lse, delta, pos, pg[s], scale, causal, kv_valid, dq, dkg[s], dvg[s])
     dk, dv = torch.empty_like(dkg[0]), torch.empty_like(dvg[0])
     for out, full in ((dk, dkg), (dv, dvg)):
-        dist.reduce_scatter_tensor(out, full.view((cp * out.shape[0],) + tuple(out.shape[1:])), group=group)
+        _reduce_scatter(out, full.view((cp * out.shape[0],) + tuple(out.shape[1:])), group)
     return dq, dk, dv

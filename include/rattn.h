@@ -212,6 +212,17 @@ rattn_status rattn_partial_fwd(const void* q, const void* k, const void* v,
                                rattn_dtype dtype, float scale, int causal, int64_t kv_valid,
                                float* o, float* lse, void* stream);
 
+/* rattn_partial_fwd with grouped key/value heads ([Megatron-CP] "CP vs SP"
+ * sizes the ring's K/V traffic by the key/value heads): k and v are
+ * [B,H_kv,Lk,D] with H a multiple of H_kv, and query head h reads key/value
+ * head h / (H / H_kv). Otherwise as rattn_partial_fwd; H_kv == H is that
+ * call. RATTN_ERR_INVALID_ARG when H_kv < 1 or H % H_kv != 0. */
+rattn_status rattn_partial_fwd_gqa(const void* q, const void* k, const void* v,
+                                   const int32_t* q_pos, const int32_t* kv_pos,
+                                   int B, int H, int H_kv, int64_t Lq, int64_t Lk, int D,
+                                   rattn_dtype dtype, float scale, int causal, int64_t kv_valid,
+                                   float* o, float* lse, void* stream);
+
 /* [Ring-page] "Technical insight": online-softmax fold of a block result into
  * an accumulator, in place, fp32:
  *   LSE' = m + log(exp(LSE_acc - m) + exp(LSE_blk - m)),  m = max(LSE_acc, LSE_blk)

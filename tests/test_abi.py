@@ -147,6 +147,12 @@ def test_attention_calls_reject_bad_arguments(rattn):
     assert part(o=MIS) == rattn.ERR_INVALID_ARG
     assert part(D=80) == rattn.ERR_UNSUPPORTED
     assert part(Lq=0) == rattn.OK
+    gqa = lambda H, H_kv, Lq=8: L.rattn_partial_fwd_gqa(FAKE, FAKE, FAKE, None, None, 1, H, H_kv, Lq, 8, 64, 1,
+                                                         ctypes.c_float(0.1), 1, 1 << 40, FAKE, FAKE, None)
+    assert gqa(4, 3) == rattn.ERR_INVALID_ARG            # H not a multiple of H_kv
+    assert gqa(4, 0) == rattn.ERR_INVALID_ARG
+    assert gqa(4, 8) == rattn.ERR_INVALID_ARG
+    assert gqa(8, 2, Lq=0) == rattn.OK
     assert L.rattn_merge(FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 6, None) == rattn.ERR_INVALID_ARG
     assert L.rattn_merge(MIS, FAKE, FAKE, FAKE, 1, 1, 4, 8, None) == rattn.ERR_INVALID_ARG
     assert L.rattn_merge(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 8, None) == rattn.OK

@@ -28,8 +28,9 @@ class OracleOps:
     only), with the interface of ``ring_dist.KernelOps``."""
 
     def fwd(self, q, k, v, q_pos, kv_pos, scale, causal, kv_valid):
-        o, lse = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale, causal, q_pos.numpy(), kv_pos.numpy(),
-                                  kv_valid)
+        H = q.shape[1]
+        k, v = (oracle.gqa_expand(x.numpy(), H) for x in (k, v))
+        o, lse = oracle.attention(q.numpy(), k, v, scale, causal, q_pos.numpy(), kv_pos.numpy(), kv_valid)
         return torch.from_numpy(o), torch.from_numpy(lse)
 
     def merge(self, o_acc, lse_acc, o_blk, lse_blk):
@@ -41,9 +42,12 @@ class OracleOps:
         return delta, torch.zeros(do.shape, dtype=torch.float64)
 
     def bwd(self, q, k, v, do, lse, delta, q_pos, kv_pos, scale, causal, kv_valid, dq_acc, dk=None, dv=None):
-        gq, gk, gv = (torch.from_numpy(np.ascontiguousarray(x)) for x in oracle.attention_bwd_block(
-            q.numpy(), k.numpy(), v.numpy(), do.numpy(), lse.numpy(), delta.numpy(), scale, causal, q_pos.numpy(),
-            kv_pos.numpy(), kv_valid))
+        H, H_kv = q.shape[1], k.shape[1]
+        ke, ve = (oracle.gqa_expand(x.numpy(), H) for x in (k, v))
+        gq, gk, gv = oracle.attention_bwd_block(q.numpy(), ke, ve, do.numpy(), lse.numpy(), delta.numpy(), scale,
+                                                causal, q_pos.numpy(), kv_pos.numpy(), kv_valid)
+        gk, gv = oracle.gqa_reduce(gk, H_kv), oracle.gqa_reduce(gv, H_kv)
+        gq, gk, gv = (torch.from_numpy(np.ascontiguousarray(x)) for x in (gq, gk, gv))
         dq_acc += gq
         if dk is None:
             return gk, gv
@@ -137,6 +141,61 @@ def test_ring_and_allgather_match_full_attention(world):
         for j, ref in enumerate((dq_ref, dk_ref, dv_ref)):
             ag = _assemble([x["ag"][j] for x in ranks], L, world, layout)
             np.testing.assert_allclose(ag, ref, rtol=0, atol=1e-12)
+
+
+GQA_HEADS = ((4, 2), (4, 1))   # (H, H_kv)
+
+
+def _gqa_inputs(L, H, H_kv, seed):
+    g = np.random.default_rng(seed)
+    shapes = ((B, H, L, D), (B, H_kv, L, D), (B, H_kv, L, D), (B, H, L, D))
+    return [g.standard_normal(s) for s in shapes]
+
+
+def _gqa_main(rank, world, port, out):
+    """The ring and all-gather schedules with K, V on fewer heads than Q: only
+    the H_kv heads travel, and dK, dV come back summed over each group."""
+    _init(rank, world, port)
+    ops = OracleOps()
+    try:
+        for i, (H, H_kv) in enumerate(GQA_HEADS):
+            L = 6 * world - 1
+            q, k, v, do = _gqa_inputs(L, H, H_kv, 300 + 10 * world + i)
+            _, _, pos = oracle.perm_index(L, world, oracle.HEAD_TAIL)
+            qp, kp, vp, dop = (torch.from_numpy(oracle.permute(x, world, oracle.HEAD_TAIL)[0]) for x in (q, k, v, do))
+            pl = ring_dist.rank_slice(torch.from_numpy(np.asarray(pos, dtype=np.int32)), rank, world)
+            ql, kl, vl, dol = (ring_dist.rank_slice(x, rank, world) for x in (qp, kp, vp, dop))
+            o, lse = ring_dist.ring_fwd(ql, kl, vl, pl, SCALE, True, L, ops=ops)
+            dq, dk, dv = ring_dist.ring_bwd(ql, kl, vl, o, dol, lse, pl, SCALE, True, L, ops=ops)
+            g2 = ring_dist.allgather_bwd(ql, kl, vl, o, dol, lse, pl, SCALE, True, L, ops=ops)
+            out[(rank, i)] = dict(o=o.numpy(), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy(),
+                                  ag=[x.numpy() for x in g2])
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_ring_carries_grouped_kv_heads(world):
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_gqa_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for i, (H, H_kv) in enumerate(GQA_HEADS):
+        L = 6 * world - 1
+        q, k, v, do = _gqa_inputs(L, H, H_kv, 300 + 10 * world + i)
+        ke, ve = oracle.gqa_expand(k, H), oracle.gqa_expand(v, H)
+        o_ref, _ = oracle.attention(q, ke, ve, SCALE, True)
+        dq_ref, dke, dve = oracle.attention_bwd(q, ke, ve, do, SCALE, True)
+        refs = {"dq": dq_ref, "dk": oracle.gqa_reduce(dke, H_kv), "dv": oracle.gqa_reduce(dve, H_kv)}
+        ranks = [res[(r, i)] for r in range(world)]
+        get = lambda name: _assemble([x[name] for x in ranks], L, world, oracle.HEAD_TAIL)
+        np.testing.assert_allclose(get("o"), o_ref, rtol=0, atol=1e-12)
+        for name, ref in refs.items():
+            np.testing.assert_allclose(get(name), ref, rtol=0, atol=1e-12, err_msg=f"{name} H={H} H_kv={H_kv}")
+        for j, name in enumerate(("dq", "dk", "dv")):
+            ag = _assemble([x["ag"][j] for x in ranks], L, world, oracle.HEAD_TAIL)
+            np.testing.assert_allclose(ag, refs[name], rtol=0, atol=1e-12)
 
 
 def _subgroup_main(rank, world, port, out):
