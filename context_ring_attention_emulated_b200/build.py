@@ -1,6 +1,11 @@
 """Builds librattn.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-Usage: python -m context_ring_attention_emulated_b200.build [-v]
+Usage: python -m context_ring_attention_emulated_b200.build [-v] [--debug]
+
+--debug builds librattn_debug.so instead: the same sources with RATTN_DEBUG
+defined, which adds device-side bounds checks to the attention kernels
+(failures are reported through rattn_get_device_error as RATTN_ERR_BOUNDS).
+The Python binding loads it when RATTN_DEBUG=1 is set.
 """
 import concurrent.futures
 import glob
@@ -13,6 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "librattn.so")
+OBJ_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "librattn_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -20,13 +27,13 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxe
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]
 
 
-def _compile(src, verbose):
-    obj = os.path.join(OBJ, os.path.basename(src).replace(".cu", ".o"))
+def _compile(src, verbose, debug=False):
+    obj = os.path.join(OBJ_DEBUG if debug else OBJ, os.path.basename(src).replace(".cu", ".o"))
     deps = [src] + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(ROOT, "include", "*.h"))
     if os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(d) for d in deps):
         return obj, ""
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+    cmd = [NVCC, *ARCH, *FLAGS, *(["-DRATTN_DEBUG"] if debug else []), "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -35,24 +42,25 @@ def _compile(src, verbose):
     return obj, r.stdout + r.stderr
 
 
-def build(verbose=False):
-    os.makedirs(OBJ, exist_ok=True)
+def build(verbose=False, debug=False):
+    obj_dir, lib = (OBJ_DEBUG, LIB_DEBUG) if debug else (OBJ, LIB)
+    os.makedirs(obj_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose), srcs))
+        results = list(ex.map(lambda s: _compile(s, verbose, debug), srcs))
     objs = [o for o, _ in results]
     if verbose:
         for o, log in results:
             if log:
                 print(f"== {os.path.basename(o)}\n{log}")
     newest = max(os.path.getmtime(o) for o in objs)
-    if not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs]
+    if not os.path.exists(lib) or os.path.getmtime(lib) < newest:
+        cmd = [NVCC, *ARCH, "-shared", "-o", lib, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, debug="--debug" in sys.argv))

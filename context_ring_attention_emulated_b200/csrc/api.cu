@@ -139,6 +139,7 @@ const char* rattn_status_string(rattn_status s) {
     case RATTN_ERR_UNSUPPORTED: return "RATTN_ERR_UNSUPPORTED";
     case RATTN_ERR_CUDA: return "RATTN_ERR_CUDA";
     case RATTN_ERR_TIMEOUT: return "RATTN_ERR_TIMEOUT";
+    case RATTN_ERR_BOUNDS: return "RATTN_ERR_BOUNDS";
   }
   return "RATTN_ERR_UNKNOWN";
 }
@@ -575,7 +576,7 @@ rattn_status rattn_get_device_error(int* site) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return RATTN_ERR_CUDA;
-    return RATTN_ERR_TIMEOUT;
+    return v >= SITE_BOUNDS ? RATTN_ERR_BOUNDS : RATTN_ERR_TIMEOUT;
   }
   return RATTN_OK;
 }

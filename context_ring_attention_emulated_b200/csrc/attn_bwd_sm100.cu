@@ -45,6 +45,7 @@
 #include <limits.h>
 #include <math.h>
 
+#include "debug_check.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -116,11 +117,15 @@ struct Params {
 };
 
 __device__ __forceinline__ int segat(const Params& p, int rank, int row) {
-  return __ldg(p.seg + static_cast<long long>(rank) * p.Lseg + row);
+  const long long i = static_cast<long long>(rank) * p.Lseg + row;
+  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lseg, p.err, 11)) return 1;
+  return __ldg(p.seg + i);
 }
 
 __device__ __forceinline__ long long posat(const Params& p, int seg, int row) {
-  return static_cast<long long>(__ldg(p.pos + static_cast<long long>(seg) * p.Lseg + row));
+  const long long i = static_cast<long long>(seg) * p.Lseg + row;
+  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lseg, p.err, 12)) return 0;
+  return static_cast<long long>(__ldg(p.pos + i));
 }
 
 // Query-side and key-side lengths and positions: one array of Lseg rows per
@@ -137,14 +142,24 @@ __device__ __forceinline__ int k_len(const Params& p) {
 
 template <bool SPLIT>
 __device__ __forceinline__ long long qposat(const Params& p, int seg, int row) {
-  if constexpr (SPLIT) return static_cast<long long>(__ldg(p.q_pos + static_cast<long long>(seg) * p.Lq + row));
-  else return posat(p, seg, row);
+  if constexpr (SPLIT) {
+    const long long i = static_cast<long long>(seg) * p.Lq + row;
+    if (!in_bounds(i, p.Lq, p.err, 13)) return 0;
+    return static_cast<long long>(__ldg(p.q_pos + i));
+  } else {
+    return posat(p, seg, row);
+  }
 }
 
 template <bool SPLIT>
 __device__ __forceinline__ long long kposat(const Params& p, int seg, int row) {
-  if constexpr (SPLIT) return static_cast<long long>(__ldg(p.kv_pos + static_cast<long long>(seg) * p.Lk + row));
-  else return posat(p, seg, row);
+  if constexpr (SPLIT) {
+    const long long i = static_cast<long long>(seg) * p.Lk + row;
+    if (!in_bounds(i, p.Lk, p.err, 14)) return 0;
+    return static_cast<long long>(__ldg(p.kv_pos + i));
+  } else {
+    return posat(p, seg, row);
+  }
 }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -350,10 +365,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const long long rowbase = (static_cast<long long>(bh) * p.nseg + r) * q_len<SPLIT>(p);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = lane * 4 + e;
+            const int c = e * 32 + lane;  // coalesced loads, conflict-free stores
             const int q = i * BQ + c;
             float l2 = INFINITY, dl = 0.f;
-            if (q < q_len<SPLIT>(p)) {
+            if (q < q_len<SPLIT>(p) &&
+                in_bounds(rowbase + q, static_cast<long long>(p.BH) * p.nseg * q_len<SPLIT>(p), p.err, 15)) {
               const float l = __ldg(p.lse + rowbase + q);
               l2 = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
               dl = __ldg(p.delta + rowbase + q);
@@ -509,6 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = row < k_rows;
     const long long my_kpos = key_ok ? kposat<SPLIT>(p, s, k0 + row) : k_max;
+    if (kDebugChecks && wg == 0 && key_ok && k0 + row > 0)
+      check_order(kposat<SPLIT>(p, s, k0 + row - 1) <= my_kpos, p.err, 18);
     const int my_seg = (SEG && key_ok) ? segat(p, s, k0 + row) : 0;
     const bool key_dead = !key_ok || my_kpos >= p.kv_valid || (my_seg & 1);  // odd segid: padding
     const float sl2 = p.scale_log2;
@@ -526,23 +544,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = it % C::NSQ;
         const float* lse2 = s_lse + st * 128 + qc0;
         const float* dlt = s_delta + st * 128 + qc0;
-        // Query columns of this tile that see this key: [first, last).
-        // Without packed sequences the hop table says which tiles need a
-        // search, which then runs per thread before the wait for the tile's
-        // scores; packed, the tile's query positions and segids are spread
-        // over the warp (four per lane) and searched through shuffles (all
-        // lanes, eight steps) once the tile's flag is known.
+        // Query columns of this tile that see this key: [first, last). The
+        // tile's query positions (and segids when packed) are spread over
+        // the warp, four per lane, read with one coalesced load before the
+        // wait for the tile's scores; every lane then finds its key's bounds
+        // by binary search through shuffles (eight steps cover 128 queries;
+        // all lanes take every step). Only tiles with a masked element need
+        // it: without packed sequences the hop table says which, packed the
+        // producer's flag does.
         int first = 0, last = BQ;
-        auto search = [&]() {
-          const int n = min(BQ, q_len<SPLIT>(p) - i * BQ);
+        const int n = min(BQ, q_len<SPLIT>(p) - i * BQ);
+        int qp4[4], qs4[4];
+        auto load_tile_keys = [&]() {
           const long long qbase = static_cast<long long>(r) * q_len<SPLIT>(p) + i * BQ;
-          int qp4[4], qs4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int idx = 4 * lane + e;
-            qp4[e] = idx < n ? __ldg((SPLIT ? p.q_pos : p.pos) + qbase + idx) : INT_MAX;
-            qs4[e] = (SEG && idx < n) ? __ldg(p.seg + qbase + idx) : INT_MAX;
+            const bool inb = idx < n && in_bounds(qbase + idx, static_cast<long long>(p.nseg) * q_len<SPLIT>(p), p.err, 16);
+            qp4[e] = inb ? __ldg((SPLIT ? p.q_pos : p.pos) + qbase + idx) : INT_MAX;
+            qs4[e] = (SEG && inb) ? __ldg(p.seg + qbase + idx) : INT_MAX;
           }
+        };
+        auto search = [&]() {
           int lo = 0, hi = n;
 #pragma unroll 1
           for (int step = 0; step < 8; ++step) {  // first query at or after this key (same sequence when packed)
@@ -568,23 +591,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             last = lo;
           }
         };
-        if (!SEG && !key_dead && i < s_hop[t].y) {
-          // first query column at or after this key (the visible suffix)
-          int lo = 0, hi = min(BQ, q_len<SPLIT>(p) - i * BQ);
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (qposat<SPLIT>(p, r, i * BQ + mid) >= my_kpos) hi = mid; else lo = mid + 1;
-          }
-          first = lo;
+        // Without packed sequences only tiles before the hop table's y hold
+        // masked elements (the same for the whole warp).
+        const bool unpacked_masked = !SEG && i < s_hop[t].y;
+        if (unpacked_masked) load_tile_keys();
+        if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns)) {
+          if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
+          ok = false;
+          break;
         }
-        if (!warp_wait(&bar_q_full[st], (it / C::NSQ) & 1, s_abort, p.wait_ns) ||
-            !warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
+        const bool packed_masked = SEG && !s_full[st];  // the same for the whole warp
+        if (packed_masked) load_tile_keys();
+        if (!warp_wait(bar_s_full, it & 1, s_abort, p.wait_ns)) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
           ok = false;
           break;
         }
         tc_fence_after();
-        if (SEG && !s_full[st]) search();  // the same for the whole warp
+        if (unpacked_masked || packed_masked) search();
         if (key_dead) first = BQ;
         first -= qc0;  // relative to this warpgroup's columns
         last -= qc0;
@@ -670,6 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       if (NIT > 0) tc_fence_after();
       const long long krow = (static_cast<long long>(kvh) * p.nseg + s) * k_len<SPLIT>(p) + k0 + row;
+      const bool out_ok =
+          !key_ok || in_bounds(krow, static_cast<long long>(p.BH / p.group) * p.nseg * k_len<SPLIT>(p), p.err, 17);
       __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + krow * D + wg * (D / 2);
       __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + krow * D + wg * (D / 2);
       float* dk32 = static_cast<float*>(p.dk) + krow * D + wg * (D / 2);
@@ -685,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) gk[e] = gv[e] = 0u;
         }
-        if (SPLIT && key_ok) {  // fp32 shares, written or added (this thread owns these elements)
+        if (SPLIT && key_ok && out_ok) {  // fp32 shares, written or added (this thread owns these elements)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             float4 wk = make_float4(__uint_as_float(gk[4 * e + 0]) * p.scale, __uint_as_float(gk[4 * e + 1]) * p.scale,
@@ -702,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *pk = wk;
             *pv = wv;
           }
-        } else if (key_ok) {
+        } else if (key_ok && out_ok) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             uint4 wk, wv;

@@ -37,6 +37,7 @@
 #include <limits.h>
 #include <math.h>
 
+#include "debug_check.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -84,15 +85,21 @@ struct Params {
 };
 
 __device__ __forceinline__ long long qpos(const Params& p, int seg, int row) {
-  return p.q_pos ? static_cast<long long>(__ldg(p.q_pos + static_cast<long long>(seg) * p.Lq_seg + row)) : row;
+  const long long i = static_cast<long long>(seg) * p.Lq_seg + row;
+  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lq_seg, p.err, 1)) return 0;
+  return p.q_pos ? static_cast<long long>(__ldg(p.q_pos + i)) : row;
 }
 __device__ __forceinline__ long long kpos(const Params& p, int seg, int row) {
-  return p.kv_pos ? static_cast<long long>(__ldg(p.kv_pos + static_cast<long long>(seg) * p.Lk_seg + row)) : row;
+  const long long i = static_cast<long long>(seg) * p.Lk_seg + row;
+  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lk_seg, p.err, 2)) return 0;
+  return p.kv_pos ? static_cast<long long>(__ldg(p.kv_pos + i)) : row;
 }
 // segid of a slot (packed sequences; only called when p.seg is set). Query and
 // key slots share one array (rank-major, Lq_seg == Lk_seg in ring calls).
 __device__ __forceinline__ int segat(const Params& p, int rank, int row) {
-  return __ldg(p.seg + static_cast<long long>(rank) * p.Lk_seg + row);
+  const long long i = static_cast<long long>(rank) * p.Lk_seg + row;
+  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lk_seg, p.err, 3)) return 1;
+  return __ldg(p.seg + i);
 }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -351,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool row_valid = row < q_rows;
     const long long my_pos = row_valid ? qpos(p, r, q0 + row) : q_max;
+    if (kDebugChecks && row_valid && q0 + row > 0) check_order(qpos(p, r, q0 + row - 1) <= my_pos, p.err, 6);
     const int my_seg = (SEG && row_valid) ? segat(p, r, q0 + row) : 1;  // odd: sees nothing
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
@@ -384,8 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int idx = 4 * lane + e;
-            kp4[e] = idx < n ? (p.kv_pos ? __ldg(p.kv_pos + kbase + idx) : j * BN + idx) : INT_MAX;
-            ks4[e] = (SEG && idx < n) ? __ldg(p.seg + kbase + idx) : INT_MAX;
+            const bool inb = idx < n && in_bounds(kbase + idx, static_cast<long long>(p.nseg) * p.Lk_seg, p.err, 4);
+            kp4[e] = inb ? (p.kv_pos ? __ldg(p.kv_pos + kbase + idx) : j * BN + idx) : INT_MAX;
+            ks4[e] = (SEG && inb) ? __ldg(p.seg + kbase + idx) : INT_MAX;
           }
           int klo = 0;
           if (SEG) {
@@ -487,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------- epilogue
     const long long out_row = (static_cast<long long>(bh) * p.nseg + r) * p.Lq_seg + q0 + row;
+    const bool out_ok = !row_valid || in_bounds(out_row, static_cast<long long>(p.BH) * p.nseg * p.Lq_seg, p.err, 5);
     const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
     if (ok && G > 0) {
       if (!warp_wait(&bar_o_done[(G - 1) % C::NSB], ((G - 1) / C::NSB) & 1, s_abort, p.wait_ns)) {
@@ -507,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) orr[i] = 0u;
         }
-        if (row_valid) {
+        if (row_valid && out_ok) {
           if (p.o_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + out_row * D + c * 32);
 #pragma unroll
@@ -528,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (row_valid)
+      if (row_valid && out_ok)
         p.lse[out_row] = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }

@@ -29,6 +29,7 @@ enum WaitSite : int {
   SITE_BWD_COMPUTE = 7,
   SITE_BWD_EPILOGUE = 8,
   SITE_DRAIN = 9,
+  SITE_BOUNDS = 100,  // + check number: a debug build's bounds check failed
 };
 
 // Fixed limit for the teardown drains (copies and MMAs already in flight

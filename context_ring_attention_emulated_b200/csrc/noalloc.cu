@@ -6,7 +6,8 @@
 // library holds it (RATTN_NOALLOC_SCRATCH_BYTES) until the process exits.
 // Host code cannot use the array's name as a device address, so its address
 // is looked up once per device with cudaGetSymbolAddress, on the first call
-// made while that device is current, and cached.
+// made while that device is current, and cached for the life of the process
+// (the cache assumes the device's primary context is never reset).
 #include <mutex>
 
 #include "internal.h"

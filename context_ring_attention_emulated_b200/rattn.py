@@ -15,9 +15,12 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "librattn.so")
+# RATTN_DEBUG=1 selects the debug build (device-side bounds checks; built by
+# ``python -m context_ring_attention_emulated_b200.build --debug``).
+DEBUG = os.environ.get("RATTN_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(_PKG, "librattn_debug.so" if DEBUG else "librattn.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = 0, 1, 2, 3, 4, 5
 F32, BF16 = 0, 1
 LAYOUT_CONTIGUOUS, LAYOUT_HEAD_TAIL, LAYOUT_STRIPED = 0, 1, 2
 ROPE_HALF, ROPE_INTERLEAVED = 0, 1
@@ -72,7 +75,8 @@ class RattnError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m context_ring_attention_emulated_b200.build` (no fallback exists)")
+                          "`python -m context_ring_attention_emulated_b200.build"
+                          f"{' --debug' if DEBUG else ''}` (no fallback exists)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, res, args in SIGNATURES:
         f = getattr(lib, name)

@@ -64,7 +64,9 @@ typedef enum {
   RATTN_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or enum       */
   RATTN_ERR_UNSUPPORTED = 2,   /* valid request the library does not handle  */
   RATTN_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed          */
-  RATTN_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up         */
+  RATTN_ERR_TIMEOUT = 4,       /* a bounded device-side wait gave up         */
+  RATTN_ERR_BOUNDS = 5         /* a debug build's device-side bounds check    */
+                               /* failed (librattn_debug.so only)             */
 } rattn_status;
 
 typedef enum { RATTN_F32 = 0, RATTN_BF16 = 1 } rattn_dtype;
@@ -234,7 +236,10 @@ rattn_status rattn_merge(float* o_acc, float* lse_acc, const float* o_blk, const
 
 /* [CP-glossary], [Ring-page]: the whole emulated ring forward. q, k, v
  * [B,H,Lp,D] in rank-major order (as cp_layout_permute writes them) with
- * positions pos int32 [Lp]. Every emulated rank r keeps its Q slice fixed and,
+ * positions pos int32 [Lp], non-decreasing within each of the cp_size slices
+ * (cp_layout_permute's output is): the kernels find visible and unmasked
+ * tiles by binary search over them, so unsorted positions give wrong O / LSE
+ * without an error (the debug build reports them as RATTN_ERR_BOUNDS). Every emulated rank r keeps its Q slice fixed and,
  * for hops t = 0..cp_size-1, attends the K/V slice of rank s = (r - t) mod
  * cp_size (blocks move to the next rank each hop), folding each block into a
  * running max / normaliser in ring order; the next block's K/V loads overlap
@@ -254,8 +259,9 @@ size_t rattn_ring_bwd_workspace_size(int B, int H, int64_t Lp, int D);
 
 /* [CP-glossary] "Practical use and trade-offs" (`.backward()` through the CP
  * attention): gradients of the ring forward, recomputing P from the saved fp32
- * LSE. Inputs as rattn_ring_fwd plus o (forward output, `dtype`), dout (dL/dO,
- * `dtype`) and lse (fp32). Outputs dq, dk, dv [B,H,Lp,D] in `dtype`. The
+ * LSE. Inputs as rattn_ring_fwd (pos non-decreasing within each of the cp_size
+ * slices, as there) plus o (forward output, `dtype`), dout (dL/dO, `dtype`)
+ * and lse (fp32). Outputs dq, dk, dv [B,H,Lp,D] in `dtype`. The
  * caller passes `workspace` (device, 256-byte aligned, at least
  * rattn_ring_bwd_workspace_size bytes); its contents on entry are ignored and
  * on return undefined. Calls sharing a workspace must not overlap. */
@@ -348,8 +354,10 @@ rattn_status rattn_grad_fold(float* acc, const float* blk, int64_t n, void* stre
  * whose rattn_ring_bwd_workspace_size exceeds that size returns
  * RATTN_ERR_UNSUPPORTED and launches nothing. The first call on a device,
  * with that device current, looks up the array's device address (once per
- * device); make that first call before any stream capture on the device. All
- * calls share the one array and it keeps the previous call's contents (the
+ * device); make that first call before any stream capture on the device. The
+ * looked-up address is cached for the life of the process: it assumes the
+ * device's primary context is never destroyed (after cudaDeviceReset it would
+ * be stale). All calls share the one array and it keeps the previous call's contents (the
  * parts that must start at zero are cleared on the device by the call
  * itself), so calls whose execution overlaps on the GPU, on any streams,
  * race on it: order them on one stream or synchronise between them. */
@@ -362,7 +370,13 @@ rattn_status rattn_ring_bwd_noalloc(const void* q, const void* k, const void* v,
 /* Reads and clears the device-side error word of the current device
  * (synchronises the device). Returns RATTN_OK if no kernel recorded an
  * error, RATTN_ERR_TIMEOUT if a bounded wait gave up (*site, if non-NULL,
- * receives the recorded wait site), RATTN_ERR_CUDA if the read failed. */
+ * receives the recorded wait site, 1..99), RATTN_ERR_BOUNDS if a bounds check
+ * of the debug build (librattn_debug.so, built with RATTN_DEBUG) failed (*site
+ * receives 100 + the check's number), RATTN_ERR_CUDA if the read failed. The
+ * word is process-wide per device and keeps the first failure; the library
+ * caches its device address per device, assuming the device's primary
+ * context lives as long as the process (after cudaDeviceReset the cached
+ * address is stale). */
 rattn_status rattn_get_device_error(int* site);
 
 /* Test hook: the per-wait time limit in nanoseconds used by subsequent

@@ -28,7 +28,7 @@ TOL_GRAD = 3e-2
 
 def load_rattn():
     from context_ring_attention_emulated_b200 import build as b
-    b.build()
+    b.build(debug=os.environ.get("RATTN_DEBUG", "0") == "1")
     from context_ring_attention_emulated_b200 import rattn
     return rattn
 

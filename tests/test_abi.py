@@ -34,9 +34,20 @@ def test_every_declared_symbol_is_exported(rattn):
     assert sorted(n for n, _, _ in rattn.SIGNATURES) == names
 
 
+def test_debug_build_compiles_and_exports_every_symbol():
+    """The RATTN_DEBUG variant (device-side bounds checks) builds from the same
+    sources and exports the same C ABI."""
+    from context_ring_attention_emulated_b200 import build as b
+    path = b.build(debug=True)
+    assert os.path.basename(path) == "librattn_debug.so"
+    lib = ctypes.CDLL(path)
+    for n in header_functions():
+        assert hasattr(lib, n), f"{n} missing from the debug build"
+
+
 def test_status_strings(rattn):
     for code, name in enumerate(["RATTN_OK", "RATTN_ERR_INVALID_ARG", "RATTN_ERR_UNSUPPORTED", "RATTN_ERR_CUDA",
-                                 "RATTN_ERR_TIMEOUT"]):
+                                 "RATTN_ERR_TIMEOUT", "RATTN_ERR_BOUNDS"]):
         assert rattn.status_string(code) == name
     assert rattn.status_string(99) == "RATTN_ERR_UNKNOWN"
 
