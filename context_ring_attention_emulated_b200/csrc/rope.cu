@@ -157,40 +157,51 @@ __global__ void __launch_bounds__(256) rope_kernel(RopeArgs a) {
         sn[t] = a.sign * sf;
       }
     }
-    // Two (batch, head) rows per step, both loads issued before either is
-    // used, so every thread keeps at least two 16-byte loads in flight.
-    for (int bh0 = blockIdx.y; bh0 < a.BH; bh0 += 2 * gridDim.y) {
-      const int bh1 = bh0 + gridDim.y;
-      const bool two = bh1 < a.BH;
-      const uint4* s0 = a.src + (static_cast<long long>(bh0) * n_src + sr) * a.vpr;
-      const uint4* s1 = a.src + (static_cast<long long>(two ? bh1 : bh0) * n_src + sr) * a.vpr;
-      uint4* d0 = a.dst + (static_cast<long long>(bh0) * n_out + o) * a.vpr;
-      uint4* d1 = a.dst + (static_cast<long long>(two ? bh1 : bh0) * n_out + o) * a.vpr;
+    // NR (batch, head) rows per step, all loads issued before any is used,
+    // so every thread keeps four 16-byte loads in flight (HALF: two rows of
+    // two vectors; INTERLEAVED: four rows of one vector).
+    constexpr int NR = STYLE == RATTN_ROPE_HALF ? 2 : 4;
+    for (int bh0 = blockIdx.y; bh0 < a.BH; bh0 += NR * gridDim.y) {
+      const uint4* sp[NR];
+      uint4* dp[NR];
+      bool have[NR];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const int bh = bh0 + k * gridDim.y;
+        have[k] = bh < a.BH;
+        const int b = have[k] ? bh : bh0;
+        sp[k] = a.src + (static_cast<long long>(b) * n_src + sr) * a.vpr;
+        dp[k] = a.dst + (static_cast<long long>(b) * n_out + o) * a.vpr;
+      }
       if (!live) {
         const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        d0[v0] = z;
-        if (two) d1[v0] = z;
-        if (STYLE == RATTN_ROPE_HALF) {
-          d0[v1] = z;
-          if (two) d1[v1] = z;
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          if (!have[k]) continue;
+          dp[k][v0] = z;
+          if (STYLE == RATTN_ROPE_HALF) dp[k][v1] = z;
         }
         continue;
       }
       if (STYLE == RATTN_ROPE_HALF) {
-        const uint4 u00 = __ldg(s0 + v0), u01 = __ldg(s0 + v1);
-        uint4 u10 = u00, u11 = u01;
-        if (two) {
-          u10 = __ldg(s1 + v0);
-          u11 = __ldg(s1 + v1);
+        uint4 u0[NR], u1[NR];
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          if (!have[k]) continue;
+          u0[k] = __ldg(sp[k] + v0);
+          u1[k] = __ldg(sp[k] + v1);
         }
-        rotate_half<T, NP>(u00, u01, cs, sn, d0 + v0, d0 + v1);
-        if (two) rotate_half<T, NP>(u10, u11, cs, sn, d1 + v0, d1 + v1);
+#pragma unroll
+        for (int k = 0; k < NR; ++k)
+          if (have[k]) rotate_half<T, NP>(u0[k], u1[k], cs, sn, dp[k] + v0, dp[k] + v1);
       } else {
-        const uint4 u0 = __ldg(s0 + v0);
-        uint4 u1 = u0;
-        if (two) u1 = __ldg(s1 + v0);
-        rotate_interleaved<T, NP>(u0, cs, sn, d0 + v0);
-        if (two) rotate_interleaved<T, NP>(u1, cs, sn, d1 + v0);
+        uint4 u[NR];
+#pragma unroll
+        for (int k = 0; k < NR; ++k)
+          if (have[k]) u[k] = __ldg(sp[k] + v0);
+#pragma unroll
+        for (int k = 0; k < NR; ++k)
+          if (have[k]) rotate_interleaved<T, NP>(u[k], cs, sn, dp[k] + v0);
       }
     }
   }
