@@ -34,6 +34,9 @@ METRIC = "ring-attn fwd/bwd TFLOP/s (causal FLOPs) on 1 B200; % of BF16 tensor p
 DEFAULT = "bf16_L32000_cp4_fwdbwd"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ROPE_BASE = 10000.0  # rotary base of the RoPE workloads (RoFormer's value)
+# Packed workloads pad every document's share of a rank slice to whole
+# 128-row tiles, so that no kernel tile straddles two documents.
+VARLEN_ALIGN = 128
 # DRAM bytes (read + write) per launch of the dominant kernel from one ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the kernel as it
 # stands, taken on a smaller case and scaled to the workload's launch by the
@@ -166,7 +169,7 @@ def run_ours(args, w, rank, world, local):
     B, H, D, Hkv = w.B, w.H, w.D, w.kv_heads
     heads = {"q": H, "k": Hkv, "v": Hkv, "do": H, "o": H, "dq": H, "dk": Hkv, "dv": Hkv}
     if w.docs:  # packed sequences: host-side layout plan, index arrays resident on the device
-        plan = rattn.cp_layout_varlen_plan(w.cu_seqlens, cp, layout)
+        plan = rattn.cp_layout_varlen_plan(w.cu_seqlens, cp, layout, VARLEN_ALIGN)
         Lp = plan["Tp"]
         src, gkey, segid = (plan[n].to(dev) for n in ("src", "gkey", "segid"))
     else:
@@ -511,7 +514,8 @@ def main():
     flops_step, fwd_flops = step_flops(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "D": w.D, "cp": w.cp,
               "layout": ("contiguous", "head_tail", "striped")[w.layout], "causal": w.causal,
-              "docs": len(w.docs) or None, "H_kv": w.kv_heads, "rope": ("half pairs, base %g, fused into the permute of q,k and the "
+              "docs": len(w.docs) or None,
+              "varlen_align": VARLEN_ALIGN if w.docs else None, "H_kv": w.kv_heads, "rope": ("half pairs, base %g, fused into the permute of q,k and the "
                                               "unpermute of dQ,dK" % ROPE_BASE) if w.rope else None,
               "step": "permute q,k,v" + (",dO" if w.bwd else "") + " -> ring fwd -> unpermute O" +
                       (" -> ring bwd -> unpermute dQ,dK,dV" if w.bwd else ""),

@@ -110,7 +110,8 @@ rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t r
   return r == CUDA_SUCCESS ? RATTN_OK : RATTN_ERR_CUDA;
 }
 
-rattn_status make_tmap_f32_acc(CUtensorMap* map, void* base, int D, int64_t rows, int nseg, int64_t outer) {
+rattn_status make_tmap_f32_acc(CUtensorMap* map, void* base, int D, int64_t rows, int nseg, int64_t outer,
+                               int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return RATTN_ERR_CUDA;
   if (rows < 1) rows = 1;
@@ -118,7 +119,7 @@ rattn_status make_tmap_f32_acc(CUtensorMap* map, void* base, int D, int64_t rows
                               static_cast<cuuint64_t>(nseg), static_cast<cuuint64_t>(outer)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(rows) * D * 4,
                                  static_cast<cuuint64_t>(nseg) * rows * D * 4};
-  const cuuint32_t box[4] = {32u, 128u, 1u, 1u};
+  const cuuint32_t box[4] = {32u, static_cast<cuuint32_t>(box_rows), 1u, 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -180,29 +181,46 @@ rattn_status cp_layout_unpermute(const void* y, void* x, int B, int H, int64_t L
 
 rattn_status cp_layout_varlen_plan(const int32_t* cu_seqlens, int nseq, int cp_size, rattn_layout layout,
                                    int64_t* Tp, int32_t* src, int32_t* pos, int32_t* segid, int32_t* gkey) {
-  if (!cu_seqlens || nseq < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1 || !Tp) return RATTN_ERR_INVALID_ARG;
+  return cp_layout_varlen_plan_aligned(cu_seqlens, nseq, cp_size, layout, 1, Tp, src, pos, segid, gkey);
+}
+
+rattn_status cp_layout_varlen_plan_aligned(const int32_t* cu_seqlens, int nseq, int cp_size, rattn_layout layout,
+                                           int align, int64_t* Tp, int32_t* src, int32_t* pos, int32_t* segid,
+                                           int32_t* gkey) {
+  if (!cu_seqlens || nseq < 0 || cp_size < 1 || chunks_of(cp_size, layout) < 1 || !Tp || align < 1)
+    return RATTN_ERR_INVALID_ARG;
   if (cu_seqlens[0] != 0) return RATTN_ERR_INVALID_ARG;
+  // Rows of each sequence's share on one rank: its padded length over cp,
+  // rounded up to a multiple of align.
+  auto share_rows = [&](int64_t L) {
+    const int64_t n = cp_layout_padded_len(L, cp_size, layout) / cp_size;
+    return (n + align - 1) / align * align;
+  };
   int64_t total = 0;
   for (int i = 0; i < nseq; ++i) {
     const int64_t L = static_cast<int64_t>(cu_seqlens[i + 1]) - cu_seqlens[i];
     if (L < 0) return RATTN_ERR_INVALID_ARG;
-    total += cp_layout_padded_len(L, cp_size, layout);
+    total += share_rows(L) * cp_size;
     if (total > INT32_MAX) return RATTN_ERR_INVALID_ARG;
   }
   *Tp = total;
   if (!src && !pos && !segid && !gkey) return RATTN_OK;
   // Rank r's slice holds, for every sequence in order, the rows rank r holds
-  // when that sequence alone is permuted.
+  // when that sequence alone is permuted, then (align > 1) pad rows up to the
+  // aligned share; those carry positions Lp + r * e + k past every position
+  // of the sequence, so that gkey keeps increasing along the slice.
   const int64_t per_rank = total / cp_size;
   int64_t seq_off = 0, rank_off = 0;  // sequence offset in the padded pack / in a rank slice
   for (int i = 0; i < nseq; ++i) {
     const int L = cu_seqlens[i + 1] - cu_seqlens[i];
     const int Lp = static_cast<int>(cp_layout_padded_len(L, cp_size, layout));
     const int n = Lp / cp_size;
+    const int n_al = static_cast<int>(share_rows(L));
+    const int e = n_al - n;
     const int c = cp_map_c(Lp, cp_size, layout);
     for (int r = 0; r < cp_size; ++r) {
-      for (int t = 0; t < n; ++t) {
-        const int g = slot_to_global(r * n + t, c, cp_size, layout);
+      for (int t = 0; t < n_al; ++t) {
+        const int g = t < n ? slot_to_global(r * n + t, c, cp_size, layout) : Lp + r * e + (t - n);
         const int64_t slot = r * per_rank + rank_off + t;
         if (src) src[slot] = g < L ? cu_seqlens[i] + g : -1;
         if (pos) pos[slot] = g;
@@ -210,8 +228,8 @@ rattn_status cp_layout_varlen_plan(const int32_t* cu_seqlens, int nseq, int cp_s
         if (gkey) gkey[slot] = static_cast<int32_t>(seq_off + g);
       }
     }
-    seq_off += Lp;
-    rank_off += n;
+    seq_off += static_cast<int64_t>(n_al) * cp_size;
+    rank_off += n_al;
   }
   return RATTN_OK;
 }

@@ -16,15 +16,19 @@
 // next tiles are computed; the workspace is converted to the output dtype at
 // the end.
 //
-// Warp roles (448 threads):
-//   warps 0..3   dQ read-out: one thread per query row, 32-column chunks
-//                staged 128-byte swizzled, one thread issues the reduce-adds;
+// Warp roles (512 threads):
+//   warps 0..3   dQ read-out: one thread per query row; the whole dQ tile is
+//                read out of TMEM into registers (freeing its columns at
+//                once), then staged 128-byte swizzled in 32-column chunks,
+//                one thread issuing the reduce-adds;
 //   warps 4..11  two warpgroups, one thread per key row (TMEM lane) each:
 //                P^T and dS^T over the warpgroup's 64 query columns, finally
 //                half of dK/dV each;
 //   warp 12      producer: K, V once; per query tile Q and dO by TMA and the
 //                tile's LSE (pre-scaled by log2 e) and Delta into shared memory;
-//   warp 13      TMEM allocation and tcgen05.mma issue (one thread).
+//   warp 13      TMEM allocation and tcgen05.mma issue (one thread);
+//   warps 14, 15 idle (they complete the producer/MMA warpgroup, whose
+//                registers the dQ warpgroup takes over: setmaxnreg).
 // TMEM columns: [0,128) S^T, then P^T (bf16, warpgroup g at [64g, 64g+32));
 // [128,256) dP^T, then dS^T (bf16, at 128 + [64g, 64g+32)), then dQ;
 // dV [256,256+D); dK [256+D,256+2D). dS also goes to a swizzled shared tile,
@@ -52,13 +56,21 @@
 namespace rattn {
 namespace {
 
-constexpr int kThreads = 448;  // 14 warps
+constexpr int kThreads = 512;  // 16 warps
 constexpr int BQ = 128;        // query rows per tile
 constexpr int BK = 128;        // key rows per CTA
 constexpr int kMaxHops = 64;
 constexpr int kWarpProducer = 12;
 constexpr int kWarpMma = 13;
 constexpr int kWarpCompute0 = 4;  // warps 4..11: two compute warpgroups
+// Registers per thread: the kernel is launched with kLaunchRegs; the dQ
+// warpgroup (warps 0..3) then grows to kRegsReduce, taken from the
+// producer/MMA warpgroup (warps 12..15), which shrinks to kRegsLoad; the
+// compute warpgroups keep kLaunchRegs. 144 + 2 x 128 + 112 = 4 x 128.
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsReduce = 144;
+constexpr int kRegsLoad = 112;
+static_assert(kRegsReduce + 2 * kLaunchRegs + kRegsLoad == 4 * kLaunchRegs, "register split must balance");
 constexpr int kReduceBar = 1;     // named barrier of the dQ warpgroup (warps 0..3)
 
 template <int D>
@@ -84,8 +96,8 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_DELTA + NSQ * 128 * 4;
   // barrier indices
   static constexpr int B_KV = 0, B_QF = 1, B_QE = B_QF + NSQ, B_OF = B_QE + NSQ, B_OE = B_OF + NSO,
-                       B_SF = B_OE + NSO, B_PR = B_SF + 1, B_DPF = B_PR + 1, B_DSR = B_DPF + 1, B_DKD = B_DSR + 1,
-                       B_DVD = B_DKD + 1, B_DQF = B_DVD + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
+                       B_SF = B_OE + NSO, B_PR = B_SF + 1, B_DPF = B_PR + 1, B_DSR = B_DPF + 1,
+                       B_DQF = B_DSR + 1, B_DQE = B_DQF + 1, B_FIN = B_DQE + 1,
                        B_DRAIN = B_FIN + 1, NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_FULL = OFF_MISC + 16;  // NSQ ints: tile needs no masking
@@ -202,8 +214,8 @@ __device__ __forceinline__ void stage_dq_chunk(const uint32_t (&v)[32], uint8_t*
   }
 }
 
-// 14 warps share an SM's four register-file partitions 4/4/3/3, so a thread
-// may hold at most 16,384 / (4 x 32) = 128 registers.
+// 16 warps share an SM's four register-file partitions 4/4/4/4: 16,384 / (4 x
+// 32) = 128 registers per thread at launch.
 template <int D, bool SEG, bool SPLIT>  // SEG: packed sequences; SPLIT: one hop across processes
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -221,8 +233,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_p_ready = bars + C::B_PR;     // P^T(j) written over it (one arrival per compute warp)
   uint64_t* bar_dp_full = bars + C::B_DPF;    // dP^T(j) in TMEM
   uint64_t* bar_ds_ready = bars + C::B_DSR;   // dS^T(j) over dP^T(j) and dS(j) in shared memory
-  uint64_t* bar_dk_done = bars + C::B_DKD;    // dK MMA of j completed (dS^T(j) consumed)
-  uint64_t* bar_dv_done = bars + C::B_DVD;    // dV MMA of j completed (P^T(j) consumed)
   uint64_t* bar_dq_full = bars + C::B_DQF;    // dQ(j) in TMEM (dS(j) in shared memory consumed)
   uint64_t* bar_dq_empty = bars + C::B_DQE;   // dQ(j) read out of TMEM (one arrival per dQ warp)
   uint64_t* bar_fin = bars + C::B_FIN;        // every MMA completed
@@ -273,8 +283,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_p_ready, 8);
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_ds_ready, 8);
-    mbar_init(bar_dk_done, 1);
-    mbar_init(bar_dv_done, 1);
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_empty, 4);
     mbar_init(bar_fin, 1);
@@ -332,6 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int issued_q = 0, issued_o = 0;
   bool kv_issued = false;
 
+  if (warp >= kWarpProducer) {
+    regs_dec<kRegsLoad>();  // warps 12..15 (14 and 15 idle)
   if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     if (NIT > 0) {
@@ -420,10 +430,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------------- MMA issue
     // Per query tile j: S^T(j) = K Q^T, dP^T(j) = V dO^T, dV += P^T dO,
     // dK += dS^T Q (dS^T read from TMEM over dP^T), dQ(j) = dS K (into the
-    // dP^T columns once dK(j) has read them). Issue order, steady state:
-    //   dK(i), dQ(i), dV(i+1), dP(i+1), S(i+2)
-    // so that the read-out of dQ(i) overlaps dV(i+1), and the softmax of
-    // tile i+2 and the dS of tile i+1 overlap dK / dQ and S.
+    // dP^T columns). Issue order, steady state:
+    //   dK(i), dQ(i), dP(i+1), dV(i+1), S(i+2)
+    // dP(i+1) is on the chain dS(i) -> dK / dQ(i) -> read-out of dQ(i) ->
+    // dP(i+1) -> dS(i+1), so it goes first once dQ(i) is out of TMEM; dV and
+    // S fill the pipe while the compute warpgroups form dS(i+1). MMAs issued
+    // by one thread execute in issue order, so dQ(i) follows dK(i) without a
+    // wait although it overwrites the dS^T columns dK(i) reads, and S(j)
+    // follows dV(j-1), which reads the P^T columns S(j) overwrites.
     if (lane == 0 && NIT > 0) {
       const uint32_t idesc_t = idesc_bf16_f32(BK, BQ, 0, 0);  // S^T, dP^T: K-major A and B
       const uint32_t idesc_g = idesc_bf16_f32(BK, D, 0, 1);   // dV, dK: A in TMEM, B MN-major
@@ -437,7 +451,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       auto mma_s = [&](int j) -> bool {
         if (!wt(&bar_q_full[j % C::NSQ], (j / C::NSQ) & 1)) return false;
-        if (j > 0 && !wt(bar_dv_done, (j - 1) & 1)) return false;  // P^T(j-1) consumed
         tc_fence_after();
         const uint32_t q = sQ(j);
 #pragma unroll
@@ -461,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_dp_full);
-        umma_commit(&bar_o_empty[j % C::NSO]);  // dV(j) was issued before dP(j)
+        if (j == 0) umma_commit(&bar_o_empty[0]);  // dV(0) was issued before dP(0)
         return true;
       };
       auto mma_dv = [&](int j) -> bool {
@@ -475,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ts(tmem + C::T_DV, tmem + a_col, sdesc_sw128(o + kk * 2048, C::BOX, 1024), idesc_g,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar_dv_done);
+        if (j > 0) umma_commit(&bar_o_empty[j % C::NSO]);  // dP(j) was issued before dV(j)
         return true;
       };
       auto mma_dk = [&](int j) -> bool {
@@ -488,12 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_ts(tmem + C::T_DK, tmem + a_col, sdesc_sw128(q + kk * 2048, C::BOX, 1024), idesc_g,
                   (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar_dk_done);
         umma_commit(&bar_q_empty[j % C::NSQ]);  // S(j) and dK(j) were Q's readers
         return true;
       };
       auto mma_dq = [&](int j) -> bool {
-        if (!wt(bar_dk_done, j & 1)) return false;  // dQ overwrites the dS^T columns dK(j) reads
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
@@ -507,12 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = ok && mma_s(0) && mma_dv(0) && mma_dp(0) && (NIT < 2 || mma_s(1));
       for (int i = 0; i < NIT && ok; ++i) {
         ok = mma_dk(i) && mma_dq(i);
-        if (ok && i + 1 < NIT) ok = mma_dv(i + 1) && mma_dp(i + 1);
+        if (ok && i + 1 < NIT) ok = mma_dp(i + 1) && mma_dv(i + 1);
         if (ok && i + 2 < NIT) ok = mma_s(i + 2);
       }
       if (ok) umma_commit(bar_fin);
       else record_failure(s_abort, p.err, SITE_BWD_MMA);
     }
+  }
   } else if (warp >= kWarpCompute0) {
     // ------------------------------------------------- P^T and dS^T per key
     // Two warpgroups; warpgroup wg owns query columns [64 wg, 64 wg + 64) of
@@ -656,11 +668,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // by dQ (box wg, row = key), 16 query columns at a time (the packed
         // pairs of chunk c land on columns already read).
         uint8_t* rowp = sds + row * 128;
+        uint32_t dpb[2][16];  // chunk c in dpb[c & 1]; chunk c + 1 is read while c is processed
+        tmem_ld16(t_dp, dpb[0]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t dp[16];
-          tmem_ld16(t_dp + c * 16, dp);
           tmem_wait_ld();
+          if (c + 1 < 4) tmem_ld16(t_dp + (c + 1) * 16, dpb[(c + 1) & 1]);
+          const uint32_t (&dp)[16] = dpb[c & 1];
           uint32_t pk[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -747,14 +761,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
+    regs_inc<kRegsReduce>();
     // ------------------------------------------------------ dQ read-out
     // Warps 0..3, one thread per query row (TMEM lane): each dQ(j) is read
-    // out of TMEM in 32-column chunks (the dP^T columns are released as soon
-    // as the last chunk is in registers), staged in shared memory and added
-    // into the fp32 accumulator by TMA tile reduce-adds, which run on in the
-    // background while the next tiles are computed. One thread issues the
-    // copies; named barriers keep the warpgroup in step, and every decision
-    // to stop is taken together (so no thread is left at a barrier).
+    // out of TMEM whole (D registers per thread), which releases the dP^T
+    // columns at once; then it is staged in shared memory in 32-column
+    // chunks and added into the fp32 accumulator by TMA tile reduce-adds,
+    // which run on in the background while the next tiles are computed. One
+    // thread issues the copies; named barriers keep the warpgroup in step,
+    // and every decision to stop is taken together (so no thread is left at
+    // a barrier).
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // query row
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -776,29 +792,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        uint32_t v[C::NCH][32];
 #pragma unroll
-        for (int h = 0; h < C::NCH / 2; ++h) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tmem + lane_base + C::T_DP + (2 * h) * 32, v0);
-          tmem_ld32(tmem + lane_base + C::T_DP + (2 * h + 1) * 32, v1);
-          tmem_wait_ld();
-          if (h == C::NCH / 2 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_dq_empty);  // one arrival per warp
-          }
-          if constexpr (SPLIT) {  // the caller's accumulator holds dQ itself
+        for (int c = 0; c < C::NCH; ++c) tmem_ld32(tmem + lane_base + C::T_DP + c * 32, v[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dq_empty);  // one arrival per warp
+        if constexpr (SPLIT) {  // the caller's accumulator holds dQ itself
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              v0[e] = __float_as_uint(__uint_as_float(v0[e]) * p.scale);
-              v1[e] = __float_as_uint(__uint_as_float(v1[e]) * p.scale);
-            }
-          }
-          stage_dq_chunk<D>(v0, stg + (n_staged % C::NSTG) * C::CHUNK, row, elected, n_staged >= C::NSTG, &tm_dq,
-                            (2 * h) * 32, i * BQ, r, bh);
-          ++n_staged;
-          stage_dq_chunk<D>(v1, stg + (n_staged % C::NSTG) * C::CHUNK, row, elected, n_staged >= C::NSTG, &tm_dq,
-                            (2 * h + 1) * 32, i * BQ, r, bh);
+          for (int c = 0; c < C::NCH; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[c][e] = __float_as_uint(__uint_as_float(v[c][e]) * p.scale);
+        }
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          stage_dq_chunk<D>(v[c], stg + (n_staged % C::NSTG) * C::CHUNK, row, elected, n_staged >= C::NSTG, &tm_dq,
+                            c * 32, i * BQ, r, bh);
           ++n_staged;
         }
       }
@@ -880,6 +890,16 @@ unsigned grid_for(long long work, int threads) {
   return static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
+// The register split among the warpgroups balances only if the kernel is
+// launched with exactly kLaunchRegs per thread (a lower count would leave the
+// dQ warpgroup's increase waiting for registers that never come): refuse to
+// launch otherwise.
+rattn_status check_launch_regs(const void* kfn) {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kfn) != cudaSuccess) return RATTN_ERR_CUDA;
+  return fa.numRegs == kLaunchRegs ? RATTN_OK : RATTN_ERR_UNSUPPORTED;
+}
+
 template <int D>
 rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   using C = Cfg<D>;
@@ -901,6 +921,7 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   const void* kfn = a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true, false>)
                          : reinterpret_cast<const void*>(&bwd_kernel<D, false, false>);
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
+  if ((st = check_launch_regs(kfn)) != RATTN_OK) return st;
   bwd_prep_kernel<D, true><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
@@ -967,6 +988,7 @@ rattn_status launch_split(const PartialBwdArgs& a, const DevCtx& ctx) {
   if ((st = make_tmap_f32_acc(&tdq, a.dq_acc, D, a.Lq, 1, a.BH)) != RATTN_OK) return st;
   const void* kfn = reinterpret_cast<const void*>(&bwd_kernel<D, false, true>);
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
+  if ((st = check_launch_regs(kfn)) != RATTN_OK) return st;
   Params p;
   p.lse = a.lse;
   p.delta = a.delta;

@@ -41,10 +41,11 @@ constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,
                             int box_rows);
 
-// 4-D fp32 tensor map over [outer][nseg][rows][D] with a (32 x 128-row) box
+// 4-D fp32 tensor map over [outer][nseg][rows][D] with a (32 x box_rows) box
 // and 128-byte swizzle, for tile reduce-adds into an accumulator; rows past
 // `rows` are outside the tensor (reduce-adds there are dropped).
-rattn_status make_tmap_f32_acc(CUtensorMap* map, void* base, int D, int64_t rows, int nseg, int64_t outer);
+rattn_status make_tmap_f32_acc(CUtensorMap* map, void* base, int D, int64_t rows, int nseg, int64_t outer,
+                               int box_rows = 128);
 
 // Sets the max dynamic shared memory attribute of a kernel once per device.
 rattn_status set_smem_attr(const void* kernel, int bytes);

@@ -37,6 +37,7 @@ SIGNATURES = [
     ("cp_layout_permute", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
     ("cp_layout_unpermute", _I, [_P, _P, _I, _I, _I64, _I64, _I, _I, _I, _I, _P]),
     ("cp_layout_varlen_plan", _I, [_P, _I, _I, _I, ctypes.POINTER(_I64), _P, _P, _P, _P]),
+    ("cp_layout_varlen_plan_aligned", _I, [_P, _I, _I, _I, _I, ctypes.POINTER(_I64), _P, _P, _P, _P]),
     ("cp_layout_gather", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _P]),
     ("cp_layout_scatter", _I, [_P, _P, _P, _I, _I, _I64, _I64, _I, _I, _P]),
     ("rattn_ring_fwd_varlen", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I64, _I, _I, _I, _I, _F, _P, _P, _P]),
@@ -245,19 +246,22 @@ def cp_layout_unpermute_rope_grad(dy, L, cp_size, layout=LAYOUT_HEAD_TAIL, rope_
     return dx
 
 
-def cp_layout_varlen_plan(cu_seqlens, cp_size, layout=LAYOUT_HEAD_TAIL):
+def cp_layout_varlen_plan(cu_seqlens, cp_size, layout=LAYOUT_HEAD_TAIL, align=1):
     """Host-side layout of a pack of sequences (boundaries cu_seqlens, a list or
-    1-D int tensor starting at 0). Returns a dict of CPU int32 tensors
-    src, pos, segid, gkey [Tp] and Tp."""
+    1-D int tensor starting at 0), every sequence's share of every rank slice
+    padded to a multiple of ``align`` rows (1: the plain packed layout; 128:
+    no kernel tile straddles two sequences). Returns a dict of CPU int32
+    tensors src, pos, segid, gkey [Tp] and Tp."""
     cu = torch.as_tensor(cu_seqlens, dtype=torch.int32).contiguous().cpu()
     nseq = cu.numel() - 1
     tp = ctypes.c_int64(0)
-    _check("cp_layout_varlen_plan", lib.cp_layout_varlen_plan(_ptr(cu), nseq, cp_size, layout, ctypes.byref(tp),
-                                                                None, None, None, None))
+    fn = "cp_layout_varlen_plan_aligned"
+    _check(fn, lib.cp_layout_varlen_plan_aligned(_ptr(cu), nseq, cp_size, layout, int(align), ctypes.byref(tp),
+                                                 None, None, None, None))
     out = {n: torch.empty(tp.value, dtype=torch.int32) for n in ("src", "pos", "segid", "gkey")}
-    _check("cp_layout_varlen_plan", lib.cp_layout_varlen_plan(
-        _ptr(cu), nseq, cp_size, layout, ctypes.byref(tp), _ptr(out["src"]), _ptr(out["pos"]), _ptr(out["segid"]),
-        _ptr(out["gkey"])))
+    _check(fn, lib.cp_layout_varlen_plan_aligned(
+        _ptr(cu), nseq, cp_size, layout, int(align), ctypes.byref(tp), _ptr(out["src"]), _ptr(out["pos"]),
+        _ptr(out["segid"]), _ptr(out["gkey"])))
     out["Tp"] = tp.value
     return out
 

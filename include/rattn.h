@@ -165,6 +165,23 @@ rattn_status cp_layout_unpermute_rope_grad(const void* dy, void* dx,
 rattn_status cp_layout_varlen_plan(const int32_t* cu_seqlens, int nseq, int cp_size, rattn_layout layout,
                                    int64_t* Tp, int32_t* src, int32_t* pos, int32_t* segid, int32_t* gkey);
 
+/* cp_layout_varlen_plan with every sequence's share of every rank slice
+ * padded further, to a multiple of `align` rows (align >= 1; 1 gives
+ * cp_layout_varlen_plan's layout). The page fixes only the multiple-of-2cp
+ * padding; padding more keeps the pairing and changes nothing but pad slots,
+ * which every attention kernel masks. With align = 128 (the kernels' tile
+ * height) no 128-row tile of a rank slice straddles two sequences, so the
+ * kernels skip what lies between sequences tile by tile instead of masking
+ * inside tiles. The extra pad slots of rank r's share of sequence i follow its
+ * real rows, with pos = Lp_i + r * e_i + k (e_i extra slots per rank,
+ * k = 0..e_i-1), src = -1, segid = 2i + 1; a sequence takes cp_size times its
+ * aligned share in the padded pack, and gkey = that offset + pos still
+ * increases along every rank slice. RATTN_ERR_INVALID_ARG also when
+ * align < 1. */
+rattn_status cp_layout_varlen_plan_aligned(const int32_t* cu_seqlens, int nseq, int cp_size, rattn_layout layout,
+                                           int align, int64_t* Tp, int32_t* src, int32_t* pos, int32_t* segid,
+                                           int32_t* gkey);
+
 /* Row gather for the varlen layout: y [B,H,T_out,D] with
  * y[:, :, i] = x[:, :, src[i]] for src[i] >= 0 and zero rows where
  * src[i] < 0; src is a device int32 array [T_out] with entries < T_in

@@ -102,7 +102,7 @@ def unpermute(y, L, cp, layout):
     return x
 
 
-def varlen_index(cu_seqlens, cp, layout):
+def varlen_index(cu_seqlens, cp, layout, align=1):
     """Layout of a pack of sequences with boundaries cu_seqlens [nseq + 1].
 
     Returns (Tp, src, pos, seg, gkey), each per slot of the permuted pack:
@@ -112,22 +112,38 @@ def varlen_index(cu_seqlens, cp, layout):
     Rank r's slice (rows [r Tp / cp, (r + 1) Tp / cp)) holds, for every
     sequence in order, the rows rank r holds under ``perm_index`` of that
     sequence alone.
+
+    align > 1 (a reading: the page fixes only the multiple-of-2cp padding, as
+    the least a sequence needs; padding more is allowed since pad rows are
+    masked) pads every sequence's share on every rank to a multiple of align
+    rows, so that align-row tiles never straddle two sequences. The extra pad
+    rows of rank r's share come after its real rows, with positions
+    Lp_i + r * e + k (e extra rows per rank, k = 0..e-1), past every position
+    the sequence uses; the sequence then occupies cp * (its aligned share) rows
+    of the padded pack, which is what the next sequence's offset counts.
     """
     cu = [int(x) for x in cu_seqlens]
     if any(b < a for a, b in zip(cu, cu[1:])) or (cu and cu[0] != 0):
         raise ValueError("cu_seqlens must start at 0 and be non-decreasing")
+    if align < 1:
+        raise ValueError("align must be positive")
     per_rank = [[] for _ in range(cp)]
     offset = 0
     for i in range(len(cu) - 1):
         L = cu[i + 1] - cu[i]
         Lp, src_i, pos_i = perm_index(L, cp, layout)
         n = Lp // cp
+        n_al = -(-n // align) * align
+        e = n_al - n
         for r in range(cp):
             for j in range(r * n, (r + 1) * n):
                 real = src_i[j] >= 0
                 per_rank[r].append((cu[i] + src_i[j] if real else -1, pos_i[j], i if real else -1,
                                     offset + pos_i[j]))
-        offset += Lp
+            for kk in range(e):
+                p = Lp + r * e + kk
+                per_rank[r].append((-1, p, -1, offset + p))
+        offset += cp * n_al
     rows = [t for r in range(cp) for t in per_rank[r]]
     Tp = len(rows)
     src = np.array([t[0] for t in rows], dtype=np.int64)
@@ -137,9 +153,9 @@ def varlen_index(cu_seqlens, cp, layout):
     return Tp, src, pos, seg, gkey
 
 
-def varlen_permute(x, cu_seqlens, cp, layout):
+def varlen_permute(x, cu_seqlens, cp, layout, align=1):
     """x [..., T, D] (a pack) -> y [..., Tp, D] in rank-major order; pad rows zero."""
-    Tp, src, _, _, _ = varlen_index(cu_seqlens, cp, layout)
+    Tp, src, _, _, _ = varlen_index(cu_seqlens, cp, layout, align)
     y = np.zeros(x.shape[:-2] + (Tp, x.shape[-1]), dtype=x.dtype)
     for i in range(Tp):
         if src[i] >= 0:
@@ -147,9 +163,9 @@ def varlen_permute(x, cu_seqlens, cp, layout):
     return y
 
 
-def varlen_unpermute(y, cu_seqlens, cp, layout):
+def varlen_unpermute(y, cu_seqlens, cp, layout, align=1):
     """Inverse of varlen_permute: y [..., Tp, D] -> x [..., T, D], pad rows dropped."""
-    Tp, src, _, _, _ = varlen_index(cu_seqlens, cp, layout)
+    Tp, src, _, _, _ = varlen_index(cu_seqlens, cp, layout, align)
     T = int(cu_seqlens[-1])
     x = np.zeros(y.shape[:-2] + (T, y.shape[-1]), dtype=y.dtype)
     for i in range(Tp):

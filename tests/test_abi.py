@@ -188,23 +188,24 @@ def test_bwd_rejects_bad_arguments_and_sizes_workspace(rattn):
 @pytest.mark.parametrize("layout", [0, 1, 2])
 @pytest.mark.parametrize("cp", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("cu", [[0, 5, 16, 16, 23], [0, 64], [0], [0, 1, 2, 3], [0, 4000, 4001, 9000, 32000]])
-def test_varlen_plan_matches_oracle(rattn, layout, cp, cu):
-    """The library's host-side packed layout against the oracle's, slot by slot;
-    the kernels' segid is 2 * sequence (+1 for padding)."""
+@pytest.mark.parametrize("align", [1, 8, 128])
+def test_varlen_plan_matches_oracle(rattn, layout, cp, cu, align):
+    """The library's host-side packed layout against the oracle's, slot by slot
+    (plain and aligned); the kernels' segid is 2 * sequence (+1 for padding)."""
     import oracle
-    plan = rattn.cp_layout_varlen_plan(cu, cp, layout)
-    Tp, src, pos, seg, gkey = oracle.varlen_index(cu, cp, layout)
+    plan = rattn.cp_layout_varlen_plan(cu, cp, layout, align)
+    Tp, src, pos, seg, gkey = oracle.varlen_index(cu, cp, layout, align)
     assert plan["Tp"] == Tp
     assert np.array_equal(plan["src"].numpy(), src)
     assert np.array_equal(plan["pos"].numpy(), pos)
     assert np.array_equal(plan["gkey"].numpy(), gkey)
-    seq = np.repeat(np.arange(len(cu) - 1), [oracle.padded_len(b - a, cp, layout) for a, b in zip(cu, cu[1:])])
     # every pad slot belongs to its sequence's block: recover the sequence of each slot from gkey
-    offsets = np.cumsum([0] + [oracle.padded_len(b - a, cp, layout) for a, b in zip(cu, cu[1:])])
+    sizes = [-(-oracle.padded_len(b - a, cp, layout) // cp // align) * align * cp for a, b in zip(cu, cu[1:])]
+    offsets = np.cumsum([0] + sizes)
     slot_seq = np.searchsorted(offsets, gkey, side="right") - 1 if Tp else np.zeros(0, int)
     assert np.array_equal(plan["segid"].numpy(), 2 * slot_seq + (src < 0))
     assert np.array_equal(np.where(src >= 0, slot_seq, -1), seg)
-    assert len(seq) == Tp
+    assert sum(sizes) == Tp
 
 
 def test_varlen_calls_reject_bad_arguments(rattn):
@@ -219,6 +220,11 @@ def test_varlen_calls_reject_bad_arguments(rattn):
     ok = torch.tensor([0, 5], dtype=torch.int32)
     assert L.cp_layout_varlen_plan(ok.data_ptr(), 1, 0, 1, ctypes.byref(tp), None, None, None, None) == \
         rattn.ERR_INVALID_ARG
+    for align in (0, -128):
+        assert L.cp_layout_varlen_plan_aligned(ok.data_ptr(), 1, 2, 1, align, ctypes.byref(tp), None, None, None,
+                                               None) == rattn.ERR_INVALID_ARG
+    assert L.cp_layout_varlen_plan_aligned(ok.data_ptr(), 1, 2, 1, 128, ctypes.byref(tp), None, None, None,
+                                           None) == rattn.OK and tp.value == 256
     assert L.cp_layout_gather(FAKE, FAKE, FAKE, 1, 1, 16, 16, 3, 1, None) == rattn.ERR_UNSUPPORTED
     assert L.cp_layout_gather(FAKE, MIS, FAKE, 1, 1, 16, 16, 64, 1, None) == rattn.ERR_INVALID_ARG
     assert L.cp_layout_gather(FAKE, FAKE, FAKE, 1, 1, 16, 0, 64, 1, None) == rattn.OK

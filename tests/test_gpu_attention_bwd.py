@@ -86,3 +86,35 @@ def test_ring_bwd_full_size_loss_grad(rattn):
         ref = oracle.attention_bwd(qh, kh, vh, to64(do1[0, h]), w.scale, True, row_block=1024)
         for got, r in zip((dq, dk, dv), ref):
             check_grad(got[0, h].float().cpu().numpy(), r)
+
+
+def test_ring_bwd_full_size_last_head_sampled(rattn):
+    """The 32k / cp=4 backward with dO ~ N(0, 1), checked on the last head on
+    sampled rows: dK, dV of the first and last four keys of every chunk and of
+    128 seeded random keys (each summed over all 32,000 queries), and dQ of
+    the same query rows (each over all visible keys). The oracle computes
+    them as one block's share of the gradient (attention_bwd_block) from the
+    head's exact LSE and Delta = rowsum(dO * O)."""
+    import numpy as np
+    w = WORKLOADS["bf16_L32000_cp4_fwdbwd"]
+    q, k, v = make_qkv(w, "cuda", seed=0)
+    do = make_tensor(q.shape, q.dtype, "cuda", seed=1)
+    dq, dk, dv = _run_bwd(rattn, q, k, v, do, w.cp, w.layout, True)
+    h, L = w.H - 1, w.L
+    c = L // (2 * w.cp)
+    rng = np.random.default_rng(5)
+    idx = sorted(set([j for ch in range(2 * w.cp) for j in (*range(ch * c, ch * c + 4), *range((ch + 1) * c - 4,
+                                                                                          (ch + 1) * c))] +
+                     rng.choice(L, 128, replace=False).tolist()))
+    idx = np.asarray(idx)
+    qh, kh, vh, doh = to64(q[0, h]), to64(k[0, h]), to64(v[0, h]), to64(do[0, h])
+    o_ref, lse_ref = oracle.attention(qh, kh, vh, w.scale, True, row_block=1024)
+    delta = (doh * o_ref).sum(-1)
+    allpos = np.arange(L)
+    _, dk_ref, dv_ref = oracle.attention_bwd_block(qh, kh[idx], vh[idx], doh, lse_ref, delta, w.scale, True,
+                                                   q_pos=allpos, kv_pos=idx)
+    dq_ref, _, _ = oracle.attention_bwd_block(qh[idx], kh, vh, doh[idx], lse_ref[idx], delta[idx], w.scale, True,
+                                              q_pos=idx, kv_pos=allpos)
+    check_grad(dk[0, h][idx].float().cpu().numpy(), dk_ref)
+    check_grad(dv[0, h][idx].float().cpu().numpy(), dv_ref)
+    check_grad(dq[0, h][idx].float().cpu().numpy(), dq_ref)

@@ -25,21 +25,22 @@ def _bits(t):
 @pytest.mark.parametrize("dtype,D", [(torch.bfloat16, 128), (torch.float32, 64)])
 @pytest.mark.parametrize("layout", [0, 1, 2])
 @pytest.mark.parametrize("cu,cp", [([0, 5, 16, 16, 23], 2), ([0, 300, 301, 1000], 4), ([0, 64], 1)])
-def test_gather_scatter_bit_exact(rattn, dtype, D, layout, cu, cp):
+@pytest.mark.parametrize("align", [1, 128])
+def test_gather_scatter_bit_exact(rattn, dtype, D, layout, cu, cp, align):
     T = cu[-1]
     x = make_tensor((2, 3, T, D), dtype, "cuda", seed=T + cp)
-    plan = rattn.cp_layout_varlen_plan(cu, cp, layout)
+    plan = rattn.cp_layout_varlen_plan(cu, cp, layout, align)
     src = plan["src"].cuda()
     y = rattn.cp_layout_gather(x, src)
-    y_ref = oracle.varlen_permute(_bits(x), cu, cp, layout)
+    y_ref = oracle.varlen_permute(_bits(x), cu, cp, layout, align)
     assert np.array_equal(_bits(y), y_ref)
     back = rattn.cp_layout_scatter(y, src, T)
     assert np.array_equal(_bits(back), _bits(x))
 
 
-def _run(rattn, q, k, v, do, cu, cp, layout, causal):
+def _run(rattn, q, k, v, do, cu, cp, layout, causal, align=1):
     T = cu[-1]
-    plan = rattn.cp_layout_varlen_plan(cu, cp, layout)
+    plan = rattn.cp_layout_varlen_plan(cu, cp, layout, align)
     src, gkey, segid = (plan[n].cuda() for n in ("src", "gkey", "segid"))
     qp, kp, vp, dop = (rattn.cp_layout_gather(t, src) for t in (q, k, v, do))
     scale = q.shape[-1] ** -0.5
@@ -69,14 +70,15 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("align", [1, 128])
 @pytest.mark.parametrize("case", CASES)
-def test_ring_varlen_fwd_bwd_per_sequence(rattn, case):
+def test_ring_varlen_fwd_bwd_per_sequence(rattn, case, align):
     dtype, D, cu, cp, layout, causal, H, H_kv = case
     T = cu[-1]
     q = make_tensor((1, H, T, D), dtype, "cuda", seed=81)
     k, v = (make_tensor((1, H_kv, T, D), dtype, "cuda", seed=s) for s in (82, 83))
     do = make_tensor((1, H, T, D), dtype, "cuda", seed=84)
-    (o, dq, dk, dv), lse = _run(rattn, q, k, v, do, cu, cp, layout, causal)
+    (o, dq, dk, dv), lse = _run(rattn, q, k, v, do, cu, cp, layout, causal, align)
     scale = D ** -0.5
     for i in range(len(cu) - 1):
         a, b = cu[i], cu[i + 1]
@@ -93,10 +95,12 @@ def test_ring_varlen_fwd_bwd_per_sequence(rattn, case):
         check_grad(dv[..., a:b, :].float().cpu().numpy(), oracle.gqa_reduce(dve, H_kv))
 
 
-def test_ring_varlen_32k_pack(rattn):
+@pytest.mark.parametrize("align", [1, 128])
+def test_ring_varlen_32k_pack(rattn, align):
     """A 32,000-token pack of 24 documents of mixed lengths (64 to 3000
-    tokens), 8 heads, D = 128, cp = 4 head-tail, causal: every sequence of
-    heads 0 and 7 against the oracle, forward and backward."""
+    tokens), 8 heads, D = 128, cp = 4 head-tail, causal, in the plain and the
+    tile-aligned packed layout: every sequence of heads 0 and 7 against the
+    oracle, forward and backward."""
     g = np.random.default_rng(7)
     lens = g.integers(64, 3000, 23)
     lens = np.append(lens, 32000 - lens.sum()) if lens.sum() < 32000 else lens
@@ -106,7 +110,7 @@ def test_ring_varlen_32k_pack(rattn):
         cu.append(32000)
     H, D, cp = 8, 128, 4
     q, k, v, do = (make_tensor((1, H, 32000, D), torch.bfloat16, "cuda", seed=s) for s in (91, 92, 93, 94))
-    (o, dq, dk, dv), lse = _run(rattn, q, k, v, do, cu, cp, 1, True)
+    (o, dq, dk, dv), lse = _run(rattn, q, k, v, do, cu, cp, 1, True, align)
     scale = D ** -0.5
     for h in (0, 7):
         for i in range(len(cu) - 1):

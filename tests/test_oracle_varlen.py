@@ -125,3 +125,59 @@ def test_invalid_pack():
         oracle.varlen_index([0, 5, 3], 2, oracle.HEAD_TAIL)
     with pytest.raises(ValueError):
         oracle.varlen_index([1, 5], 2, oracle.HEAD_TAIL)
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("cp", [1, 2, 3, 4])
+@pytest.mark.parametrize("align", [1, 4, 8, 128])
+@pytest.mark.parametrize("cu", PACKS)
+def test_aligned_shares(layout, cp, align, cu):
+    """With align, every sequence's share of every rank slice starts and ends
+    on a multiple of align rows; its real rows are those of the unaligned
+    layout, in order, followed only by pad rows; gkey still increases along
+    every slice, and align = 1 is the unaligned layout."""
+    Tp, src, pos, seg, gkey = oracle.varlen_index(cu, cp, layout, align)
+    T1, src1, pos1, seg1, gkey1 = oracle.varlen_index(cu, cp, layout)
+    if align == 1:
+        assert Tp == T1 and all(np.array_equal(a, b) for a, b in ((src, src1), (pos, pos1), (seg, seg1),
+                                                                  (gkey, gkey1)))
+    n, n1 = Tp // cp, T1 // cp
+    assert Tp % cp == 0
+    for r in range(cp):
+        sl, sl1 = slice(r * n, (r + 1) * n), slice(r * n1, (r + 1) * n1)
+        off = off1 = 0
+        for i in range(len(cu) - 1):
+            m1 = oracle.padded_len(cu[i + 1] - cu[i], cp, layout) // cp
+            m = -(-m1 // align) * align
+            assert off % align == 0
+            assert np.array_equal(src[sl][off:off + m1], src1[sl1][off1:off1 + m1])
+            assert np.array_equal(pos[sl][off:off + m1], pos1[sl1][off1:off1 + m1])
+            assert np.all(src[sl][off + m1:off + m] == -1) and np.all(seg[sl][off + m1:off + m] == -1)
+            assert np.all(pos[sl][off + m1:off + m] >= cp * m1)   # past every position of the sequence
+            off += m
+            off1 += m1
+        assert off == n
+        assert np.all(np.diff(gkey[sl]) > 0)
+    assert sorted(src[src >= 0].tolist()) == list(range(cu[-1]))
+
+
+@pytest.mark.parametrize("align", [8, 128])
+def test_aligned_pack_attention_is_per_sequence_attention(align):
+    """The aligned layout changes only padding: attention over the permuted
+    pack with its segment mask, put back in pack order, is still per-sequence
+    attention (forward and gradient)."""
+    cu = [0, 30, 33, 100]
+    cp = 2
+    rng = np.random.default_rng(11)
+    q, k, v, do = (rng.standard_normal((1, 2, cu[-1], 4)) for _ in range(4))
+    Tp, src, pos, seg, gkey = oracle.varlen_index(cu, cp, oracle.HEAD_TAIL, align)
+    qp, kp, vp, dop = (oracle.varlen_permute(x, cu, cp, oracle.HEAD_TAIL, align) for x in (q, k, v, do))
+    segk = np.where(seg >= 0, seg, -1)
+    o, _ = oracle.attention(qp, kp, vp, 0.5, True, gkey, gkey, None, q_seg=seg, kv_seg=segk)
+    g = oracle.attention_bwd(qp, kp, vp, dop, 0.5, True, gkey, gkey, None, q_seg=seg, kv_seg=segk)
+    o_ref = np.concatenate(_per_sequence(lambda a, b, c: oracle.attention(a, b, c, 0.5, True)[0], cu, q, k, v), -2)
+    np.testing.assert_allclose(oracle.varlen_unpermute(o, cu, cp, oracle.HEAD_TAIL, align), o_ref, atol=1e-12)
+    g_ref = _per_sequence(lambda a, b, c, d: oracle.attention_bwd(a, b, c, d, 0.5, True), cu, q, k, v, do)
+    for j in range(3):
+        want = np.concatenate([x[j] for x in g_ref], -2)
+        np.testing.assert_allclose(oracle.varlen_unpermute(g[j], cu, cp, oracle.HEAD_TAIL, align), want, atol=1e-12)
