@@ -1,6 +1,7 @@
 // api.cu -- the C ABI entry points declared in include/rattn.h: host-side
 // argument validation (nothing is launched on a bad argument), dispatch to
 // the kernels, the device error word and the TMA descriptor helper.
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -19,6 +20,7 @@ constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultWaitNs = 4000000000ull;
 
 std::mutex g_mu;
+std::atomic<int> g_fwd_tiling{0};
 int* g_err_ptr[kMaxDevices] = {nullptr};
 unsigned long long g_wait_ns[kMaxDevices] = {0};
 std::set<std::pair<const void*, int>> g_smem_done;
@@ -78,6 +80,7 @@ rattn_status get_dev_ctx(DevCtx* out) {
   }
   out->err_word = g_err_ptr[dev];
   out->wait_ns = g_wait_ns[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
+  out->fwd_tiling = g_fwd_tiling.load();
   return RATTN_OK;
 }
 
@@ -596,6 +599,12 @@ rattn_status rattn_get_device_error(int* site) {
     if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return RATTN_ERR_CUDA;
     return v >= SITE_BOUNDS ? RATTN_ERR_BOUNDS : RATTN_ERR_TIMEOUT;
   }
+  return RATTN_OK;
+}
+
+rattn_status rattn_set_fwd_tiling(int mode) {
+  if (mode < 0 || mode > 2) return RATTN_ERR_INVALID_ARG;
+  g_fwd_tiling.store(mode);
   return RATTN_OK;
 }
 

@@ -610,7 +610,16 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
 
 }  // namespace
 
+// Two query tiles per CTA (attn_fwd_pair_sm100.cu) halve the K/V traffic per
+// FLOP but serialise each tile's score -> softmax -> product chain (one TMEM
+// score buffer per tile); on B200 that tiling is the faster one only for long
+// rows, whose launches run long enough to be held at the power-capped clock.
+constexpr long long kPairMinKeys = 262144;
+
 rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx) {
+  const bool pair = ctx.fwd_tiling == 2 ||
+                    (ctx.fwd_tiling == 0 && static_cast<long long>(a.nseg) * a.Lk_seg >= kPairMinKeys);
+  if (pair) return launch_fwd_sm100_pair(a, ctx);
   if (a.D == 128) return launch<128>(a, ctx);
   if (a.D == 64) return launch<64>(a, ctx);
   return RATTN_ERR_UNSUPPORTED;

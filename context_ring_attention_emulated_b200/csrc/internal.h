@@ -15,6 +15,7 @@ namespace rattn {
 struct DevCtx {
   int* err_word;
   unsigned long long wait_ns;
+  int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two (rattn_set_fwd_tiling)
 };
 rattn_status get_dev_ctx(DevCtx* out);
 
@@ -76,6 +77,7 @@ struct FwdArgs {
   cudaStream_t stream;
 };
 rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx);
+rattn_status launch_fwd_sm100_pair(const FwdArgs& a, const DevCtx& ctx);  // two query tiles per CTA
 rattn_status launch_fwd_simt(const FwdArgs& a);
 
 struct BwdArgs {

@@ -63,6 +63,7 @@ SIGNATURES = [
                                _P, _P, _P, _I, _P]),
     ("rattn_grad_fold", _I, [_P, _P, _I64, _P]),
     ("rattn_get_device_error", _I, [ctypes.POINTER(_I)]),
+    ("rattn_set_fwd_tiling", _I, [_I]),
     ("rattn_set_wait_limit_ns", _I, [ctypes.c_ulonglong]),
 ]
 
@@ -565,6 +566,11 @@ def rattn_get_device_error():
     site = ctypes.c_int(0)
     code = lib.rattn_get_device_error(ctypes.byref(site))
     return code, site.value
+
+
+def rattn_set_fwd_tiling(mode):
+    """0: automatic (by row length), 1: one query tile per CTA, 2: two."""
+    _check("rattn_set_fwd_tiling", lib.rattn_set_fwd_tiling(int(mode)))
 
 
 def rattn_set_wait_limit_ns(ns):

@@ -396,6 +396,15 @@ rattn_status rattn_ring_bwd_noalloc(const void* q, const void* k, const void* v,
  * address is stale). */
 rattn_status rattn_get_device_error(int* site);
 
+/* Tuning and test hook: how the bf16 attention forward (ring, GQA, packed and
+ * partial calls) tiles the queries, for launches made after the call, on
+ * every device. 0 (the default) chooses by row length: two 128-row query
+ * tiles per CTA, sharing each staged K/V tile, when a query row attends at
+ * least 262,144 keys (cp_size x slice length), else one. 1 forces one tile
+ * per CTA, 2 forces two. Both give bit-identical O and LSE. Returns
+ * RATTN_ERR_INVALID_ARG for any other mode. */
+rattn_status rattn_set_fwd_tiling(int mode);
+
 /* Test hook: the per-wait time limit in nanoseconds used by subsequent
  * launches on the current device (default 4e9; 0 restores the default). A
  * tiny limit makes waits give

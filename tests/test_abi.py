@@ -45,6 +45,13 @@ def test_debug_build_compiles_and_exports_every_symbol():
         assert hasattr(lib, n), f"{n} missing from the debug build"
 
 
+def test_fwd_tiling_hook_rejects_unknown_modes(rattn):
+    for mode in (-1, 3, 7):
+        assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.ERR_INVALID_ARG
+    for mode in (1, 2, 0):
+        assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.OK
+
+
 def test_status_strings(rattn):
     for code, name in enumerate(["RATTN_OK", "RATTN_ERR_INVALID_ARG", "RATTN_ERR_UNSUPPORTED", "RATTN_ERR_CUDA",
                                  "RATTN_ERR_TIMEOUT", "RATTN_ERR_BOUNDS"]):

@@ -1,0 +1,106 @@
+"""The two tilings of the bf16 attention forward (one 128-row query tile per
+CTA, or two sharing each staged K/V tile) against each other and the oracle.
+
+The library picks the tiling by row length; rattn_set_fwd_tiling forces one.
+Both evaluate every row's online softmax over the same key tiles in the same
+order with the same arithmetic, so O and LSE must be bit-identical; the
+two-tile results are also checked against the oracle at the bf16 tolerances.
+Cases cover odd tile counts (the last pair has no second tile), ragged and
+padded lengths, both masks, the striped and contiguous layouts, D = 64,
+grouped key/value heads, packed sequences and the partial (one block) call."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from context_ring_attention_emulated_b200.workloads import make_tensor
+from tests.gpu_common import check_lse, check_o, load_rattn, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rattn():
+    r = load_rattn()
+    yield r
+    r.rattn_set_fwd_tiling(0)
+
+
+def _both(rattn, fn):
+    outs = []
+    for mode in (1, 2):
+        rattn.rattn_set_fwd_tiling(mode)
+        outs.append([t.clone() for t in fn()])
+        torch.cuda.synchronize()
+        assert rattn.rattn_get_device_error()[0] == rattn.OK
+    rattn.rattn_set_fwd_tiling(0)
+    for a, b in zip(*outs):
+        assert torch.equal(a, b), "the two tilings differ"
+    return outs[1]
+
+
+RING = [
+    # B, H, H_kv, L, D, cp, layout, causal
+    (1, 2, 2, 1000, 128, 2, 1, True),     # 500-row slices: 4 tiles, a ragged last one
+    (1, 4, 2, 2000, 128, 4, 1, True),     # GQA
+    (2, 2, 2, 777, 64, 3, 1, True),       # padded to 780, 3 tiles a slice, D = 64
+    (1, 2, 1, 1500, 128, 4, 2, True),     # striped, MQA, 3 tiles a slice
+    (1, 2, 2, 1300, 128, 2, 0, False),    # contiguous, non-causal
+    (1, 1, 1, 8192, 128, 2, 1, True),     # 32 tiles per slice
+    (1, 2, 2, 1664, 128, 2, 1, True),     # 832-row slices: 7 tiles, an odd count
+    (1, 2, 2, 640, 64, 1, 0, True),       # one rank: 5 tiles, D = 64
+]
+
+
+@pytest.mark.parametrize("case", RING)
+def test_ring_fwd_tilings_agree_and_match_oracle(rattn, case):
+    B, H, H_kv, L, D, cp, layout, causal = case
+    scale = D ** -0.5
+    q = make_tensor((B, H, L, D), torch.bfloat16, "cuda", seed=61)
+    k, v = (make_tensor((B, H_kv, L, D), torch.bfloat16, "cuda", seed=s) for s in (62, 63))
+    qp, pos = rattn.cp_layout_permute(q, cp, layout)
+    kp, _ = rattn.cp_layout_permute(k, cp, layout)
+    vp, _ = rattn.cp_layout_permute(v, cp, layout)
+    fwd = rattn.rattn_ring_fwd_gqa if H_kv != H else rattn.rattn_ring_fwd
+    o, lse = _both(rattn, lambda: fwd(qp, kp, vp, pos, cp, layout, causal, scale, L_valid=L))
+    out = rattn.cp_layout_unpermute(o, L, cp, layout)
+    ke, ve = oracle.gqa_expand(to64(k), H), oracle.gqa_expand(to64(v), H)
+    o_ref, l_ref = oracle.attention(to64(q), ke, ve, scale, causal)
+    check_o(out.float().cpu().numpy(), o_ref, torch.bfloat16)
+    real = pos.cpu().numpy() < L
+    l_ref_p, _ = oracle.permute(l_ref[..., None], cp, layout)
+    check_lse(lse.cpu().numpy()[..., real], l_ref_p[..., 0][..., real], torch.bfloat16)
+
+
+def test_partial_fwd_tilings_agree(rattn):
+    """One block with separate query and key positions, masked pad keys, and
+    an empty key block."""
+    q = make_tensor((1, 2, 700, 128), torch.bfloat16, "cuda", seed=71)
+    k, v = (make_tensor((1, 2, 900, 128), torch.bfloat16, "cuda", seed=s) for s in (72, 73))
+    qpos = np.arange(200, 900, dtype=np.int32)
+    kpos = np.arange(0, 900, dtype=np.int32)
+    qd, kd = torch.from_numpy(qpos).cuda(), torch.from_numpy(kpos).cuda()
+    o, lse = _both(rattn, lambda: rattn.rattn_partial_fwd(q, k, v, qd, kd, causal=True, kv_valid=850))
+    o_ref, l_ref = oracle.attention(to64(q), to64(k), to64(v), 128 ** -0.5, True, qpos, kpos, 850)
+    check_lse(lse.cpu().numpy(), l_ref, torch.bfloat16)
+    check_o(o.cpu().numpy(), o_ref, torch.bfloat16)
+    e_k = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device="cuda")
+    o0, l0 = _both(rattn, lambda: rattn.rattn_partial_fwd(q, e_k, e_k, causal=True))
+    assert torch.all(o0 == 0) and torch.all(torch.isneginf(l0))
+
+
+def test_packed_fwd_tilings_agree(rattn):
+    cu = [0, 5, 300, 301, 1000, 1900]
+    cp = 2
+    plan = rattn.cp_layout_varlen_plan(cu, cp, 1, 128)
+    src, gkey, segid = (plan[n].cuda() for n in ("src", "gkey", "segid"))
+    q, k, v = (make_tensor((1, 2, cu[-1], 128), torch.bfloat16, "cuda", seed=s) for s in (81, 82, 83))
+    qp, kp, vp = (rattn.cp_layout_gather(t, src) for t in (q, k, v))
+    o, lse = _both(rattn, lambda: rattn.rattn_ring_fwd_varlen(qp, kp, vp, gkey, segid, cp, True))
+    out = rattn.cp_layout_scatter(o, src, cu[-1])
+    for a, b in zip(cu, cu[1:]):
+        if a == b:
+            continue
+        o_ref, _ = oracle.attention(to64(q[..., a:b, :]), to64(k[..., a:b, :]), to64(v[..., a:b, :]),
+                                    128 ** -0.5, True)
+        check_o(out[..., a:b, :].float().cpu().numpy(), o_ref, torch.bfloat16)
