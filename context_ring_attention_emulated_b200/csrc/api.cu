@@ -23,6 +23,7 @@ std::mutex g_mu;
 std::atomic<int> g_fwd_tiling{0};
 int* g_err_ptr[kMaxDevices] = {nullptr};
 unsigned long long g_wait_ns[kMaxDevices] = {0};
+int g_sm_count[kMaxDevices] = {0};
 std::set<std::pair<const void*, int>> g_smem_done;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -78,6 +79,13 @@ rattn_status get_dev_ctx(DevCtx* out) {
     if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return RATTN_ERR_CUDA;
     g_err_ptr[dev] = static_cast<int*>(p);
   }
+  if (!g_sm_count[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      return RATTN_ERR_CUDA;
+    g_sm_count[dev] = n;
+  }
+  out->sm_count = g_sm_count[dev];
   out->err_word = g_err_ptr[dev];
   out->wait_ns = g_wait_ns[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
   out->fwd_tiling = g_fwd_tiling.load();

@@ -294,40 +294,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Per hop t the query segment is r = (s + t) mod nseg. Visible query tiles
   // form a range [first_vis, end_vis): positions (and segids for packed
-  // sequences) are non-decreasing in a segment, so both ends are found by
-  // binary search; without packed sequences end_vis = nq_tiles.
+  // sequences) are non-decreasing in a segment, so both ends are partition
+  // points of predicates that hold on a prefix (one warp per hop, 32-way
+  // searches); without packed sequences end_vis = nq_tiles.
   const bool live = k_min < p.kv_valid;
   const int sk_lo = SEG ? segat(p, s, k0) : 0;
   const int sk_hi = SEG ? segat(p, s, k0 + k_rows - 1) : 0;
-  for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
+  for (int t = warp; t < p.nseg; t += kThreads / 32) {
     const int r = (s + t) % p.nseg;
     int first_vis = p.nq_tiles, end_vis = p.nq_tiles;
     if (live) {
-      int lo = 0, hi = p.nq_tiles;
-      while (lo < hi) {  // first tile whose last query may see a key of this tile
-        const int mid = (lo + hi) >> 1;
-        const int last = min((mid + 1) * BQ, q_len<SPLIT>(p)) - 1;
-        const bool reach = (!p.causal || qposat<SPLIT>(p, r, last) >= k_min) && (!SEG || segat(p, r, last) >= sk_lo);
-        if (reach) hi = mid; else lo = mid + 1;
-      }
-      first_vis = lo;
-      hi = p.nq_tiles;
-      if (SEG) {
-        while (lo < hi) {  // first tile wholly past the key tile's last segment
-          const int mid = (lo + hi) >> 1;
-          if (segat(p, r, mid * BQ) > sk_hi) hi = mid; else lo = mid + 1;
-        }
-      } else if (p.causal) {
-        while (lo < hi) {  // first tile whose first query sees every key
-          const int mid = (lo + hi) >> 1;
-          if (qposat<SPLIT>(p, r, mid * BQ) >= k_max) hi = mid; else lo = mid + 1;
-        }
-      } else {
-        lo = first_vis;  // non-causal: every visible tile is unmasked
-      }
-      end_vis = lo;
+      first_vis = warp_partition_point(0, p.nq_tiles, lane, [&](int m) {  // last query sees no key of this tile
+        const int last = min((m + 1) * BQ, q_len<SPLIT>(p)) - 1;
+        return !((!p.causal || qposat<SPLIT>(p, r, last) >= k_min) && (!SEG || segat(p, r, last) >= sk_lo));
+      });
+      if (SEG)  // up to the first tile wholly past the key tile's last segment
+        end_vis = warp_partition_point(first_vis, p.nq_tiles, lane, [&](int m) { return segat(p, r, m * BQ) <= sk_hi; });
+      else if (p.causal)  // up to the first tile whose first query sees every key
+        end_vis = warp_partition_point(first_vis, p.nq_tiles, lane,
+                                       [&](int m) { return qposat<SPLIT>(p, r, m * BQ) < k_max; });
+      else
+        end_vis = first_vis;  // non-causal: every visible tile is unmasked
     }
-    s_hop[t] = make_int2(first_vis, end_vis);
+    if (lane == 0) s_hop[t] = make_int2(first_vis, end_vis);
   }
   tc_fence_before();
   __syncthreads();

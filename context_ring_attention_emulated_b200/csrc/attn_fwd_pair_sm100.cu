@@ -135,61 +135,37 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 // the sub-range with no masked element: x = first visible tile, y = end of
 // the visible tiles, [z, w) = tiles fully visible to every row of the range.
 // Keys are sorted by position (and by segid for packed sequences) within a
-// segment, so every bound is a binary search; without packed sequences the
-// visible tiles are a prefix.
+// segment, so every bound is the partition point of a predicate that holds on
+// a prefix of a tile range; without packed sequences the visible tiles are a
+// prefix. All 32 lanes of a warp call it together.
 template <bool SEG>
-__device__ int4 hop_ranges(const Params& p, int r, int s, int qa, int qb, int nk_tiles) {
+__device__ int4 hop_ranges(const Params& p, int r, int s, int qa, int qb, int nk_tiles, int lane) {
   const long long q_min = qpos(p, r, qa), q_max = qpos(p, r, qb);
   const int sq_lo = SEG ? segat(p, r, qa) : 0;
   const int sq_hi = SEG ? segat(p, r, qb) : 0;
-  int first = 0;
-  if (SEG) {  // first tile whose last key is in the query range's first segment or later
-    int lo = 0, hi = nk_tiles;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (segat(p, s, min((mid + 1) * BN, p.Lk_seg) - 1) >= sq_lo) hi = mid; else lo = mid + 1;
-    }
-    first = lo;
-  }
-  int lo = first, hi = nk_tiles;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    const long long kmin = kpos(p, s, mid * BN);
-    const bool vis = kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!SEG || segat(p, s, mid * BN) <= sq_hi);
-    if (vis) lo = mid + 1; else hi = mid;
-  }
-  const int n_vis = lo;
+  const int first = SEG ? warp_partition_point(0, nk_tiles, lane, [&](int m) {
+    return segat(p, s, min((m + 1) * BN, p.Lk_seg) - 1) < sq_lo;  // tile ends before the query segments
+  }) : 0;
+  const int n_vis = warp_partition_point(first, nk_tiles, lane, [&](int m) {
+    const long long kmin = kpos(p, s, m * BN);
+    return kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!SEG || segat(p, s, m * BN) <= sq_hi);
+  });
   int f_lo = first, f_hi = first;
   const bool one_seg = !SEG || (sq_lo == sq_hi && (sq_lo & 1) == 0);
   if (one_seg && first < n_vis) {
     int a = first, b = n_vis;
     if (SEG) {  // tiles lying wholly in the query range's segment: [a, b)
-      lo = first;
-      hi = n_vis;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (segat(p, s, mid * BN) >= sq_lo) hi = mid; else lo = mid + 1;
-      }
-      a = lo;
-      lo = a;
-      hi = n_vis;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (segat(p, s, min((mid + 1) * BN, p.Lk_seg) - 1) > sq_lo) hi = mid; else lo = mid + 1;
-      }
-      b = lo;
-    }
-    lo = a;
-    hi = b;
-    while (lo < hi) {  // leading tiles of [a, b) visible to every query row
-      const int mid = (lo + hi) >> 1;
-      const bool complete = (mid + 1) * BN <= p.Lk_seg;
-      const long long kmax = kpos(p, s, min((mid + 1) * BN, p.Lk_seg) - 1);
-      const bool full = complete && kmax < p.kv_valid && (!p.causal || kmax <= q_min);
-      if (full) lo = mid + 1; else hi = mid;
+      a = warp_partition_point(first, n_vis, lane, [&](int m) { return segat(p, s, m * BN) < sq_lo; });
+      b = warp_partition_point(a, n_vis, lane, [&](int m) {
+        return segat(p, s, min((m + 1) * BN, p.Lk_seg) - 1) <= sq_lo;
+      });
     }
     f_lo = a;
-    f_hi = lo;
+    f_hi = warp_partition_point(a, b, lane, [&](int m) {  // leading tiles visible to every query row
+      const bool complete = (m + 1) * BN <= p.Lk_seg;
+      const long long kmax = kpos(p, s, min((m + 1) * BN, p.Lk_seg) - 1);
+      return complete && kmax < p.kv_valid && (!p.causal || kmax <= q_min);
+    });
   }
   return make_int4(first, n_vis, f_lo, f_hi);
 }
@@ -228,14 +204,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  // Work item: (batch, head) slowest, so the CTAs resident at any time share
-  // one head's K/V in L2; within a head the heaviest tile pairs (largest
-  // local index, hence largest positions under every layout) go first.
+  // Work item: (batch, head) slowest, then rank, then tile pair, heaviest
+  // first (largest local index, hence largest positions under every layout):
+  // the CTAs resident at any time walk the same hop's K/V block together.
   int item = blockIdx.x;
-  const int r = item % p.nseg;
-  item /= p.nseg;
   const int pq = p.n_pairs - 1 - (item % p.n_pairs);
-  const int bh = item / p.n_pairs;
+  item /= p.n_pairs;
+  const int r = item % p.nseg;
+  const int bh = item / p.nseg;
   const int kvh = bh / p.group;  // (batch, key/value head): query heads of a group are contiguous
   const int qa0 = pq * 2 * BM;                             // first row of Q0
   const int rows0 = min(BM, p.Lq_seg - qa0);
@@ -265,13 +241,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 1) tmem_alloc(s_tmem, C::T_COLS);
 
-  for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
+  for (int t = warp; t < p.nseg; t += kThreads / 32) {  // one warp per hop
     const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
-    const int4 all = hop_ranges<SEG>(p, r, s, qa0, q_last, nk_tiles);
-    const int4 h0 = hop_ranges<SEG>(p, r, s, qa0, qa0 + rows0 - 1, nk_tiles);
-    const int4 h1 = rows1 > 0 ? hop_ranges<SEG>(p, r, s, qa0 + BM, q_last, nk_tiles) : make_int4(0, 0, 0, 0);
-    s_hop[t] = make_int4(all.x, all.y, h0.z, h0.w);
-    s_hop1[t] = h1;
+    const int4 all = hop_ranges<SEG>(p, r, s, qa0, q_last, nk_tiles, lane);
+    const int4 h0 = hop_ranges<SEG>(p, r, s, qa0, qa0 + rows0 - 1, nk_tiles, lane);
+    const int4 h1 = rows1 > 0 ? hop_ranges<SEG>(p, r, s, qa0 + BM, q_last, nk_tiles, lane) : make_int4(0, 0, 0, 0);
+    if (lane == 0) {
+      s_hop[t] = make_int4(all.x, all.y, h0.z, h0.w);
+      s_hop1[t] = h1;
+    }
   }
   tc_fence_before();
   __syncthreads();

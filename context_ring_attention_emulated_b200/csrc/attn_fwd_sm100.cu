@@ -150,14 +150,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work item: (batch, head) slowest, so the CTAs resident at any time share
-  // one head's K/V in L2; within a head the heaviest query tiles (largest
-  // local index, hence largest positions under every layout) go first.
+  // Work item: (batch, head) slowest, then rank, then query tile, heaviest
+  // first (largest local index, hence largest positions under every layout).
+  // The CTAs resident at any time then belong to one rank of one head and
+  // walk the same hop's K/V block at about the same time, so the block is
+  // read from HBM about once per wave even when a head's K/V exceed L2.
   int item = blockIdx.x;
-  const int r = item % p.nseg;
-  item /= p.nseg;
   const int qt = p.n_qtiles - 1 - (item % p.n_qtiles);
-  const int bh = item / p.n_qtiles;
+  item /= p.n_qtiles;
+  const int r = item % p.nseg;
+  const int bh = item / p.nseg;
   const int kvh = bh / p.group;  // (batch, key/value head): query heads of a group are contiguous
   const int q0 = qt * BM;
   const int q_rows = min(BM, p.Lq_seg - q0);
@@ -187,62 +189,39 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Per hop: the K/V tiles not fully masked form a range [first, n_vis) and
   // the tiles with no masked element a range [f_lo, f_hi) inside it; keys are
   // sorted by position (and by segid for packed sequences) within a segment,
-  // so every bound is found by binary search. Without packed sequences the
-  // visible tiles are a prefix.
-  for (int t = threadIdx.x; t < p.nseg; t += kThreads) {
+  // so every bound is the partition point of a predicate that holds on a
+  // prefix of a tile range. Without packed sequences the visible tiles are a
+  // prefix. One warp per hop, 32-way searches (two rounds of loads for up to
+  // 1024 tiles).
+  for (int t = warp; t < p.nseg; t += kThreads / 32) {
     const int s = ((r - t) % p.nseg + p.nseg) % p.nseg;
     const int sq_lo = SEG ? segat(p, r, q0) : 0;
     const int sq_hi = SEG ? segat(p, r, q0 + q_rows - 1) : 0;
-    int first = 0;
-    if (SEG) {  // first tile whose last key is in the query tile's first segment or later
-      int lo = 0, hi = nk_tiles;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (segat(p, s, min((mid + 1) * BN, p.Lk_seg) - 1) >= sq_lo) hi = mid; else lo = mid + 1;
-      }
-      first = lo;
-    }
-    int lo = first, hi = nk_tiles;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      const long long kmin = kpos(p, s, mid * BN);
-      const bool vis = kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!SEG || segat(p, s, mid * BN) <= sq_hi);
-      if (vis) lo = mid + 1; else hi = mid;
-    }
-    const int n_vis = lo;
+    const int first = SEG ? warp_partition_point(0, nk_tiles, lane, [&](int m) {
+      return segat(p, s, min((m + 1) * BN, p.Lk_seg) - 1) < sq_lo;  // tile ends before the query segments
+    }) : 0;
+    const int n_vis = warp_partition_point(first, nk_tiles, lane, [&](int m) {
+      const long long kmin = kpos(p, s, m * BN);
+      return kmin < p.kv_valid && (!p.causal || kmin <= q_max) && (!SEG || segat(p, s, m * BN) <= sq_hi);
+    });
     int f_lo = first, f_hi = first;
     const bool one_seg = !SEG || (sq_lo == sq_hi && (sq_lo & 1) == 0);
     if (one_seg && first < n_vis) {
       int a = first, b = n_vis;
       if (SEG) {  // tiles lying wholly in the query tile's segment: [a, b)
-        lo = first;
-        hi = n_vis;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (segat(p, s, mid * BN) >= sq_lo) hi = mid; else lo = mid + 1;
-        }
-        a = lo;
-        lo = a;
-        hi = n_vis;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (segat(p, s, min((mid + 1) * BN, p.Lk_seg) - 1) > sq_lo) hi = mid; else lo = mid + 1;
-        }
-        b = lo;
-      }
-      lo = a;
-      hi = b;
-      while (lo < hi) {  // leading tiles of [a, b) visible to every query row
-        const int mid = (lo + hi) >> 1;
-        const bool complete = (mid + 1) * BN <= p.Lk_seg;
-        const long long kmax = kpos(p, s, min((mid + 1) * BN, p.Lk_seg) - 1);
-        const bool full = complete && kmax < p.kv_valid && (!p.causal || kmax <= q_min);
-        if (full) lo = mid + 1; else hi = mid;
+        a = warp_partition_point(first, n_vis, lane, [&](int m) { return segat(p, s, m * BN) < sq_lo; });
+        b = warp_partition_point(a, n_vis, lane, [&](int m) {
+          return segat(p, s, min((m + 1) * BN, p.Lk_seg) - 1) <= sq_lo;
+        });
       }
       f_lo = a;
-      f_hi = lo;
+      f_hi = warp_partition_point(a, b, lane, [&](int m) {  // leading tiles visible to every query row
+        const bool complete = (m + 1) * BN <= p.Lk_seg;
+        const long long kmax = kpos(p, s, min((m + 1) * BN, p.Lk_seg) - 1);
+        return complete && kmax < p.kv_valid && (!p.causal || kmax <= q_min);
+      });
     }
-    s_hop[t] = make_int4(first, n_vis, f_lo, f_hi);
+    if (lane == 0) s_hop[t] = make_int4(first, n_vis, f_lo, f_hi);
   }
   tc_fence_before();
   __syncthreads();
@@ -610,10 +589,12 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
 
 }  // namespace
 
-// Two query tiles per CTA (attn_fwd_pair_sm100.cu) halve the K/V traffic per
-// FLOP but serialise each tile's score -> softmax -> product chain (one TMEM
-// score buffer per tile); on B200 that tiling is the faster one only for long
-// rows, whose launches run long enough to be held at the power-capped clock.
+// Two query tiles per CTA (attn_fwd_pair_sm100.cu) halve the K/V bytes moved
+// from L2 into shared memory per FLOP but serialise each tile's score ->
+// softmax -> product chain (one TMEM score buffer per tile). Measured on B200
+// (causal, D = 128): one tile is faster up to 131,072 keys per row, two from
+// 262,144 keys on, where one head's K and V (L x D x 4 bytes) outgrow L2 and
+// the launches run long enough to be held at the power-capped clock.
 constexpr long long kPairMinKeys = 262144;
 
 rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx) {

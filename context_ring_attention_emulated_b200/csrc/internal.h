@@ -16,6 +16,7 @@ struct DevCtx {
   int* err_word;
   unsigned long long wait_ns;
   int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two (rattn_set_fwd_tiling)
+  int sm_count;    // multiprocessors of the device (persistent grids)
 };
 rattn_status get_dev_ctx(DevCtx* out);
 

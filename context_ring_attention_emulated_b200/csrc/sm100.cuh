@@ -169,6 +169,26 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 // Waits until every bulk group this thread committed has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// First index of [lo, hi) at which a predicate that holds on a prefix of the
+// range turns false (hi if it never does). All 32 lanes call it together and
+// probe 32 evenly spaced indices per level, so the answer takes
+// ceil(log32(hi - lo)) rounds of independent loads instead of log2(hi - lo)
+// dependent ones.
+template <class Pred>
+__device__ __forceinline__ int warp_partition_point(int lo, int hi, int lane, Pred pred) {
+  while (lo < hi) {
+    const int step = (hi - lo + 31) >> 5;
+    const int m = lo + lane * step;
+    const bool t = m < hi && pred(m);
+    const int c = __popc(__ballot_sync(0xffffffffu, t));  // the true probes are a prefix
+    if (c == 0) return lo;
+    const int next_hi = min(hi, lo + c * step);
+    lo += (c - 1) * step + 1;
+    hi = next_hi;
+  }
+  return lo;
+}
+
 // Named barrier over `count` threads (a multiple of 32) that also returns,
 // to every participant, whether any of them passed pred = true.
 __device__ __forceinline__ bool bar_any(int id, int count, bool pred) {

@@ -37,6 +37,9 @@ PARTIAL_CASES = [
     (torch.float32, 64, 200, 333, True, True, None),
     (torch.float32, 128, 65, 97, False, False, 50),
     (torch.float32, 36, 33, 40, True, True, None),
+    # more than 1024 key tiles: the tile-range searches take three rounds
+    (torch.bfloat16, 64, 256, 140000, True, True, None),
+    (torch.bfloat16, 128, 200, 140000, False, True, 100000),
 ]
 
 

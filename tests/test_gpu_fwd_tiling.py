@@ -89,6 +89,20 @@ def test_partial_fwd_tilings_agree(rattn):
     assert torch.all(o0 == 0) and torch.all(torch.isneginf(l0))
 
 
+def test_partial_fwd_tilings_agree_on_long_key_blocks(rattn):
+    """More than 1024 key tiles per block (three rounds of the tile-range
+    searches), causal with the query rows in the middle of the keys."""
+    q = make_tensor((1, 1, 300, 64), torch.bfloat16, "cuda", seed=74)
+    k, v = (make_tensor((1, 1, 140000, 64), torch.bfloat16, "cuda", seed=s) for s in (75, 76))
+    qpos = np.arange(70000, 70300, dtype=np.int32)
+    kpos = np.arange(0, 140000, dtype=np.int32)
+    qd, kd = torch.from_numpy(qpos).cuda(), torch.from_numpy(kpos).cuda()
+    o, lse = _both(rattn, lambda: rattn.rattn_partial_fwd(q, k, v, qd, kd, causal=True))
+    o_ref, l_ref = oracle.attention(to64(q), to64(k), to64(v), 64 ** -0.5, True, qpos, kpos)
+    check_lse(lse.cpu().numpy(), l_ref, torch.bfloat16)
+    check_o(o.cpu().numpy(), o_ref, torch.bfloat16)
+
+
 def test_packed_fwd_tilings_agree(rattn):
     cu = [0, 5, 300, 301, 1000, 1900]
     cp = 2

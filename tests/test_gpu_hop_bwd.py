@@ -56,6 +56,7 @@ CASES = [
     (128, 2, 1, (np.arange(129), np.arange(257)), True, None),                 # MQA, ragged tails, causal cut
     (64, 2, 2, (np.arange(200), np.arange(190, 450)), False, 400),             # non-causal, pad keys masked
     (128, 1, 1, (np.arange(0, 100), np.arange(500, 900)), True, None),         # keys all in the future
+    (64, 1, 1, (np.arange(0, 140000), np.arange(70000, 70300)), True, None),  # 1094 query tiles: 3-round searches
 ]
 
 
