@@ -13,6 +13,7 @@ namespace rattn {
 
 // Device-side error word written by kernels whose bounded waits gave up.
 __device__ int g_err_word;
+__device__ unsigned int g_work[kWorkSlots * 2];  // zero at load; see DevCtx::work
 
 namespace {
 
@@ -24,6 +25,8 @@ std::atomic<int> g_fwd_tiling{0};
 int* g_err_ptr[kMaxDevices] = {nullptr};
 unsigned long long g_wait_ns[kMaxDevices] = {0};
 int g_sm_count[kMaxDevices] = {0};
+unsigned int* g_work_ptr[kMaxDevices] = {nullptr};
+std::atomic<unsigned> g_work_next{0};
 std::set<std::pair<const void*, int>> g_smem_done;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -85,7 +88,13 @@ rattn_status get_dev_ctx(DevCtx* out) {
       return RATTN_ERR_CUDA;
     g_sm_count[dev] = n;
   }
+  if (!g_work_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_work) != cudaSuccess) return RATTN_ERR_CUDA;
+    g_work_ptr[dev] = static_cast<unsigned int*>(p);
+  }
   out->sm_count = g_sm_count[dev];
+  out->work = g_work_ptr[dev] + 2 * (g_work_next.fetch_add(1) % kWorkSlots);
   out->err_word = g_err_ptr[dev];
   out->wait_ns = g_wait_ns[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
   out->fwd_tiling = g_fwd_tiling.load();
@@ -611,7 +620,7 @@ rattn_status rattn_get_device_error(int* site) {
 }
 
 rattn_status rattn_set_fwd_tiling(int mode) {
-  if (mode < 0 || mode > 2) return RATTN_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 3) return RATTN_ERR_INVALID_ARG;
   g_fwd_tiling.store(mode);
   return RATTN_OK;
 }

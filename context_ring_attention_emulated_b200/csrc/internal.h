@@ -15,9 +15,15 @@ namespace rattn {
 struct DevCtx {
   int* err_word;
   unsigned long long wait_ns;
-  int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two (rattn_set_fwd_tiling)
+  int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two, 3 persistent (rattn_set_fwd_tiling)
   int sm_count;    // multiprocessors of the device (persistent grids)
+  // A pair of work counters for one persistent launch (next work item, CTAs
+  // finished), zero when the launch starts; its last CTA zeroes them again.
+  // Each context fetch takes the next of kWorkSlots pairs, so launches in
+  // flight on different streams use different pairs.
+  unsigned int* work;
 };
+constexpr int kWorkSlots = 256;
 rattn_status get_dev_ctx(DevCtx* out);
 
 // Wait sites recorded in the error word.
@@ -79,6 +85,7 @@ struct FwdArgs {
 };
 rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx);
 rattn_status launch_fwd_sm100_pair(const FwdArgs& a, const DevCtx& ctx);  // two query tiles per CTA
+rattn_status launch_fwd_sm100_persist(const FwdArgs& a, const DevCtx& ctx);  // persistent, one tile per item
 rattn_status launch_fwd_simt(const FwdArgs& a);
 
 struct BwdArgs {

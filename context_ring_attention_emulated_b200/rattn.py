@@ -569,7 +569,7 @@ def rattn_get_device_error():
 
 
 def rattn_set_fwd_tiling(mode):
-    """0: automatic (by row length), 1: one query tile per CTA, 2: two."""
+    """0: automatic, 1: one query tile per CTA, 2: two, 3: persistent (one tile per work item)."""
     _check("rattn_set_fwd_tiling", lib.rattn_set_fwd_tiling(int(mode)))
 
 

@@ -398,10 +398,12 @@ rattn_status rattn_get_device_error(int* site);
 
 /* Tuning and test hook: how the bf16 attention forward (ring, GQA, packed and
  * partial calls) tiles the queries, for launches made after the call, on
- * every device. 0 (the default) chooses by row length: two 128-row query
- * tiles per CTA, sharing each staged K/V tile, when a query row attends at
- * least 262,144 keys (cp_size x slice length), else one. 1 forces one tile
- * per CTA, 2 forces two. Both give bit-identical O and LSE. Returns
+ * every device. 0 (the default) chooses: two 128-row query tiles per CTA,
+ * sharing each staged K/V tile, when a query row attends at least 262,144
+ * keys (cp_size x slice length); else, for packed sequences, a persistent
+ * kernel (one CTA per SM taking one-tile work items from a per-launch
+ * counter); else one tile per CTA. 1 forces one tile per CTA, 2 two, 3 the
+ * persistent kernel. All give bit-identical O and LSE. Returns
  * RATTN_ERR_INVALID_ARG for any other mode. */
 rattn_status rattn_set_fwd_tiling(int mode);
 

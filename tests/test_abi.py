@@ -46,9 +46,9 @@ def test_debug_build_compiles_and_exports_every_symbol():
 
 
 def test_fwd_tiling_hook_rejects_unknown_modes(rattn):
-    for mode in (-1, 3, 7):
+    for mode in (-1, 4, 7):
         assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.ERR_INVALID_ARG
-    for mode in (1, 2, 0):
+    for mode in (1, 2, 3, 0):
         assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.OK
 
 

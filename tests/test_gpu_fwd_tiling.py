@@ -1,10 +1,12 @@
-"""The two tilings of the bf16 attention forward (one 128-row query tile per
-CTA, or two sharing each staged K/V tile) against each other and the oracle.
+"""The three forms of the bf16 attention forward (one 128-row query tile per
+CTA; two sharing each staged K/V tile; a persistent kernel taking one-tile
+work items from a per-launch counter) against each other and the oracle.
 
-The library picks the tiling by row length; rattn_set_fwd_tiling forces one.
-Both evaluate every row's online softmax over the same key tiles in the same
-order with the same arithmetic, so O and LSE must be bit-identical; the
-two-tile results are also checked against the oracle at the bf16 tolerances.
+The library picks the form by row length and packing; rattn_set_fwd_tiling
+forces one. All evaluate every row's online softmax over the same key tiles in
+the same order with the same arithmetic, so O and LSE must be bit-identical;
+the two-tile results are also checked against the oracle at the bf16
+tolerances.
 Cases cover odd tile counts (the last pair has no second tile), ragged and
 padded lengths, both masks, the striped and contiguous layouts, D = 64,
 grouped key/value heads, packed sequences and the partial (one block) call."""
@@ -26,16 +28,17 @@ def rattn():
     r.rattn_set_fwd_tiling(0)
 
 
-def _both(rattn, fn):
+def _all_forms(rattn, fn):
     outs = []
-    for mode in (1, 2):
+    for mode in (1, 2, 3):
         rattn.rattn_set_fwd_tiling(mode)
         outs.append([t.clone() for t in fn()])
         torch.cuda.synchronize()
         assert rattn.rattn_get_device_error()[0] == rattn.OK
     rattn.rattn_set_fwd_tiling(0)
-    for a, b in zip(*outs):
-        assert torch.equal(a, b), "the two tilings differ"
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b), "the tilings differ"
     return outs[1]
 
 
@@ -62,7 +65,7 @@ def test_ring_fwd_tilings_agree_and_match_oracle(rattn, case):
     kp, _ = rattn.cp_layout_permute(k, cp, layout)
     vp, _ = rattn.cp_layout_permute(v, cp, layout)
     fwd = rattn.rattn_ring_fwd_gqa if H_kv != H else rattn.rattn_ring_fwd
-    o, lse = _both(rattn, lambda: fwd(qp, kp, vp, pos, cp, layout, causal, scale, L_valid=L))
+    o, lse = _all_forms(rattn, lambda: fwd(qp, kp, vp, pos, cp, layout, causal, scale, L_valid=L))
     out = rattn.cp_layout_unpermute(o, L, cp, layout)
     ke, ve = oracle.gqa_expand(to64(k), H), oracle.gqa_expand(to64(v), H)
     o_ref, l_ref = oracle.attention(to64(q), ke, ve, scale, causal)
@@ -80,12 +83,12 @@ def test_partial_fwd_tilings_agree(rattn):
     qpos = np.arange(200, 900, dtype=np.int32)
     kpos = np.arange(0, 900, dtype=np.int32)
     qd, kd = torch.from_numpy(qpos).cuda(), torch.from_numpy(kpos).cuda()
-    o, lse = _both(rattn, lambda: rattn.rattn_partial_fwd(q, k, v, qd, kd, causal=True, kv_valid=850))
+    o, lse = _all_forms(rattn, lambda: rattn.rattn_partial_fwd(q, k, v, qd, kd, causal=True, kv_valid=850))
     o_ref, l_ref = oracle.attention(to64(q), to64(k), to64(v), 128 ** -0.5, True, qpos, kpos, 850)
     check_lse(lse.cpu().numpy(), l_ref, torch.bfloat16)
     check_o(o.cpu().numpy(), o_ref, torch.bfloat16)
     e_k = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device="cuda")
-    o0, l0 = _both(rattn, lambda: rattn.rattn_partial_fwd(q, e_k, e_k, causal=True))
+    o0, l0 = _all_forms(rattn, lambda: rattn.rattn_partial_fwd(q, e_k, e_k, causal=True))
     assert torch.all(o0 == 0) and torch.all(torch.isneginf(l0))
 
 
@@ -97,7 +100,7 @@ def test_partial_fwd_tilings_agree_on_long_key_blocks(rattn):
     qpos = np.arange(70000, 70300, dtype=np.int32)
     kpos = np.arange(0, 140000, dtype=np.int32)
     qd, kd = torch.from_numpy(qpos).cuda(), torch.from_numpy(kpos).cuda()
-    o, lse = _both(rattn, lambda: rattn.rattn_partial_fwd(q, k, v, qd, kd, causal=True))
+    o, lse = _all_forms(rattn, lambda: rattn.rattn_partial_fwd(q, k, v, qd, kd, causal=True))
     o_ref, l_ref = oracle.attention(to64(q), to64(k), to64(v), 64 ** -0.5, True, qpos, kpos)
     check_lse(lse.cpu().numpy(), l_ref, torch.bfloat16)
     check_o(o.cpu().numpy(), o_ref, torch.bfloat16)
@@ -110,7 +113,7 @@ def test_packed_fwd_tilings_agree(rattn):
     src, gkey, segid = (plan[n].cuda() for n in ("src", "gkey", "segid"))
     q, k, v = (make_tensor((1, 2, cu[-1], 128), torch.bfloat16, "cuda", seed=s) for s in (81, 82, 83))
     qp, kp, vp = (rattn.cp_layout_gather(t, src) for t in (q, k, v))
-    o, lse = _both(rattn, lambda: rattn.rattn_ring_fwd_varlen(qp, kp, vp, gkey, segid, cp, True))
+    o, lse = _all_forms(rattn, lambda: rattn.rattn_ring_fwd_varlen(qp, kp, vp, gkey, segid, cp, True))
     out = rattn.cp_layout_scatter(o, src, cu[-1])
     for a, b in zip(cu, cu[1:]):
         if a == b:
@@ -118,3 +121,36 @@ def test_packed_fwd_tilings_agree(rattn):
         o_ref, _ = oracle.attention(to64(q[..., a:b, :]), to64(k[..., a:b, :]), to64(v[..., a:b, :]),
                                     128 ** -0.5, True)
         check_o(out[..., a:b, :].float().cpu().numpy(), o_ref, torch.bfloat16)
+
+
+def test_persistent_work_counters_reset_between_launches(rattn):
+    """Persistent launches back to back on one stream (sizes from one work
+    item per CTA to many, and one with no visible key at all), then two at
+    once on two streams: every launch must take each of its work items
+    exactly once, or its rows would be missing or stale."""
+    shapes = [(1, 1, 300, 300), (2, 4, 3000, 3000), (1, 2, 700, 0), (1, 8, 5000, 5000), (1, 1, 130, 130)]
+    inputs, refs = [], []
+    rattn.rattn_set_fwd_tiling(1)
+    try:
+        for i, (B, H, Lq, Lk) in enumerate(shapes):
+            q = make_tensor((B, H, Lq, 128), torch.bfloat16, "cuda", seed=90 + i)
+            k, v = (make_tensor((B, H, Lk, 128), torch.bfloat16, "cuda", seed=95 + i + j) for j in (0, 7))
+            inputs.append((q, k, v))
+            refs.append([t.clone() for t in rattn.rattn_partial_fwd(q, k, v, causal=True)])
+        rattn.rattn_set_fwd_tiling(3)
+        for rep in range(2):
+            outs = [rattn.rattn_partial_fwd(q, k, v, causal=True) for q, k, v in inputs]
+            torch.cuda.synchronize()
+            for got, want in zip(outs, refs):
+                assert torch.equal(got[0], want[0]) and torch.equal(got[1], want[1])
+        s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s1):
+            a = rattn.rattn_partial_fwd(*inputs[1], causal=True)
+        with torch.cuda.stream(s2):
+            b = rattn.rattn_partial_fwd(*inputs[3], causal=True)
+        torch.cuda.synchronize()
+        assert torch.equal(a[0], refs[1][0]) and torch.equal(b[0], refs[3][0])
+        assert rattn.rattn_get_device_error()[0] == rattn.OK
+    finally:
+        rattn.rattn_set_fwd_tiling(0)
