@@ -25,6 +25,7 @@ std::atomic<int> g_fwd_tiling{0};
 int* g_err_ptr[kMaxDevices] = {nullptr};
 unsigned long long g_wait_ns[kMaxDevices] = {0};
 int g_sm_count[kMaxDevices] = {0};
+// Cached like g_err_ptr: device addresses of a context that lives as long as the process.
 unsigned int* g_work_ptr[kMaxDevices] = {nullptr};
 std::atomic<unsigned> g_work_next{0};
 std::set<std::pair<const void*, int>> g_smem_done;
