@@ -174,20 +174,6 @@ __device__ __forceinline__ long long kposat(const Params& p, int seg, int row) {
   }
 }
 
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kDrainLimitNs) return false;
-  }
-  return true;
-}
-
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
-                                          uint64_t limit) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
-}
-
 // The dQ warpgroup's hand-off of one 128-row x 32-column fp32 chunk (this
 // thread's row in v) to the TMA: wait until the staging buffer's previous
 // reduce-add has read it, write the row 128-byte swizzled (16-byte piece j of

@@ -53,6 +53,7 @@
 #include <math.h>
 
 #include "debug_check.cuh"
+#include "fwd_positions.cuh"
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -105,39 +106,6 @@ struct Params {
   int* err;
   unsigned long long wait_ns;
 };
-
-__device__ __forceinline__ long long qpos(const Params& p, int seg, int row) {
-  const long long i = static_cast<long long>(seg) * p.Lq_seg + row;
-  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lq_seg, p.err, 1)) return 0;
-  return p.q_pos ? static_cast<long long>(__ldg(p.q_pos + i)) : row;
-}
-__device__ __forceinline__ long long kpos(const Params& p, int seg, int row) {
-  const long long i = static_cast<long long>(seg) * p.Lk_seg + row;
-  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lk_seg, p.err, 2)) return 0;
-  return p.kv_pos ? static_cast<long long>(__ldg(p.kv_pos + i)) : row;
-}
-// segid of a slot (packed sequences; only called when p.seg is set). Query and
-// key slots share one array (rank-major, Lq_seg == Lk_seg in ring calls).
-__device__ __forceinline__ int segat(const Params& p, int rank, int row) {
-  const long long i = static_cast<long long>(rank) * p.Lk_seg + row;
-  if (!in_bounds(i, static_cast<long long>(p.nseg) * p.Lk_seg, p.err, 3)) return 1;
-  return __ldg(p.seg + i);
-}
-
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kDrainLimitNs) return false;
-  }
-  return true;
-}
-
-// All lanes of the warp wait; the warp fails together if any lane gave up.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
-                                          uint64_t limit) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
-}
 
 // Work item w: (batch, head) slowest, then rank, then query tile, heaviest
 // first (largest local index, hence largest positions under every layout).

@@ -40,10 +40,6 @@ enum WaitSite : int {
   SITE_BOUNDS = 100,  // + check number: a debug build's bounds check failed
 };
 
-// Fixed limit for the teardown drains (copies and MMAs already in flight
-// always finish on their own; this only bounds a broken device).
-constexpr unsigned long long kDrainLimitNs = 2000000000ull;
-
 // 4-D bf16 tensor map over [outer][nseg][rows][D] with a (64 x box_rows) box
 // and 128-byte swizzle; rows past `rows` read as zero.
 rattn_status make_tmap_bf16(CUtensorMap* map, const void* base, int D, int64_t rows, int nseg, int64_t outer,

@@ -126,6 +126,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Fixed limit for the teardown drains (copies and MMAs already in flight
+// always finish on their own; this only bounds a broken device).
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+
+// Teardown wait for copies or MMAs already issued: spins (they complete on
+// their own) up to kDrainLimitNs, independent of the test hook's limit.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kDrainLimitNs) return false;
+  }
+  return true;
+}
+
+// All lanes of the warp wait; the warp fails together if any lane gave up.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit)) != 0;
+}
+
 // Records the first failure of a kernel launch: the CTA-local abort flag stops
 // the other roles' waits, the global word reports the site to the host.
 __device__ __forceinline__ void record_failure(volatile int* abort, int* err_word, int site) {
