@@ -43,6 +43,8 @@ BWD_CASES = [
     (torch.bfloat16, 128, 1000, 4, 2, True),
     (torch.bfloat16, 64, 29, 3, 2, True),
     (torch.float32, 64, 29, 3, 2, True),
+    (torch.bfloat16, 128, 1000, 64, 1, True),   # the most ranks a call takes: 64 hops
+    (torch.bfloat16, 64, 3000, 64, 2, True),    # striped, 64 ranks
 ]
 
 

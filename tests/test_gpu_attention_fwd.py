@@ -146,6 +146,9 @@ RAGGED = [
     (torch.bfloat16, 128, 2048, 8, 2, False, 1, 1),    # striped non-causal
     (torch.bfloat16, 64, 4100, 3, 2, True, 1, 1),      # striped, padded, several tiles per hop
     (torch.float32, 64, 29, 3, 2, True, 1, 2),
+    (torch.bfloat16, 128, 1000, 64, 1, True, 1, 2),   # the most ranks a call takes: 64 hops, 8-token chunks
+    (torch.bfloat16, 64, 3000, 64, 2, True, 1, 1),    # striped, 64 ranks
+    (torch.float32, 64, 500, 64, 1, True, 1, 1),      # fp32 path, 64 ranks
 ]
 
 

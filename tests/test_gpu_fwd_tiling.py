@@ -52,6 +52,7 @@ RING = [
     (1, 1, 1, 8192, 128, 2, 1, True),     # 32 tiles per slice
     (1, 2, 2, 1664, 128, 2, 1, True),     # 832-row slices: 7 tiles, an odd count
     (1, 2, 2, 640, 64, 1, 0, True),       # one rank: 5 tiles, D = 64
+    (1, 2, 2, 3000, 128, 64, 1, True),    # 64 ranks (the most a call takes): 64 hops per tile
 ]
 
 
