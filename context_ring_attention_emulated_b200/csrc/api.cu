@@ -22,6 +22,7 @@ constexpr unsigned long long kDefaultWaitNs = 4000000000ull;
 
 std::mutex g_mu;
 std::atomic<int> g_fwd_tiling{0};
+std::atomic<int> g_bwd_deterministic{0};
 int* g_err_ptr[kMaxDevices] = {nullptr};
 unsigned long long g_wait_ns[kMaxDevices] = {0};
 int g_sm_count[kMaxDevices] = {0};
@@ -99,6 +100,7 @@ rattn_status get_dev_ctx(DevCtx* out) {
   out->err_word = g_err_ptr[dev];
   out->wait_ns = g_wait_ns[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
   out->fwd_tiling = g_fwd_tiling.load();
+  out->bwd_deterministic = g_bwd_deterministic.load();
   return RATTN_OK;
 }
 
@@ -617,6 +619,12 @@ rattn_status rattn_get_device_error(int* site) {
     if (cudaMemcpyToSymbol(g_err_word, &zero, sizeof(int)) != cudaSuccess) return RATTN_ERR_CUDA;
     return v >= SITE_BOUNDS ? RATTN_ERR_BOUNDS : RATTN_ERR_TIMEOUT;
   }
+  return RATTN_OK;
+}
+
+rattn_status rattn_set_bwd_deterministic(int on) {
+  if (on != 0 && on != 1) return RATTN_ERR_INVALID_ARG;
+  g_bwd_deterministic.store(on);
   return RATTN_OK;
 }
 

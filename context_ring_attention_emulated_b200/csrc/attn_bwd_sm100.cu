@@ -897,6 +897,7 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
                          : reinterpret_cast<const void*>(&bwd_kernel<D, false, false>);
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
   if ((st = check_launch_regs(kfn)) != RATTN_OK) return st;
+  if (ctx.bwd_deterministic && (st = launch_bwd_dq_sm100(a, ctx, false)) != RATTN_OK) return st;
   bwd_prep_kernel<D, true><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
@@ -930,6 +931,9 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
     bwd_kernel<D, false, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq,
                                                                                                p);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
+  // Deterministic mode: dQ again, by one CTA per query tile in a fixed key
+  // order, written over what the accumulator would give.
+  if (ctx.bwd_deterministic) return launch_bwd_dq_sm100(a, ctx, true);
   const long long n4 = rows * D / 4;
   dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
                                                             static_cast<uint2*>(a.dq), a.scale, n4);

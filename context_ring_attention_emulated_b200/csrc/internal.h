@@ -17,6 +17,7 @@ struct DevCtx {
   unsigned long long wait_ns;
   int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two, 3 persistent (rattn_set_fwd_tiling)
   int sm_count;    // multiprocessors of the device (persistent grids)
+  int bwd_deterministic;  // 1: dQ of the ring backward by the query-stationary pass (rattn_set_bwd_deterministic)
   // A pair of work counters for one persistent launch (next work item, CTAs
   // finished), zero when the launch starts; its last CTA zeroes them again.
   // Each context fetch takes the next of kWorkSlots pairs, so launches in
@@ -110,6 +111,11 @@ struct BwdArgs {
   cudaStream_t stream;
 };
 rattn_status launch_bwd_sm100(const BwdArgs& a, const DevCtx& ctx);
+// The query-stationary dQ pass (attn_bwd_dq_sm100.cu): dq (bf16) from q, k, v,
+// dout, lse, delta and the positions of a; run = false only prepares and
+// checks everything on the host (so that a later failure cannot follow a
+// launch).
+rattn_status launch_bwd_dq_sm100(const BwdArgs& a, const DevCtx& ctx, bool run);
 
 // One hop of the ring backward with query rows of one rank and key rows of
 // another: q, dout [BH][Lq][D], lse, delta [BH][Lq], q_pos [Lq]; k, v

@@ -64,6 +64,7 @@ SIGNATURES = [
     ("rattn_grad_fold", _I, [_P, _P, _I64, _P]),
     ("rattn_get_device_error", _I, [ctypes.POINTER(_I)]),
     ("rattn_set_fwd_tiling", _I, [_I]),
+    ("rattn_set_bwd_deterministic", _I, [_I]),
     ("rattn_set_wait_limit_ns", _I, [ctypes.c_ulonglong]),
 ]
 
@@ -566,6 +567,11 @@ def rattn_get_device_error():
     site = ctypes.c_int(0)
     code = lib.rattn_get_device_error(ctypes.byref(site))
     return code, site.value
+
+
+def rattn_set_bwd_deterministic(on):
+    """True: the ring backward's dQ by a query-stationary pass (bitwise reproducible gradients)."""
+    _check("rattn_set_bwd_deterministic", lib.rattn_set_bwd_deterministic(int(bool(on))))
 
 
 def rattn_set_fwd_tiling(mode):

@@ -407,6 +407,20 @@ rattn_status rattn_get_device_error(int* site);
  * RATTN_ERR_INVALID_ARG for any other mode. */
 rattn_status rattn_set_fwd_tiling(int mode);
 
+/* Reproducibility switch for the ring backward (rattn_ring_bwd, _gqa, _varlen,
+ * _noalloc), for launches made after the call, on every device. By default dQ
+ * is accumulated by the key/value-stationary kernel with fp32 reduce-adds from
+ * many CTAs, whose order varies from run to run (dK and dV are always
+ * accumulated in a fixed order). With on = 1 a second, query-stationary pass
+ * recomputes dQ = scale * sum_j dS_ij k_j for each 128-row query tile in one
+ * CTA, over the key tiles in ring order, and writes it: dQ, dK and dV are then
+ * the same, bit for bit, on every run with the same inputs, at the cost of
+ * that pass (about as long as the forward). The textbook gradient of softmax
+ * attention (the pages call .backward(); [CP-glossary] "Practical use and
+ * trade-offs"). Returns RATTN_ERR_INVALID_ARG unless on is 0 or 1. The per-hop
+ * rattn_partial_bwd is not affected. */
+rattn_status rattn_set_bwd_deterministic(int on);
+
 /* Test hook: the per-wait time limit in nanoseconds used by subsequent
  * launches on the current device (default 4e9; 0 restores the default). A
  * tiny limit makes waits give

@@ -45,6 +45,13 @@ def test_debug_build_compiles_and_exports_every_symbol():
         assert hasattr(lib, n), f"{n} missing from the debug build"
 
 
+def test_bwd_deterministic_switch_rejects_other_values(rattn):
+    for on in (-1, 2, 5):
+        assert rattn.lib.rattn_set_bwd_deterministic(on) == rattn.ERR_INVALID_ARG
+    for on in (1, 0):
+        assert rattn.lib.rattn_set_bwd_deterministic(on) == rattn.OK
+
+
 def test_fwd_tiling_hook_rejects_unknown_modes(rattn):
     for mode in (-1, 4, 7):
         assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.ERR_INVALID_ARG
