@@ -202,7 +202,9 @@ __device__ __forceinline__ void stage_dq_chunk(const uint32_t (&v)[32], uint8_t*
 
 // 16 warps share an SM's four register-file partitions 4/4/4/4: 16,384 / (4 x
 // 32) = 128 registers per thread at launch.
-template <int D, bool SEG, bool SPLIT>  // SEG: packed sequences; SPLIT: one hop across processes
+// SEG: packed sequences; SPLIT: one hop across processes; DQ = false: dK and
+// dV only (the deterministic mode forms dQ in a query-stationary pass).
+template <int D, bool SEG, bool SPLIT, bool DQ = true>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -439,7 +441,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto mma_dp = [&](int j) -> bool {
         if (!wt(&bar_o_full[j % C::NSO], (j / C::NSO) & 1)) return false;
-        if (j > 0 && !wt(bar_dq_empty, (j - 1) & 1)) return false;  // dQ(j-1) read out
+        if constexpr (DQ) {
+          if (j > 0 && !wt(bar_dq_empty, (j - 1) & 1)) return false;  // dQ(j-1) read out
+        } else {  // dK(j-1), the last reader of dS^T(j-1), has completed
+          if (j > 0 && !wt(&bar_q_empty[(j - 1) % C::NSQ], ((j - 1) / C::NSQ) & 1)) return false;
+        }
         tc_fence_after();
         const uint32_t o = sDO(j);
 #pragma unroll
@@ -492,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = wt(bar_kv_full, 0);
       ok = ok && mma_s(0) && mma_dv(0) && mma_dp(0) && (NIT < 2 || mma_s(1));
       for (int i = 0; i < NIT && ok; ++i) {
-        ok = mma_dk(i) && mma_dq(i);
+        ok = mma_dk(i) && (!DQ || mma_dq(i));
         if (ok && i + 1 < NIT) ok = mma_dp(i + 1) && mma_dv(i + 1);
         if (ok && i + 2 < NIT) ok = mma_s(i + 2);
       }
@@ -632,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar_p_ready);  // one arrival per warp
         // dS(j) goes into the shared tile that dQ(j-1) reads: wait for it.
         if (!warp_wait(bar_dp_full, it & 1, s_abort, p.wait_ns) ||
-            (it > 0 && !warp_wait(bar_dq_full, (it - 1) & 1, s_abort, p.wait_ns))) {
+            (DQ && it > 0 && !warp_wait(bar_dq_full, (it - 1) & 1, s_abort, p.wait_ns))) {
           if (lane == 0) record_failure(s_abort, p.err, SITE_BWD_COMPUTE);
           ok = false;
           break;
@@ -660,15 +666,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[e] = pack_bf16x2(a, b);
           }
           tmem_st8(t_dp + c * 8, pk);
+          if constexpr (DQ) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int chunk = c * 2 + j;
-            *reinterpret_cast<uint4*>(rowp + ((chunk ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int j = 0; j < 2; ++j) {
+              const int chunk = c * 2 + j;
+              *reinterpret_cast<uint4*>(rowp + ((chunk ^ (row & 7)) << 4)) =
+                  make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            }
           }
         }
         tmem_wait_st();
-        fence_proxy_async_smem();
+        if constexpr (DQ) fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_ds_ready);  // one arrival per warp
@@ -752,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool elected = threadIdx.x == 0;
     uint8_t* stg = smem + C::OFF_STG;
     int n_staged = 0;
-    bool ok = NIT > 0;
+    bool ok = DQ && NIT > 0;
     int it = 0;
     for (int hq = 0; hq < p.group && ok; ++hq) {
     const int bh = kvh * p.group + hq;  // (batch, query head)
@@ -893,13 +901,23 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   if ((st = make_tmap_bf16(&tv, a.v, D, a.Lseg, a.nseg, a.BH / a.group, BK)) != RATTN_OK) return st;
   if ((st = make_tmap_bf16(&tdo, a.dout, D, a.Lseg, a.nseg, a.BH, BQ)) != RATTN_OK) return st;
   if ((st = make_tmap_f32_acc(&tdq, a.dq_acc, D, a.Lseg, a.nseg, a.BH)) != RATTN_OK) return st;
-  const void* kfn = a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true, false>)
-                         : reinterpret_cast<const void*>(&bwd_kernel<D, false, false>);
+  // Deterministic mode: this kernel forms dK and dV only, and a
+  // query-stationary pass forms dQ (no accumulator to zero or convert).
+  const bool det = ctx.bwd_deterministic != 0;
+  const void* kfn = det ? (a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true, false, false>)
+                                 : reinterpret_cast<const void*>(&bwd_kernel<D, false, false, false>))
+                        : (a.seg ? reinterpret_cast<const void*>(&bwd_kernel<D, true, false>)
+                                 : reinterpret_cast<const void*>(&bwd_kernel<D, false, false>));
   if ((st = set_smem_attr(kfn, C::SMEM)) != RATTN_OK) return st;
   if ((st = check_launch_regs(kfn)) != RATTN_OK) return st;
-  if (ctx.bwd_deterministic && (st = launch_bwd_dq_sm100(a, ctx, false)) != RATTN_OK) return st;
-  bwd_prep_kernel<D, true><<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, a.stream>>>(
-      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
+  if (det && (st = launch_bwd_dq_sm100(a, ctx, false)) != RATTN_OK) return st;
+  const unsigned prep_grid = static_cast<unsigned>((rows * 16 + 255) / 256);
+  if (det)
+    bwd_prep_kernel<D, false><<<prep_grid, 256, 0, a.stream>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
+  else
+    bwd_prep_kernel<D, true><<<prep_grid, 256, 0, a.stream>>>(
+        static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.delta, a.dq_acc, rows);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
   Params p;
   p.lse = a.lse;
@@ -924,16 +942,18 @@ rattn_status launch(const BwdArgs& a, const DevCtx& ctx) {
   p.dv = a.dv;
   p.err = ctx.err_word;
   p.wait_ns = ctx.wait_ns;
-  if (a.seg)
-    bwd_kernel<D, true, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq,
-                                                                                              p);
+  const unsigned g = static_cast<unsigned>(grid);
+  if (det && a.seg)
+    bwd_kernel<D, true, false, false><<<g, kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq, p);
+  else if (det)
+    bwd_kernel<D, false, false, false><<<g, kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq, p);
+  else if (a.seg)
+    bwd_kernel<D, true, false><<<g, kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq, p);
   else
-    bwd_kernel<D, false, false><<<static_cast<unsigned>(grid), kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq,
-                                                                                               p);
+    bwd_kernel<D, false, false><<<g, kThreads, C::SMEM, a.stream>>>(tq, tk, tv, tdo, tdq, p);
   if (cudaGetLastError() != cudaSuccess) return RATTN_ERR_CUDA;
-  // Deterministic mode: dQ again, by one CTA per query tile in a fixed key
-  // order, written over what the accumulator would give.
-  if (ctx.bwd_deterministic) return launch_bwd_dq_sm100(a, ctx, true);
+  // Deterministic mode: dQ by one CTA per query tile, in a fixed key order.
+  if (det) return launch_bwd_dq_sm100(a, ctx, true);
   const long long n4 = rows * D / 4;
   dq_convert_kernel<<<grid_for(n4, 256), 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
                                                             static_cast<uint2*>(a.dq), a.scale, n4);
