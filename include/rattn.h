@@ -404,7 +404,11 @@ rattn_status rattn_get_device_error(int* site);
  * kernel (one CTA per SM taking one-tile work items from a per-launch
  * counter); else one tile per CTA. 1 forces one tile per CTA, 2 two, 3 the
  * persistent kernel. All give bit-identical O and LSE. Returns
- * RATTN_ERR_INVALID_ARG for any other mode. */
+ * RATTN_ERR_INVALID_ARG for any other mode. A persistent launch takes one of
+ * 256 counter pairs in the library's device memory, zeroed again by its last
+ * CTA; a launch captured in a CUDA graph keeps its pair, so replays of one
+ * captured launch must not overlap each other, and more than 256 persistent
+ * launches must not be in flight at once. */
 rattn_status rattn_set_fwd_tiling(int mode);
 
 /* Reproducibility switch for the ring backward (rattn_ring_bwd, _gqa, _varlen,
