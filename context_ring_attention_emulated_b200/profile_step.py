@@ -26,7 +26,9 @@ def main(argv=None):
     ap.add_argument("--layout", type=int, default=rattn.LAYOUT_HEAD_TAIL)
     ap.add_argument("--noncausal", action="store_true")
     ap.add_argument("--iters", type=int, default=2)
+    ap.add_argument("--fwd-tiling", type=int, default=0, help="rattn_set_fwd_tiling mode (0 automatic)")
     a = ap.parse_args(argv)
+    rattn.rattn_set_fwd_tiling(a.fwd_tiling)
     causal = not a.noncausal
     shape = (a.B, a.H, a.L, a.D)
     q, k, v, do = (make_tensor(shape, torch.bfloat16, "cuda", seed=s) for s in range(4))
