@@ -629,7 +629,7 @@ rattn_status rattn_set_bwd_deterministic(int on) {
 }
 
 rattn_status rattn_set_fwd_tiling(int mode) {
-  if (mode < 0 || mode > 3) return RATTN_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 4) return RATTN_ERR_INVALID_ARG;
   g_fwd_tiling.store(mode);
   return RATTN_OK;
 }

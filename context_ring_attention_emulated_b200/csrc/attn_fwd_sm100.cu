@@ -557,23 +557,34 @@ rattn_status launch(const FwdArgs& a, const DevCtx& ctx) {
 
 }  // namespace
 
-// Two query tiles per CTA (attn_fwd_pair_sm100.cu) halve the K/V bytes moved
-// from L2 into shared memory per FLOP but serialise each tile's score ->
-// softmax -> product chain (one TMEM score buffer per tile). Measured on B200
-// (causal, D = 128): one tile is faster up to 131,072 keys per row, two from
-// 262,144 keys on, where one head's K and V (L x D x 4 bytes) outgrow L2 and
-// the launches run long enough to be held at the power-capped clock.
+// Forms of the bf16 forward (all compute the same attention; measured on B200):
+//  - 256-key tiles (attn_fwd_wide_sm100.cu, D = 128, at most 32 segments): the
+//    score product runs as N = 256 MMAs, about 1.6x the rate of N = 128 ones,
+//    and the next score product overlaps the softmax; 4-8 % faster than the
+//    other forms on dense rows of every length measured (16k to 1M keys);
+//  - two 128-row query tiles per CTA (attn_fwd_pair_sm100.cu): half the K/V
+//    bytes per FLOP; faster than one tile from 262,144 keys per row (where one
+//    head's K and V outgrow L2), so the choice for long rows with D = 64;
+//  - the persistent kernel (attn_fwd_persist_sm100.cu): work items of one
+//    query tile taken from a per-launch counter; 8 % faster on packed
+//    sequences, whose items are short, and slower per tile on dense rows;
+//  - one 128-row query tile per CTA (this file): everything else.
+// rattn_set_fwd_tiling forces one form (1 one tile, 2 two tiles, 3
+// persistent, 4 256-key tiles).
 constexpr long long kPairMinKeys = 262144;
 
-// The persistent kernel (attn_fwd_persist_sm100.cu) hides each work item's
-// start-up behind the previous item; measured on B200 it is faster where items
-// are short (the packed-sequence forward, 24 documents in 32,000 tokens: +8 %)
-// and 6-10 % slower per key tile on dense rows, so it serves packed sequences.
 rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx) {
-  const bool pair = ctx.fwd_tiling == 2 ||
-                    (ctx.fwd_tiling == 0 && static_cast<long long>(a.nseg) * a.Lk_seg >= kPairMinKeys);
-  if (pair) return launch_fwd_sm100_pair(a, ctx);
-  if (ctx.fwd_tiling == 3 || (ctx.fwd_tiling == 0 && a.seg)) return launch_fwd_sm100_persist(a, ctx);
+  switch (ctx.fwd_tiling) {
+    case 1: break;
+    case 2: return launch_fwd_sm100_pair(a, ctx);
+    case 3: return launch_fwd_sm100_persist(a, ctx);
+    case 4: return launch_fwd_sm100_wide(a, ctx);
+    default:
+      if (!a.seg && a.D == 128 && a.nseg <= 32) return launch_fwd_sm100_wide(a, ctx);
+      if (static_cast<long long>(a.nseg) * a.Lk_seg >= kPairMinKeys) return launch_fwd_sm100_pair(a, ctx);
+      if (a.seg) return launch_fwd_sm100_persist(a, ctx);
+      break;
+  }
   if (a.D == 128) return launch<128>(a, ctx);
   if (a.D == 64) return launch<64>(a, ctx);
   return RATTN_ERR_UNSUPPORTED;

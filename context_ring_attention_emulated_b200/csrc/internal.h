@@ -15,7 +15,7 @@ namespace rattn {
 struct DevCtx {
   int* err_word;
   unsigned long long wait_ns;
-  int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two, 3 persistent (rattn_set_fwd_tiling)
+  int fwd_tiling;  // 0 automatic, 1 one query tile per CTA, 2 two, 3 persistent, 4 256-key tiles (rattn_set_fwd_tiling)
   int sm_count;    // multiprocessors of the device (persistent grids)
   int bwd_deterministic;  // 1: dQ of the ring backward by the query-stationary pass (rattn_set_bwd_deterministic)
   // A pair of work counters for one persistent launch (next work item, CTAs
@@ -83,6 +83,7 @@ struct FwdArgs {
 rattn_status launch_fwd_sm100(const FwdArgs& a, const DevCtx& ctx);
 rattn_status launch_fwd_sm100_pair(const FwdArgs& a, const DevCtx& ctx);  // two query tiles per CTA
 rattn_status launch_fwd_sm100_persist(const FwdArgs& a, const DevCtx& ctx);  // persistent, one tile per item
+rattn_status launch_fwd_sm100_wide(const FwdArgs& a, const DevCtx& ctx);  // 256-key tiles (D = 128)
 rattn_status launch_fwd_simt(const FwdArgs& a);
 
 struct BwdArgs {

@@ -575,7 +575,8 @@ def rattn_set_bwd_deterministic(on):
 
 
 def rattn_set_fwd_tiling(mode):
-    """0: automatic, 1: one query tile per CTA, 2: two, 3: persistent (one tile per work item)."""
+    """0: automatic, 1: one query tile per CTA, 2: two, 3: persistent (one tile per work item),
+    4: 256-key tiles (D = 128)."""
     _check("rattn_set_fwd_tiling", lib.rattn_set_fwd_tiling(int(mode)))
 
 

@@ -397,14 +397,19 @@ rattn_status rattn_ring_bwd_noalloc(const void* q, const void* k, const void* v,
 rattn_status rattn_get_device_error(int* site);
 
 /* Tuning and test hook: how the bf16 attention forward (ring, GQA, packed and
- * partial calls) tiles the queries, for launches made after the call, on
- * every device. 0 (the default) chooses: two 128-row query tiles per CTA,
- * sharing each staged K/V tile, when a query row attends at least 262,144
- * keys (cp_size x slice length); else, for packed sequences, a persistent
- * kernel (one CTA per SM taking one-tile work items from a per-launch
- * counter); else one tile per CTA. 1 forces one tile per CTA, 2 two, 3 the
- * persistent kernel. All give bit-identical O and LSE. Returns
- * RATTN_ERR_INVALID_ARG for any other mode. A persistent launch takes one of
+ * partial calls) tiles its work, for launches made after the call, on every
+ * device. 0 (the default) chooses: for unpacked calls with D = 128 and at
+ * most 32 segments, 128 query rows per CTA against 256-key tiles (the score
+ * product as N = 256 MMAs); else two 128-row query tiles per CTA sharing each
+ * staged K/V tile when a query row attends at least 262,144 keys (cp_size x
+ * slice length); else, for packed sequences, a persistent kernel (one CTA per
+ * SM taking one-tile work items from a per-launch counter); else one 128-row
+ * query tile per CTA against 128-key tiles. 1 forces one tile per CTA, 2 two,
+ * 3 the persistent kernel, 4 the 256-key tiles (RATTN_ERR_UNSUPPORTED unless
+ * D = 128 and at most 32 segments). Forms 1-3 give bit-identical O and LSE;
+ * form 4 folds the keys in 256-key steps and so rounds differently (within the
+ * bf16 tolerances of the others). Returns RATTN_ERR_INVALID_ARG for any other
+ * mode. A persistent launch takes one of
  * 256 counter pairs in the library's device memory, zeroed again by its last
  * CTA; a launch captured in a CUDA graph keeps its pair, so replays of one
  * captured launch must not overlap each other, and more than 256 persistent

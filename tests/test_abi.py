@@ -53,9 +53,9 @@ def test_bwd_deterministic_switch_rejects_other_values(rattn):
 
 
 def test_fwd_tiling_hook_rejects_unknown_modes(rattn):
-    for mode in (-1, 4, 7):
+    for mode in (-1, 5, 7):
         assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.ERR_INVALID_ARG
-    for mode in (1, 2, 3, 0):
+    for mode in (1, 2, 3, 4, 0):
         assert rattn.lib.rattn_set_fwd_tiling(mode) == rattn.OK
 
 
