@@ -235,11 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0 && G > 0) {
+    if (G > 0) {  // the whole warp walks the schedule and waits; one elected lane issues
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       const uint32_t idesc_q = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sDOa = smem_u32(sDO);
-      bool ok = mbar_wait(bar_q_full, 0, s_abort, p.wait_ns);
+      bool ok = warp_wait(bar_q_full, 0, s_abort, p.wait_ns);
       // A x B^T over D for 128 x 128 tiles, both operands K-major in smem
       auto mma_nt = [&](uint32_t d, uint32_t a, uint32_t b) {
 #pragma unroll
@@ -251,20 +251,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S_g = Q K_g^T into score buffer g % 2
       auto issue_s = [&](int g) -> bool {
         const int st = g % C::NSK;
-        if (!mbar_wait(&bar_k_full[st], (g / C::NSK) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_k_full[st], (g / C::NSK) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        mma_nt(tmem + (g & 1) * 128, sQa, smem_u32(sK + st * C::TILE));
-        umma_commit(&bar_s_full[g & 1]);
+        if (elect_one()) {
+          mma_nt(tmem + (g & 1) * 128, sQa, smem_u32(sK + st * C::TILE));
+          umma_commit(&bar_s_full[g & 1]);
+        }
+        __syncwarp();
         return true;
       };
       // dP_g = dO V_g^T
       auto issue_dp = [&](int g) -> bool {
         const int sv = g % C::NSV;
-        if (!mbar_wait(&bar_v_full[sv], (g / C::NSV) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_v_full[sv], (g / C::NSV) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        mma_nt(tmem + C::T_DP, sDOa, smem_u32(sV + sv * C::TILE));
-        umma_commit(bar_dp_full);
-        umma_commit(&bar_v_empty[sv]);
+        if (elect_one()) {
+          mma_nt(tmem + C::T_DP, sDOa, smem_u32(sV + sv * C::TILE));
+          umma_commit(bar_dp_full);
+          umma_commit(&bar_v_empty[sv]);
+        }
+        __syncwarp();
         return true;
       };
       // Per tile g: dP_{g+1} as soon as the compute warps have read dP_g (it
@@ -274,28 +280,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && G > 1) ok = issue_s(1);
       for (int g = 0; g < G && ok; ++g) {
         if (g + 1 < G) {
-          ok = mbar_wait(bar_dp_free, g & 1, s_abort, p.wait_ns) && issue_dp(g + 1);
+          ok = warp_wait(bar_dp_free, g & 1, s_abort, p.wait_ns) && issue_dp(g + 1);
           if (!ok) break;
         }
         // dQ += dS_g K_g: dS_g (bf16, 128 query rows x 128 keys) from the
         // first 64 columns of its score buffer, K_g as an MN-major B operand
-        ok = mbar_wait(&bar_ds_ready[g & 1], (g >> 1) & 1, s_abort, p.wait_ns);
+        ok = warp_wait(&bar_ds_ready[g & 1], (g >> 1) & 1, s_abort, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
-        const int st = g % C::NSK;
-        const uint32_t sKa = smem_u32(sK + st * C::TILE);
-        const uint32_t a_t = tmem + (g & 1) * 128;
+        if (elect_one()) {
+          const int st = g % C::NSK;
+          const uint32_t sKa = smem_u32(sK + st * C::TILE);
+          const uint32_t a_t = tmem + (g & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(sKa + kk * 2048, C::BOX, 1024);
-          umma_ts(tmem + C::T_DQ, a_t + kk * 8, bd, idesc_q, (g > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t bd = sdesc_sw128(sKa + kk * 2048, C::BOX, 1024);
+            umma_ts(tmem + C::T_DQ, a_t + kk * 8, bd, idesc_q, (g > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar_dq_done[g & 1]);
+          umma_commit(&bar_k_empty[st]);
         }
-        umma_commit(&bar_dq_done[g & 1]);
-        umma_commit(&bar_k_empty[st]);
+        __syncwarp();
         if (g + 2 < G)
-          ok = mbar_wait(&bar_dq_done[g & 1], (g >> 1) & 1, s_abort, p.wait_ns) && issue_s(g + 2);
+          ok = warp_wait(&bar_dq_done[g & 1], (g >> 1) & 1, s_abort, p.wait_ns) && issue_s(g + 2);
       }
-      if (!ok) record_failure(s_abort, p.err, SITE_BWD_MMA);
+      if (!ok && lane == 0) record_failure(s_abort, p.err, SITE_BWD_MMA);
     }
   } else {
     // ------------------------------------------------ dS and the epilogue
@@ -448,9 +457,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = max(0, issued_v - C::NSV); g < issued_v; ++g)
       drain_wait(&bar_v_full[g % C::NSV], (g / C::NSV) & 1);
   }
-  if (warp == 1 && lane == 0 && G > 0) {
-    umma_commit(bar_drain);
-    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  if (warp == 1 && G > 0) {  // the lane that issued the products commits
+    if (elect_one()) {
+      umma_commit(bar_drain);
+      if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -26,7 +26,11 @@
 //                half of dK/dV each;
 //   warp 12      producer: K, V once; per query tile Q and dO by TMA and the
 //                tile's LSE (pre-scaled by log2 e) and Delta into shared memory;
-//   warp 13      TMEM allocation and tcgen05.mma issue (one thread);
+//   warp 13      TMEM allocation and tcgen05.mma issue (the whole warp walks
+//                the schedule and waits, one lane chosen by elect.sync issues:
+//                with the warp converged the operands stay warp-uniform; the
+//                kernel ran about 20 % faster so than with a lone lane-0
+//                thread walking the schedule);
 //   warps 14, 15 idle (they complete the producer/MMA warpgroup, whose
 //                registers the dQ warpgroup takes over: setmaxnreg).
 // TMEM columns: [0,128) S^T, then P^T (bf16, warpgroup g at [64g, 64g+32));
@@ -415,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // by one thread execute in issue order, so dQ(i) follows dK(i) without a
     // wait although it overwrites the dS^T columns dK(i) reads, and S(j)
     // follows dV(j-1), which reads the P^T columns S(j) overwrites.
-    if (lane == 0 && NIT > 0) {
+    if (NIT > 0) {  // the whole warp walks the schedule and waits; one elected lane issues
       const uint32_t idesc_t = idesc_bf16_f32(BK, BQ, 0, 0);  // S^T, dP^T: K-major A and B
       const uint32_t idesc_g = idesc_bf16_f32(BK, D, 0, 1);   // dV, dK: A in TMEM, B MN-major
       const uint32_t idesc_q = idesc_bf16_f32(BQ, D, 1, 1);   // dQ: A (dS) and B (K) MN-major
@@ -424,19 +428,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sDS = smem_u32(smem + C::OFF_DS);
       auto sQ = [&](int j) { return smem_u32(smem + C::OFF_Q + (j % C::NSQ) * C::TILE); };
       auto sDO = [&](int j) { return smem_u32(smem + C::OFF_DO + (j % C::NSO) * C::TILE); };
-      auto wt = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, s_abort, p.wait_ns); };
+      auto wt = [&](uint64_t* bar, uint32_t parity) { return warp_wait(bar, parity, s_abort, p.wait_ns); };
 
       auto mma_s = [&](int j) -> bool {
         if (!wt(&bar_q_full[j % C::NSQ], (j / C::NSQ) & 1)) return false;
         tc_fence_after();
-        const uint32_t q = sQ(j);
+        if (elect_one()) {
+          const uint32_t q = sQ(j);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          umma_ss(tmem + C::T_S, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q + off, 16, 1024), idesc_t,
-                  kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+            umma_ss(tmem + C::T_S, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q + off, 16, 1024), idesc_t,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_s_full);
         }
-        umma_commit(bar_s_full);
+        __syncwarp();
         return true;
       };
       auto mma_dp = [&](int j) -> bool {
@@ -447,51 +454,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j > 0 && !wt(&bar_q_empty[(j - 1) % C::NSQ], ((j - 1) / C::NSQ) & 1)) return false;
         }
         tc_fence_after();
-        const uint32_t o = sDO(j);
+        if (elect_one()) {
+          const uint32_t o = sDO(j);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          umma_ss(tmem + C::T_DP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(o + off, 16, 1024), idesc_t,
-                  kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+            umma_ss(tmem + C::T_DP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(o + off, 16, 1024), idesc_t,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_dp_full);
+          if (j == 0) umma_commit(&bar_o_empty[0]);  // dV(0) was issued before dP(0)
         }
-        umma_commit(bar_dp_full);
-        if (j == 0) umma_commit(&bar_o_empty[0]);  // dV(0) was issued before dP(0)
+        __syncwarp();
         return true;
       };
       auto mma_dv = [&](int j) -> bool {
         if (!wt(bar_p_ready, j & 1)) return false;
         if (!wt(&bar_o_full[j % C::NSO], (j / C::NSO) & 1)) return false;
         tc_fence_after();
-        const uint32_t o = sDO(j);
+        if (elect_one()) {
+          const uint32_t o = sDO(j);
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint32_t a_col = C::T_S + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s P^T
-          umma_ts(tmem + C::T_DV, tmem + a_col, sdesc_sw128(o + kk * 2048, C::BOX, 1024), idesc_g,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BQ / 16; ++kk) {
+            const uint32_t a_col = C::T_S + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s P^T
+            umma_ts(tmem + C::T_DV, tmem + a_col, sdesc_sw128(o + kk * 2048, C::BOX, 1024), idesc_g,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (j > 0) umma_commit(&bar_o_empty[j % C::NSO]);  // dP(j) was issued before dV(j)
         }
-        if (j > 0) umma_commit(&bar_o_empty[j % C::NSO]);  // dP(j) was issued before dV(j)
+        __syncwarp();
         return true;
       };
       auto mma_dk = [&](int j) -> bool {
         if (!wt(bar_ds_ready, j & 1)) return false;
         tc_fence_after();
-        const uint32_t q = sQ(j);
+        if (elect_one()) {
+          const uint32_t q = sQ(j);
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint32_t a_col = C::T_DP + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s dS^T
-          umma_ts(tmem + C::T_DK, tmem + a_col, sdesc_sw128(q + kk * 2048, C::BOX, 1024), idesc_g,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BQ / 16; ++kk) {
+            const uint32_t a_col = C::T_DP + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s dS^T
+            umma_ts(tmem + C::T_DK, tmem + a_col, sdesc_sw128(q + kk * 2048, C::BOX, 1024), idesc_g,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar_q_empty[j % C::NSQ]);  // S(j) and dK(j) were Q's readers
         }
-        umma_commit(&bar_q_empty[j % C::NSQ]);  // S(j) and dK(j) were Q's readers
+        __syncwarp();
         return true;
       };
       auto mma_dq = [&](int j) -> bool {
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          umma_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
-                  sdesc_sw128(sK + kk * 2048, C::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
-        umma_commit(bar_dq_full);
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
+                    sdesc_sw128(sK + kk * 2048, C::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
+          umma_commit(bar_dq_full);
+        }
+        __syncwarp();
         return true;
       };
 
@@ -502,8 +521,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && i + 1 < NIT) ok = mma_dp(i + 1) && mma_dv(i + 1);
         if (ok && i + 2 < NIT) ok = mma_s(i + 2);
       }
-      if (ok) umma_commit(bar_fin);
-      else record_failure(s_abort, p.err, SITE_BWD_MMA);
+      if (ok) {
+        if (elect_one()) umma_commit(bar_fin);
+        __syncwarp();
+      } else if (lane == 0) {
+        record_failure(s_abort, p.err, SITE_BWD_MMA);
+      }
     }
   }
   } else if (warp >= kWarpCompute0) {
@@ -808,9 +831,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = max(0, issued_o - C::NSO); it < issued_o; ++it)
       drain_wait(&bar_o_full[it % C::NSO], (it / C::NSO) & 1);
   }
-  if (warp == kWarpMma && lane == 0 && NIT > 0) {
-    umma_commit(bar_drain);
-    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  if (warp == kWarpMma && NIT > 0) {  // the lane that issued the products commits
+    if (elect_one()) {
+      umma_commit(bar_drain);
+      if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -273,10 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0 && G > 0) {
+    if (G > 0) {  // the whole warp walks the schedule and waits; one elected lane issues
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
-      auto wt = [&](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, s_abort, p.wait_ns); };
+      auto wt = [&](uint64_t* bar, uint32_t parity) { return warp_wait(bar, parity, s_abort, p.wait_ns); };
       // S_b(g) = Q_b K_g^T into tile b's score buffer; S_b(g) overwrites
       // P_b(g-1), so it waits for PV_b(g-1) to complete.
       auto issue_s = [&](int b, int g) -> bool {
@@ -284,16 +284,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (b == 0 && !wt(&bar_k_full[st], (g / C::NSK) & 1)) return false;
         if (g > 0 && !wt(&bar_o_done[b], (g - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t sQa = smem_u32(sQ + b * C::TILE);
-        const uint32_t sKa = smem_u32(sK + st * C::TILE);
+        if (elect_one()) {
+          const uint32_t sQa = smem_u32(sQ + b * C::TILE);
+          const uint32_t sKa = smem_u32(sK + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          umma_ss(tmem + b * 128, sdesc_sw128(sQa + off, 16, 1024), sdesc_sw128(sKa + off, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+            umma_ss(tmem + b * 128, sdesc_sw128(sQa + off, 16, 1024), sdesc_sw128(sKa + off, 16, 1024), idesc_s,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_s_full[b]);
+          if (b == (two ? 1 : 0)) umma_commit(&bar_k_empty[st]);  // S0(g), S1(g) were K_g's readers
         }
-        umma_commit(&bar_s_full[b]);
-        if (b == (two ? 1 : 0)) umma_commit(&bar_k_empty[st]);  // S0(g), S1(g) were K_g's readers
+        __syncwarp();
         return true;
       };
       // O_b += P_b(g) V_g with P_b read from the first 64 columns of its buffer
@@ -302,18 +305,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wt(&bar_p_ready[b], g & 1)) return false;
         if (b == 0 && !wt(&bar_v_full[st], (g / C::NSV) & 1)) return false;
         tc_fence_after();
-        const uint32_t sVa = smem_u32(sV + st * C::TILE);
+        if (elect_one()) {
+          const uint32_t sVa = smem_u32(sV + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
-          const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
-          umma_ts(tmem + C::T_O + b * D, tmem + b * 128 + kk * 8, bd, idesc_o, (g > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
+            const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
+            umma_ts(tmem + C::T_O + b * D, tmem + b * 128 + kk * 8, bd, idesc_o, (g > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar_o_done[b]);
+          if (b == (two ? 1 : 0)) umma_commit(&bar_v_empty[st]);  // PV0(g), PV1(g) were V_g's readers
         }
-        umma_commit(&bar_o_done[b]);
-        if (b == (two ? 1 : 0)) umma_commit(&bar_v_empty[st]);  // PV0(g), PV1(g) were V_g's readers
+        __syncwarp();
         return true;
       };
-      bool ok = mbar_wait(bar_q_full, 0, s_abort, p.wait_ns);
+      bool ok = warp_wait(bar_q_full, 0, s_abort, p.wait_ns);
       ok = ok && issue_s(0, 0) && (!two || issue_s(1, 0));
       for (int g = 0; g < G && ok; ++g) {
         ok = issue_pv(0, g);
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && g + 1 < G) ok = issue_s(1, g + 1);
         }
       }
-      if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
+      if (!ok && lane == 0) record_failure(s_abort, p.err, SITE_FWD_MMA);
     }
   }
   } else if (warp >= 8 && !two) {
@@ -552,9 +558,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = max(0, issued_v - C::NSV); g < issued_v; ++g)
       drain_wait(&bar_v_full[g % C::NSV], (g / C::NSV) & 1);
   }
-  if (warp == 1 && lane == 0 && G > 0) {
-    umma_commit(bar_drain);
-    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  if (warp == 1 && G > 0) {  // the lane that issued the products commits
+    if (elect_one()) {
+      umma_commit(bar_drain);
+      if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

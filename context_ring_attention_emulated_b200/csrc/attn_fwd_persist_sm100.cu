@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0) {
+    {  // the whole warp walks the schedule and waits; one elected lane issues
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t sQa = smem_u32(sQ);
@@ -349,57 +349,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keep a later MMA's accumulator writes behind an earlier MMA's TMEM
       // operand reads.
       auto issue_s = [&](int gg) -> bool {
-        if (gg >= C::NSB && !mbar_wait(&bar_o_done[(gg - C::NSB) % C::NSB], ((gg - C::NSB) / C::NSB) & 1, s_abort,
+        if (gg >= C::NSB && !warp_wait(&bar_o_done[(gg - C::NSB) % C::NSB], ((gg - C::NSB) / C::NSB) & 1, s_abort,
                                        p.wait_ns))
           return false;
         const int st = gg % C::NS;
-        if (!mbar_wait(&bar_k_full[st], (gg / C::NS) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_k_full[st], (gg / C::NS) & 1, s_abort, p.wait_ns)) return false;
+        mma_issued = true;  // every lane: the teardown drain is taken by the whole warp
         tc_fence_after();
-        const uint32_t d_s = tmem + (gg % C::NSB) * 128;
-        const uint32_t sKa = smem_u32(sK + st * C::TILE);
+        if (elect_one()) {
+          const uint32_t d_s = tmem + (gg % C::NSB) * 128;
+          const uint32_t sKa = smem_u32(sK + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(sQa + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + off, 16, 1024);
-          umma_ss(d_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+            const uint64_t ad = sdesc_sw128(sQa + off, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sKa + off, 16, 1024);
+            umma_ss(d_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_s_full[gg % C::NSB]);
+          umma_commit(&bar_k_empty[st]);
         }
-        umma_commit(&bar_s_full[gg % C::NSB]);
-        umma_commit(&bar_k_empty[st]);
-        mma_issued = true;
+        __syncwarp();
         return true;
       };
       // O (+)= P_j V_j with P_j read from the first 64 columns of its score
       // buffer; the item's first product overwrites O.
       auto issue_pv = [&](int gg, bool first) -> bool {
-        if (!mbar_wait(&bar_p_ready[gg % C::NSB], (gg / C::NSB) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_p_ready[gg % C::NSB], (gg / C::NSB) & 1, s_abort, p.wait_ns)) return false;
         const int st = gg % C::NS;
-        if (!mbar_wait(&bar_v_full[st], (gg / C::NS) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_v_full[st], (gg / C::NS) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t a_t = tmem + (gg % C::NSB) * 128;
-        const uint32_t sVa = smem_u32(sV + st * C::TILE);
+        if (elect_one()) {
+          const uint32_t a_t = tmem + (gg % C::NSB) * 128;
+          const uint32_t sVa = smem_u32(sV + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
-          const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
-          umma_ts(tmem + C::T_O, a_t + kk * 8, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
+            const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
+            umma_ts(tmem + C::T_O, a_t + kk * 8, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar_o_done[gg % C::NSB]);
+          umma_commit(&bar_v_empty[st]);
         }
-        umma_commit(&bar_o_done[gg % C::NSB]);
-        umma_commit(&bar_v_empty[st]);
+        __syncwarp();
         return true;
       };
 
       for (int k = 0; ok; ++k) {
         const int slot = k % NSLOT;
-        if (!mbar_wait(&bar_item_full[slot], (k / NSLOT) & 1, s_abort, p.wait_ns)) {
+        if (!warp_wait(&bar_item_full[slot], (k / NSLOT) & 1, s_abort, p.wait_ns)) {
           ok = false;
           break;
         }
         const int G = s_item[slot].w;
-        mbar_arrive(&bar_item_empty[slot]);  // only G is read here
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_item_empty[slot]);  // only G is read here
         if (G < 0) break;
         if (G == 0) continue;
-        if (!mbar_wait(bar_q_full, n_live & 1, s_abort, p.wait_ns)) {
+        if (!warp_wait(bar_q_full, n_live & 1, s_abort, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -408,19 +415,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The item's first scores run while the previous item's last tiles
         // and epilogue are still in the softmax warps.
         for (int x = 0; x < min(G, C::NSB) && ok; ++x) ok = issue_s(g0 + x);
-        if (ok && G <= C::NSB) umma_commit(bar_q_empty);
-        if (ok && n_live > 0) ok = mbar_wait(bar_o_free, (n_live - 1) & 1, s_abort, p.wait_ns);
+        if (ok && G <= C::NSB) {
+          if (elect_one()) umma_commit(bar_q_empty);
+          __syncwarp();
+        }
+        if (ok && n_live > 0) ok = warp_wait(bar_o_free, (n_live - 1) & 1, s_abort, p.wait_ns);
         for (int x = 0; x < G && ok; ++x) {
           ok = issue_pv(g0 + x, x == 0);
           if (ok && x + C::NSB < G) {
             ok = issue_s(g0 + x + C::NSB);
-            if (ok && x + C::NSB == G - 1) umma_commit(bar_q_empty);
+            if (ok && x + C::NSB == G - 1) {
+              if (elect_one()) umma_commit(bar_q_empty);
+              __syncwarp();
+            }
           }
         }
         g = g0 + G;
         ++n_live;
       }
-      if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
+      if (!ok && lane == 0) record_failure(s_abort, p.err, SITE_FWD_MMA);
     }
   } else {
     // -------------------------------------------------- softmax + epilogue
@@ -648,9 +661,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = max(0, issued_k - C::NS); g < issued_k; ++g) drain_wait(&bar_k_full[g % C::NS], (g / C::NS) & 1);
     for (int g = max(0, issued_v - C::NS); g < issued_v; ++g) drain_wait(&bar_v_full[g % C::NS], (g / C::NS) & 1);
   }
-  if (warp == 1 && lane == 0 && mma_issued) {
-    umma_commit(bar_drain);
-    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  if (warp == 1 && mma_issued) {  // the lane that issued the products commits
+    if (elect_one()) {
+      umma_commit(bar_drain);
+      if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

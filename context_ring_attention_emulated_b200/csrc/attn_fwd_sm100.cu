@@ -239,47 +239,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0 && G > 0) {
+    if (G > 0) {  // the whole warp walks the schedule and waits; one elected lane issues
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t sQa = smem_u32(sQ);
-      bool ok = mbar_wait(bar_q_full, 0, s_abort, p.wait_ns);
-      if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
-
+      bool ok = warp_wait(bar_q_full, 0, s_abort, p.wait_ns);
       // S_g = Q K_g^T into score buffer g % NSB
       auto issue_s = [&](int g) -> bool {
         const int st = g % C::NS;
-        if (!mbar_wait(&bar_k_full[st], (g / C::NS) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_k_full[st], (g / C::NS) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t d_s = tmem + (g % C::NSB) * 128;
-        const uint32_t sKa = smem_u32(sK + st * C::TILE);
+        if (elect_one()) {
+          const uint32_t d_s = tmem + (g % C::NSB) * 128;
+          const uint32_t sKa = smem_u32(sK + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(sQa + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + off, 16, 1024);
-          umma_ss(d_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+            const uint64_t ad = sdesc_sw128(sQa + off, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sKa + off, 16, 1024);
+            umma_ss(d_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_s_full[g % C::NSB]);
+          umma_commit(&bar_k_empty[st]);
         }
-        umma_commit(&bar_s_full[g % C::NSB]);
-        umma_commit(&bar_k_empty[st]);
+        __syncwarp();
         return true;
       };
       // O += P_j V_j with P_j read from the first 64 columns of its score buffer
       auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&bar_p_ready[j % C::NSB], (j / C::NSB) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_p_ready[j % C::NSB], (j / C::NSB) & 1, s_abort, p.wait_ns)) return false;
         const int st = j % C::NS;
-        if (!mbar_wait(&bar_v_full[st], (j / C::NS) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_v_full[st], (j / C::NS) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t a_t = tmem + (j % C::NSB) * 128;
-        const uint32_t sVa = smem_u32(sV + st * C::TILE);
+        if (elect_one()) {
+          const uint32_t a_t = tmem + (j % C::NSB) * 128;
+          const uint32_t sVa = smem_u32(sV + st * C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
-          const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
-          umma_ts(tmem + C::T_O, a_t + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // V tile as an MN-major B operand: 16 keys = two 8-row swizzle atoms.
+            const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::BOX, 1024);
+            umma_ts(tmem + C::T_O, a_t + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar_o_done[j % C::NSB]);
+          umma_commit(&bar_v_empty[st]);
         }
-        umma_commit(&bar_o_done[j % C::NSB]);
-        umma_commit(&bar_v_empty[st]);
+        __syncwarp();
         return true;
       };
 
@@ -291,12 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < G && ok; ++g) {
         ok = issue_pv(g);
         if (ok && g + C::NSB < G) {
-          ok = mbar_wait(&bar_o_done[g % C::NSB], (g / C::NSB) & 1, s_abort, p.wait_ns);
+          ok = warp_wait(&bar_o_done[g % C::NSB], (g / C::NSB) & 1, s_abort, p.wait_ns);
           if (ok) ok = issue_s(g + C::NSB);
         }
       }
-      if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
-
+      if (!ok && lane == 0) record_failure(s_abort, p.err, SITE_FWD_MMA);
     }
   } else {
     // -------------------------------------------------- softmax + epilogue
@@ -499,9 +502,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = max(0, issued_k - C::NS); g < issued_k; ++g) drain_wait(&bar_k_full[g % C::NS], (g / C::NS) & 1);
     for (int g = max(0, issued_v - C::NS); g < issued_v; ++g) drain_wait(&bar_v_full[g % C::NS], (g / C::NS) & 1);
   }
-  if (warp == 1 && lane == 0 && G > 0) {
-    umma_commit(bar_drain);
-    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  if (warp == 1 && G > 0) {  // the lane that issued the products commits
+    if (elect_one()) {
+      umma_commit(bar_drain);
+      if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

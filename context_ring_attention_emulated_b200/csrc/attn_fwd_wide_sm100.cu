@@ -23,7 +23,8 @@
 //               V tile (256 x D) into its one stage one tile behind the K
 //               loads (so a K load never queues behind a V stage that frees
 //               late);
-//   warp 9      TMEM allocation and tcgen05.mma from one thread, in the order
+//   warp 9      TMEM allocation and tcgen05.mma (the whole warp waits, one
+//               lane chosen by elect.sync issues), in the order
 //               S_{g+1} (once the scores S_g are read), PV_g (once P_g is in
 //               TMEM);
 //   warps 0..7  softmax, two warps per TMEM lane quarter: warp half h takes
@@ -251,51 +252,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 9) {
     // ----------------------------------------------------------- MMA issue
-    if (lane == 0 && G > 0) {
+    // The whole warp walks the schedule and waits; one elected lane issues.
+    if (G > 0) {
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, 0, 0);
       const uint32_t idesc_o = idesc_bf16_f32(BM, D, 0, 1);
-      const uint32_t sQa = smem_u32(sQ);
-      bool ok = mbar_wait(bar_q_full, 0, s_abort, p.wait_ns);
+      const uint32_t sQa = smem_u32(sQ), sKa0 = smem_u32(sK), sVa = smem_u32(sV);
+      bool ok = warp_wait(bar_q_full, 0, s_abort, p.wait_ns);
       // S_g = Q K_g^T: 128 x 256 into the score buffer
       auto issue_s = [&](int g) -> bool {
         const int st = g % C::NSK;
-        if (!mbar_wait(&bar_k_full[st], (g / C::NSK) & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(&bar_k_full[st], (g / C::NSK) & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t sKa = smem_u32(sK + st * C::KTILE);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sQa + (kk >> 2) * C::QBOX + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sKa + (kk >> 2) * C::KBOX + (kk & 3) * 32, 16, 1024);
-          umma_ss(tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sQa + (kk >> 2) * C::QBOX + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sKa0 + st * C::KTILE + (kk >> 2) * C::KBOX + (kk & 3) * 32, 16, 1024);
+            umma_ss(tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_s_full);
+          umma_commit(&bar_k_empty[st]);
         }
-        umma_commit(bar_s_full);
-        umma_commit(&bar_k_empty[st]);
+        __syncwarp();
         return true;
       };
       // O += P_g V_g, P_g (bf16, 256 keys) from the P buffer, V_g MN-major
       auto issue_pv = [&](int g) -> bool {
-        if (!mbar_wait(bar_p_ready, g & 1, s_abort, p.wait_ns)) return false;
-        if (!mbar_wait(bar_v_full, g & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(bar_p_ready, g & 1, s_abort, p.wait_ns)) return false;
+        if (!warp_wait(bar_v_full, g & 1, s_abort, p.wait_ns)) return false;
         tc_fence_after();
-        const uint32_t sVa = smem_u32(sV);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(sVa + kk * 2048, C::KBOX, 1024);
-          umma_ts(tmem + C::T_O, tmem + C::T_P + kk * 8, bd, idesc_o, (g > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts(tmem + C::T_O, tmem + C::T_P + kk * 8, sdesc_sw128(sVa + kk * 2048, C::KBOX, 1024), idesc_o,
+                    (g > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar_o_done);
+          umma_commit(bar_v_empty);
         }
-        umma_commit(bar_o_done);
-        umma_commit(bar_v_empty);
+        __syncwarp();
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int g = 0; g < G && ok; ++g) {
         if (g + 1 < G) {  // S_{g+1} as soon as the softmax warps hold S_g
-          ok = mbar_wait(bar_s_free, g & 1, s_abort, p.wait_ns) && issue_s(g + 1);
+          ok = warp_wait(bar_s_free, g & 1, s_abort, p.wait_ns) && issue_s(g + 1);
           if (!ok) break;
         }
         ok = issue_pv(g);
       }
-      if (!ok) record_failure(s_abort, p.err, SITE_FWD_MMA);
+      if (!ok && lane == 0) record_failure(s_abort, p.err, SITE_FWD_MMA);
     }
   }
   } else {
@@ -535,9 +540,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(&bar_k_full[g % C::NSK], (g / C::NSK) & 1);
     if (issued_v > 0) drain_wait(bar_v_full, (issued_v - 1) & 1);
   }
-  if (warp == 9 && lane == 0 && G > 0) {
-    umma_commit(bar_drain);
-    if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+  if (warp == 9 && G > 0) {  // the lane that issued the products commits
+    if (elect_one()) {
+      umma_commit(bar_drain);
+      if (!drain_wait(bar_drain, 0)) record_failure(s_abort, p.err, SITE_DRAIN);
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

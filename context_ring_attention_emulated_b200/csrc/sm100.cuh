@@ -343,6 +343,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// One lane of a converged warp (the same lane every time for a full warp) is
+// elected to issue tcgen05 operations; the rest of the warp stays on the same
+// path, so the operands stay warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p = 0;
+  asm volatile("{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}" : "=r"(p));
+  return p != 0;
+}
+
+// Shared-memory descriptor advanced by a byte offset (the start-address field
+// holds address / 16 in 14 bits; every operand here lies below 256 KB).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t offset_bytes) {
+  return desc + static_cast<uint64_t>(offset_bytes >> 4);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T   (one K=16 step)
 __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                         uint32_t accumulate) {
