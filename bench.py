@@ -41,11 +41,11 @@ VARLEN_ALIGN = 128
 # capture (dram__bytes_read.sum + dram__bytes_write.sum) of the kernel as it
 # stands, taken on a smaller case and scaled to the workload's launch by the
 # sequence length. Empty while the kernel has changed since its last capture.
-# The ring backward at B=1 H=32 L=16000 D=128 cp=4: 792,195,072 B read +
-# 478,162,176 B written, x2 for L=32000; algorithmic 2,621,440,000 B (Q, K, V,
+# The ring backward at B=1 H=32 L=16000 D=128 cp=4: 791,380,480 B read +
+# 477,255,936 B written, x2 for L=32000; algorithmic 2,621,440,000 B (Q, K, V,
 # dO read, the fp32 dQ accumulator read and written, dK and dV written).
-NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": {"bytes": 2 * (792195072 + 478162176),
-                                          "ratio": 2 * (792195072 + 478162176) / 2621440000}}
+NCU_TRAFFIC = {"bf16_L32000_cp4_fwdbwd": {"bytes": 2 * (791380480 + 477255936),
+                                          "ratio": 2 * (791380480 + 477255936) / 2621440000}}
 # Dense bf16 tensor rate of one SM: a 128x128x16 MMA every 64 cycles.
 SM_COUNT = 148
 TENSOR_FLOP_PER_CLK_SM = 8192

@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             s_full[st] = full ? 1 : 0;
           }
           __syncwarp();
-          if (lane == 0) {
+          if (elect_one()) {
             mbar_arrive_expect_tx(&bar_q_full[st], C::TILE);
             for (int b = 0; b < C::NBOX; ++b)
               tma_load_4d(smem + C::OFF_Q + st * C::TILE + b * C::BOX, &tm_q, &bar_q_full[st], b * 64, i * BQ, r,
@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (lane == 0) {
+          if (elect_one()) {
             mbar_arrive_expect_tx(&bar_o_full[so], C::TILE);
             for (int b = 0; b < C::NBOX; ++b)
               tma_load_4d(smem + C::OFF_DO + so * C::TILE + b * C::BOX, &tm_do, &bar_o_full[so], b * 64, i * BQ,
@@ -423,22 +423,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_t = idesc_bf16_f32(BK, BQ, 0, 0);  // S^T, dP^T: K-major A and B
       const uint32_t idesc_g = idesc_bf16_f32(BK, D, 0, 1);   // dV, dK: A in TMEM, B MN-major
       const uint32_t idesc_q = idesc_bf16_f32(BQ, D, 1, 1);   // dQ: A (dS) and B (K) MN-major
-      const uint32_t sK = smem_u32(smem + C::OFF_K);
-      const uint32_t sV = smem_u32(smem + C::OFF_V);
-      const uint32_t sDS = smem_u32(smem + C::OFF_DS);
-      auto sQ = [&](int j) { return smem_u32(smem + C::OFF_Q + (j % C::NSQ) * C::TILE); };
-      auto sDO = [&](int j) { return smem_u32(smem + C::OFF_DO + (j % C::NSO) * C::TILE); };
+      // Operand descriptors as one base descriptor per layout plus byte offsets.
+      const uint64_t dk_s = sdesc_sw128(smem_u32(smem), 16, 1024);      // K-major tiles
+      const uint64_t dmn = sdesc_sw128(smem_u32(smem), C::BOX, 1024);   // MN-major tiles
+      auto oQ = [&](int j) { return static_cast<uint32_t>(C::OFF_Q + (j % C::NSQ) * C::TILE); };
+      auto oDO = [&](int j) { return static_cast<uint32_t>(C::OFF_DO + (j % C::NSO) * C::TILE); };
       auto wt = [&](uint64_t* bar, uint32_t parity) { return warp_wait(bar, parity, s_abort, p.wait_ns); };
 
       auto mma_s = [&](int j) -> bool {
         if (!wt(&bar_q_full[j % C::NSQ], (j / C::NSQ) & 1)) return false;
         tc_fence_after();
         if (elect_one()) {
-          const uint32_t q = sQ(j);
+          const uint32_t q = oQ(j);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-            umma_ss(tmem + C::T_S, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(q + off, 16, 1024), idesc_t,
+            umma_ss(tmem + C::T_S, sdesc_add(dk_s, C::OFF_K + off), sdesc_add(dk_s, q + off), idesc_t,
                     kk > 0 ? 1u : 0u);
           }
           umma_commit(bar_s_full);
@@ -455,11 +455,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         if (elect_one()) {
-          const uint32_t o = sDO(j);
+          const uint32_t o = oDO(j);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-            umma_ss(tmem + C::T_DP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(o + off, 16, 1024), idesc_t,
+            umma_ss(tmem + C::T_DP, sdesc_add(dk_s, C::OFF_V + off), sdesc_add(dk_s, o + off), idesc_t,
                     kk > 0 ? 1u : 0u);
           }
           umma_commit(bar_dp_full);
@@ -473,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wt(&bar_o_full[j % C::NSO], (j / C::NSO) & 1)) return false;
         tc_fence_after();
         if (elect_one()) {
-          const uint32_t o = sDO(j);
+          const uint32_t o = oDO(j);
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk) {
             const uint32_t a_col = C::T_S + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s P^T
-            umma_ts(tmem + C::T_DV, tmem + a_col, sdesc_sw128(o + kk * 2048, C::BOX, 1024), idesc_g,
+            umma_ts(tmem + C::T_DV, tmem + a_col, sdesc_add(dmn, o + kk * 2048), idesc_g,
                     (j > 0 || kk > 0) ? 1u : 0u);
           }
           if (j > 0) umma_commit(&bar_o_empty[j % C::NSO]);  // dP(j) was issued before dV(j)
@@ -489,11 +489,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wt(bar_ds_ready, j & 1)) return false;
         tc_fence_after();
         if (elect_one()) {
-          const uint32_t q = sQ(j);
+          const uint32_t q = oQ(j);
 #pragma unroll
           for (int kk = 0; kk < BQ / 16; ++kk) {
             const uint32_t a_col = C::T_DP + (kk >> 2) * 64 + (kk & 3) * 8;  // warpgroup (kk >> 2)'s dS^T
-            umma_ts(tmem + C::T_DK, tmem + a_col, sdesc_sw128(q + kk * 2048, C::BOX, 1024), idesc_g,
+            umma_ts(tmem + C::T_DK, tmem + a_col, sdesc_add(dmn, q + kk * 2048), idesc_g,
                     (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bar_q_empty[j % C::NSQ]);  // S(j) and dK(j) were Q's readers
@@ -506,8 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma_ss(tmem + C::T_DP, sdesc_sw128(sDS + kk * 2048, C::BOX, 1024),
-                    sdesc_sw128(sK + kk * 2048, C::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
+            umma_ss(tmem + C::T_DP, sdesc_add(dmn, C::OFF_DS + kk * 2048), sdesc_add(dmn, C::OFF_K + kk * 2048),
+                    idesc_q, kk > 0 ? 1u : 0u);
           umma_commit(bar_dq_full);
         }
         __syncwarp();

@@ -9,9 +9,9 @@
 // max grows, so the result equals full softmax attention. Tiles that the
 // causal position relation fully masks are skipped.
 //
-// Why 256-key tiles: an M = 128 x N = 128 tcgen05.mma stream reaches only about
-// half the tensor rate of an N = 256 one, so the score product S = Q K^T is
-// issued with N = 256 (256 keys at once). The TMEM plan keeps one 256-column
+// Why 256-key tiles: the score product S = Q K^T is issued as N = 256 MMAs
+// (256 keys at once), half as many instructions per FLOP as N = 128, which
+// leaves the issuing warp more slack per product. The TMEM plan keeps one 256-column
 // score buffer, a separate 128-column buffer for P (bf16, 256 keys packed two
 // per column) and O: S [0,256) P [256,384) O [384,512). Because P does not
 // overwrite the scores, the next tile's score product may start as soon as the
