@@ -29,12 +29,15 @@
 //               TMEM);
 //   warps 0..7  softmax, two warps per TMEM lane quarter: warp half h takes
 //               keys [128 h, 128 h + 128) of every tile and output columns
-//               [h D/2, (h+1) D/2). The two halves' row maxima are combined
-//               once per tile through shared memory at a named barrier of the
-//               pair (both leave together on any failure, so neither can be
-//               left waiting); row sums are added once at the end. P_g is
-//               written only after PV_{g-1}, the last reader of the P buffer,
-//               has completed.
+//               [h D/2, (h+1) D/2). P_g is first formed against the reference
+//               max kept so far, without a row max; the two warps of a pair
+//               then meet at a named barrier (bar.red.or) and, only if a row
+//               of either half needs a new reference (its first visible keys,
+//               or a half-row sum above 2^16), combine their row maxima through
+//               shared memory, rescale lazily and form P_g again. Both leave
+//               together on any failure, so neither can be left waiting; row
+//               sums are added once at the end. P_g is written only after
+//               PV_{g-1}, the last reader of the P buffer, has completed.
 //   warps 10-11 idle (they complete the producer / MMA warpgroup, whose
 //               registers go to the softmax warpgroups by setmaxnreg).
 #include <limits.h>
@@ -368,7 +371,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const bool got = !bad && warp_wait(bar_s_full, g & 1, s_abort, p.wait_ns);
         uint32_t sr[4][32];
-        float pm = -INFINITY;
+        uint32_t pk[4][16];                           // P_g, bf16 pairs
+        uint64_t sum4[4] = {0ull, 0ull, 0ull, 0ull};  // its eight partial row sums
+        // P_g against the reference max m (0 while a row has none): exponent
+        // arguments and row sums two keys at a time (f32x2).
+        auto form_p = [&](float m) {
+          const uint64_t sl2x2 = f32x2(sl2, sl2), nm2 = f32x2(-m, -m);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sum4[i] = 0ull;
+#pragma unroll
+          for (int h = 0; h < 4; ++h)  // 32 keys (16 packed columns) at a time
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 t = f32x2_split(
+                  fma_f32x2(f32x2(__uint_as_float(sr[h][2 * i]), __uint_as_float(sr[h][2 * i + 1])), sl2x2, nm2));
+              const float a = ex2_approx(t.x), b = ex2_approx(t.y);
+              sum4[i & 3] = add_f32x2(sum4[i & 3], f32x2(a, b));
+              pk[h][i] = pack_bf16x2(a, b);
+            }
+        };
+        bool full = true;  // the full path: row max, exchange, lazy rescale
         if (got) {
           tc_fence_after();
 #pragma unroll
@@ -384,77 +406,80 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 32; ++i)
                 if (c * 32 + i < klo || c * 32 + i >= khi) sr[c][i] = __float_as_uint(-INFINITY);
           }
-          float mx8[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; i += 2)
-              mx8[(i >> 1) & 7] =
-                  fmax3(mx8[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
-          pm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                     fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          // Short path: P_g against the reference max kept so far, with no row
+          // max. It stands unless a row of the quarter needs a new reference:
+          // its first visible keys, or a half-row sum above 2^16 (some score
+          // more than 9 above the reference, log2 units), where the full path
+          // below takes over. Values below 2^16 keep the fp32 sums and the
+          // bf16 P far from overflow; the result is exact either way.
+          form_p(m_run == -INFINITY ? 0.f : m_run);
+          const float2 s01 = f32x2_split(add_f32x2(sum4[0], sum4[1]));
+          const float2 s23 = f32x2_split(add_f32x2(sum4[2], sum4[3]));
+          const float lt = (s01.x + s01.y) + (s23.x + s23.y);
+          full = (m_run == -INFINITY && klo < khi) || !(lt <= 65536.f);
         }
-        // Hand over the partial max; both warps meet once per tile and leave
-        // together on any failure.
-        s_xch[((g & 1) * 2 + half) * BM + row] = pm;
-        if (bar_any(meet, 64, !got)) {
-          record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
-          ok = false;
-          break;
-        }
-        // max is exact and commutative: both halves hold the same value
-        float mx = fmaxf(pm, s_xch[((g & 1) * 2 + (half ^ 1)) * BM + row]);
-        mx *= sl2;
-        // Lazy rescale: keep the reference max unless the row max grew by > 8
-        // (log2 units), so exp2 values stay <= 256; exact either way.
-        const bool need = mx > m_run + 8.f;
-        float alpha = 1.f;
-        const bool o_live = (g > 0) && (m_run != -INFINITY);
-        if (need) {
-          alpha = ex2_approx(m_run - mx);
-          l_run *= alpha;
-        }
-        const bool warp_rescale = __any_sync(0xffffffffu, need && o_live) != 0;
-        if (need) m_run = mx;
-        // PV_{g-1} must be complete before O is rescaled and before P_g is
-        // written over P_{g-1} (the exps below are formed in registers first).
-        bool pv_prev_done = g == 0;
-        if (warp_rescale) {
-          if (!warp_wait(bar_o_done, (g - 1) & 1, s_abort, p.wait_ns)) {
+        bool pv_prev_done = g == 0;  // PV_{g-1}, the last reader of the P buffer, has completed
+        // Both warps of the quarter meet here once per tile; any failed wait
+        // also sends both into the full path, whose meeting reports it.
+        if (bar_any(meet, 64, full)) {
+          float pm = -INFINITY;
+          if (got) {
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+              for (int i = 0; i < 32; i += 2)
+                mx8[(i >> 1) & 7] =
+                    fmax3(mx8[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+            pm = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          }
+          // Hand over the partial max; both warps leave together on any failure.
+          s_xch[((g & 1) * 2 + half) * BM + row] = pm;
+          if (bar_any(meet, 64, !got)) {
             record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
-            bad = true;
-            continue;
+            ok = false;
+            break;
           }
-          pv_prev_done = true;
-          tc_fence_after();
-          const uint32_t o_addr = tmem + lane_base + C::T_O + half * (D / 2);
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(o_addr + c * 32, orr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-            tmem_st32(o_addr + c * 32, orr);
+          // max is exact and commutative: both halves hold the same value
+          float mx = fmaxf(pm, s_xch[((g & 1) * 2 + (half ^ 1)) * BM + row]);
+          mx *= sl2;
+          // Lazy rescale: keep the reference max unless the row max grew by > 8
+          // (log2 units); exact either way.
+          const bool need = mx > m_run + 8.f;
+          float alpha = 1.f;
+          const bool o_live = (g > 0) && (m_run != -INFINITY);
+          if (need) {
+            alpha = ex2_approx(m_run - mx);
+            l_run *= alpha;
           }
+          const bool warp_rescale = __any_sync(0xffffffffu, need && o_live) != 0;
+          if (need) m_run = mx;
+          // PV_{g-1} must be complete before O is rescaled.
+          if (warp_rescale) {
+            if (!warp_wait(bar_o_done, (g - 1) & 1, s_abort, p.wait_ns)) {
+              record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
+              bad = true;
+              continue;
+            }
+            pv_prev_done = true;
+            tc_fence_after();
+            const uint32_t o_addr = tmem + lane_base + C::T_O + half * (D / 2);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(o_addr + c * 32, orr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+              tmem_st32(o_addr + c * 32, orr);
+            }
+          }
+          form_p(m_run == -INFINITY ? 0.f : m_run);
         }
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float sum8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
         const uint32_t p_addr = tmem + lane_base + C::T_P + half * 64;
-        uint32_t pk[4][16];
-#pragma unroll
-        for (int h = 0; h < 4; ++h)  // 32 keys (16 packed columns) at a time
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a = ex2_approx(fmaf(__uint_as_float(sr[h][2 * i]), sl2, -m_use));
-            const float b = ex2_approx(fmaf(__uint_as_float(sr[h][2 * i + 1]), sl2, -m_use));
-            sum8[i & 7] += a + b;
-            pk[h][i] = pack_bf16x2(a, b);
-          }
         if (!pv_prev_done) {
           if (!warp_wait(bar_o_done, (g - 1) & 1, s_abort, p.wait_ns)) {
             record_failure(s_abort, p.err, SITE_FWD_SOFTMAX);
@@ -465,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int h = 0; h < 4; ++h) tmem_st16(p_addr + h * 16, pk[h]);
-        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        const float2 s01 = f32x2_split(add_f32x2(sum4[0], sum4[1])), s23 = f32x2_split(add_f32x2(sum4[2], sum4[3]));
+        l_run += (s01.x + s01.y) + (s23.x + s23.y);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
