@@ -91,6 +91,49 @@ def test_ring_fwd_tilings_agree_and_match_oracle(rattn, case):
     check_lse(lse.cpu().numpy()[..., real], l_ref_p[..., 0][..., real], torch.bfloat16)
 
 
+GROWING = [
+    # L, cp, layout, causal, drift of the scores along the keys (natural-log units)
+    (4096, 2, 1, True, 60.0),
+    (4096, 4, 0, False, 60.0),
+    (4096, 2, 1, True, -60.0),
+    (3000, 3, 2, True, 90.0),
+]
+
+
+@pytest.mark.parametrize("case", GROWING)
+def test_ring_fwd_scores_that_drift(rattn, case):
+    """Scores rising (or falling) by tens of natural-log units along the keys
+    (q ~ 1, k_j ~ t_j / sqrt(D), so q.k_j scale ~ t_j): a row's running max
+    moves many times across its tiles, which exercises every form's lazy
+    rescale and the 256-key form's short path handing over to its full path.
+    All forms against the oracle, the 256-key one (the default) included."""
+    L, cp, layout, causal, drift = case
+    B, H, D = 1, 2, 128
+    scale = D ** -0.5
+    t = drift * torch.arange(L, dtype=torch.float32, device="cuda") / L
+    q = (1.0 + 0.05 * make_tensor((B, H, L, D), torch.float32, "cuda", seed=101)).to(torch.bfloat16)
+    k = (t[None, None, :, None] * scale + 0.05 * make_tensor((B, H, L, D), torch.float32, "cuda", seed=102))
+    k = k.to(torch.bfloat16)
+    v = make_tensor((B, H, L, D), torch.bfloat16, "cuda", seed=103)
+    qp, pos = rattn.cp_layout_permute(q, cp, layout)
+    kp, _ = rattn.cp_layout_permute(k, cp, layout)
+    vp, _ = rattn.cp_layout_permute(v, cp, layout)
+    run = lambda: rattn.rattn_ring_fwd(qp, kp, vp, pos, cp, layout, causal, scale, L_valid=L)
+    _all_forms(rattn, run)
+    o_ref, l_ref = oracle.attention(to64(q), to64(k), to64(v), scale, causal)
+    l_ref_p, _ = oracle.permute(l_ref[..., None], cp, layout)
+    real = pos.cpu().numpy() < L
+    for mode in (1, 4):
+        rattn.rattn_set_fwd_tiling(mode)
+        o, lse = run()
+        torch.cuda.synchronize()
+        rattn.rattn_set_fwd_tiling(0)
+        assert rattn.rattn_get_device_error()[0] == rattn.OK
+        out = rattn.cp_layout_unpermute(o, L, cp, layout)
+        check_o(out.float().cpu().numpy(), o_ref, torch.bfloat16)
+        check_lse(lse.cpu().numpy()[..., real], l_ref_p[..., 0][..., real], torch.bfloat16)
+
+
 def test_partial_fwd_tilings_agree(rattn):
     """One block with separate query and key positions, masked pad keys, and
     an empty key block."""
