@@ -63,11 +63,6 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Vector reduction into global memory (no value returned).
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 // Element idx (0..127) of a 128-entry array spread over a warp, four
 // consecutive entries per lane (lane l holds entries 4l..4l+3 in v[0..3]).
