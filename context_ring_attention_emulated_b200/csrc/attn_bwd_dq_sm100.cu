@@ -19,7 +19,7 @@
 // Warp roles (192 threads):
 //   warp 0      TMA producer: Q and dO once, then K (3 stages for D = 128)
 //               and V (2 stages) tiles of every visible key tile;
-//   warp 1      TMEM allocation and tcgen05.mma from one thread:
+//   warp 1      TMEM allocation and tcgen05.mma (the warp waits, one elected lane issues):
 //               S_g = Q K_g^T into one of two score buffers, dP_g = dO V_g^T,
 //               dQ += dS_g K_g with dS_g read from TMEM; S_{g+2} reuses the
 //               buffer once dQ_g (its reader) has completed, dP_{g+1} once the

@@ -19,7 +19,7 @@
 // traffic per FLOP of the one-tile kernel). Warp roles (384 threads):
 //   warp 0      TMA producer: Q0, Q1 once, then K (3 stages) and V (2
 //               stages for D = 128) through rings of shared-memory buffers;
-//   warp 1      TMEM allocation and tcgen05.mma issue from one thread, in
+//   warp 1      TMEM allocation and tcgen05.mma issue (one elected lane of the warp), in
 //               the order PV0(j), S0(j+1), PV1(j), S1(j+1): S_b = Q_b K^T
 //               into tile b's score buffer, O_b += P_b V with P_b read from
 //               TMEM; S_b(j+1) waits for PV_b(j), which reads P_b(j) there;

@@ -22,7 +22,7 @@
 //               MMA has read the old one), then K and V tiles through an
 //               NS-stage ring of shared-memory buffers (the emulated KV hop:
 //               the next block's loads run while the current block's MMAs do);
-//   warp 1      allocates TMEM and issues tcgen05.mma from one thread:
+//   warp 1      allocates TMEM and issues tcgen05.mma from one elected lane:
 //               S_g = Q K_g^T into one of three TMEM score buffers, running
 //               three tiles ahead of O += P_g V_g (P read from TMEM), so the
 //               score MMAs never wait on the previous tile's softmax; an

@@ -16,7 +16,7 @@
 //   warp 0      TMA producer: Q once, then K and V tiles through a
 //               NS-stage ring of shared-memory buffers (the emulated KV hop:
 //               the next block's loads run while the current block's MMAs do);
-//   warp 1      allocates TMEM and issues tcgen05.mma from one thread:
+//   warp 1      allocates TMEM and issues tcgen05.mma from one elected lane:
 //               S_g = Q K_g^T into one of three TMEM score buffers, running
 //               three tiles ahead of O += P_g V_g (P read from TMEM), so the
 //               score MMAs never wait on the previous tile's softmax;
